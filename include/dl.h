@@ -1,0 +1,211 @@
+/*
+ * dl.h -- C ABI of the B200 (sm_100a) library for one denoising step of
+ * sink-aware, query-predicted, block-sparse bidirectional attention over a
+ * cached long-context KV (diffusion LLM inference).
+ *
+ * Method sources (page title, then the part of the page):
+ *   [F1] "Focus-dLLM: Accelerating Long-Context Diffusion LLM Inference via
+ *        Confidence-Guided Context Focusing" -- abstract.
+ *   [F2] same paper -- research.elamur.ai summary and key points.
+ *   [P1] "Prefilling-dLLM: Predictive Prefilling for Long-Context Inference
+ *        in Diffusion Language Models" -- abstract.
+ *
+ * Conventions shared by every call
+ *   - Every pointer argument is caller-owned DEVICE memory unless stated.
+ *     The library allocates nothing; calls that need scratch take a
+ *     caller-provided workspace (size from dl_workspace_size).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL means the legacy default stream) and returns a dl_status.
+ *     Argument errors are reported before anything is launched; the message
+ *     is available from dl_last_error_message() on the calling thread.
+ *   - Out-of-range indices read from device memory (page-table slots, block
+ *     indices, token positions, sink positions) are detected by the kernels:
+ *     the offending tile is skipped and a device error word is set, which
+ *     dl_get_status() reports as DL_ERR_BAD_INDEX.  No kernel traps.
+ *   - Shapes: b = sequence, h = query head, g = KV head, G = H / H_kv query
+ *     heads per KV head, d = head dimension, L_q = decode-block length.
+ *   - scale = 1/sqrt(d) for scoring and attention (the pages give none; the
+ *     standard scaled dot product is used).
+ *   - Layouts (row-major, innermost last):
+ *       Q_dec          [batch][H][L_q][d]          bf16 or fp32
+ *       K_dec, V_dec   [batch][H_kv][L_q][d]       same dtype as Q_dec
+ *       K_pool, V_pool [n_slots][H_kv][page][d]    same dtype; one page of one
+ *                                                  KV head is page*d contiguous
+ *       page_table     int32 [batch][n_pages]      logical page -> pool slot
+ *       O              [batch][L_q][H][d]          dtype of the inputs
+ *       lse            fp32 [batch][H][L_q]        natural-log LSE of the
+ *                                                  scaled logits of each row
+ *     Logical token t of sequence b lives in slot page_table[b][t / page],
+ *     row t % page.  A contiguous cache uses the identity page table.
+ */
+#ifndef DL_H
+#define DL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DL_OK = 0,
+  DL_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, shape out of range      */
+  DL_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, page != 64, dtype mix, ...    */
+  DL_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required       */
+  DL_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed             */
+  DL_ERR_BAD_INDEX = 5,    /* device-detected out-of-range index (dl_get_status) */
+  DL_ERR_TIMEOUT = 6       /* a bounded device wait gave up (dl_get_status)    */
+} dl_status;
+
+typedef enum { DL_BF16 = 0, DL_FP32 = 1 } dl_dtype;
+
+/* Shape of one layer's attention problem. */
+typedef struct {
+  int batch;    /* sequences                                               */
+  int H;        /* query heads                                             */
+  int H_kv;     /* KV heads; H % H_kv == 0                                 */
+  int d;        /* head dimension: 64 or 128                               */
+  int L_ctx;    /* logical context tokens per sequence (same for all b);   */
+                /* tokens at t >= L_ctx are never read                     */
+  int L_q;      /* decode-block length, 1..256                             */
+  int page;     /* tokens per pool page = key-block size B; must be 64     */
+  int n_pages;  /* logical pages per sequence (row length of page_table);  */
+                /* n_pages * page >= L_ctx                                 */
+  int n_slots;  /* pages in the pool                                       */
+  int dtype;    /* dl_dtype of Q_dec, K/V pools, K_dec/V_dec and O         */
+} dl_attn_desc;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int dl_version(void);
+
+/* Message of the last error returned on this thread ("" if none). */
+const char* dl_last_error_message(void);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  Returns DL_OK, DL_ERR_BAD_INDEX, DL_ERR_TIMEOUT or
+ * DL_ERR_CUDA. */
+dl_status dl_get_status(void* stream);
+
+/* Bytes of workspace that suffice for every call below made with `desc`
+ * (any number of selected blocks or gathered tokens).  The workspace needs
+ * 256-byte alignment; its contents need no initialisation and are not
+ * preserved between calls.  Calls that share one workspace must be ordered
+ * (same stream). */
+dl_status dl_workspace_size(const dl_attn_desc* desc, size_t* bytes);
+
+/* (a1) Past-confidence-guided query prediction.  [F2 summary; key point 1]
+ * For each sequence: among positions with still_masked != 0 take the top-k
+ * by conf_prev (ties -> lower index; all of them if fewer than k are masked),
+ * widen each chosen p to [p-w, p+w] clipped to [0, L_q), and write the union
+ * in ascending order.
+ *   conf_prev    fp32  [batch][L_q]   finite values
+ *   still_masked uint8 [batch][L_q]
+ *   q_idx        int32 [batch][L_q]   out: positions, then -1 padding
+ *   q_cnt        int32 [batch]        out: number of predicted positions
+ * Requires 1 <= L_q <= 1024, k >= 0, w >= 0. */
+dl_status dl_predict_queries(const float* conf_prev, const uint8_t* still_masked, int batch,
+                             int L_q, int k, int w, int32_t* q_idx, int32_t* q_cnt,
+                             void* stream);
+
+/* (a2) Mean-pooled keys.  [F2 summary: predicted queries select the most
+ * relevant KV; pooling reading: one mean key per block]
+ * Unit u of sequence b covers logical tokens
+ *   [u*unit_stride + unit_offset, u*unit_stride + unit_offset + unit_len)
+ * clipped to [0, L_ctx).  Kbar[b][g][u] = (exact sum of those K rows) / n,
+ * rounded once to fp32 (units with no valid token get 0).  Key blocks use
+ * (stride, offset, len) = (page, 0, page); Prefilling-dLLM chunks [P1] with a
+ * BOS anchor first use (chunk_stride, 1, chunk_content).
+ *   K_pool  see layouts;  Kbar fp32 [batch][H_kv][n_units][d]  (out) */
+dl_status dl_pool_keys(const dl_attn_desc* desc, const void* K_pool, const int32_t* page_table,
+                       int n_units, int unit_stride, int unit_offset, int unit_len,
+                       float* Kbar, void* stream);
+
+/* (a3) Block scores with a fused block-level softmax.  [F2 summary]
+ * For KV head g, rows r = (h in g's query heads, i in predicted positions):
+ *   score[b][g][j] = sum_r softmax_j( scale * q_{h,i} . Kbar[b][g][j] )
+ * computed in fp64 from the bf16/fp32 queries and fp32 pooled keys.
+ * q_idx/q_cnt as written by dl_predict_queries; q_idx == NULL means every
+ * decode position is a row (q_cnt ignored).  q_cnt[b] == 0 gives all-zero
+ * scores.
+ *   score fp64 [batch][H_kv][n_units]  (out) */
+dl_status dl_block_scores(const dl_attn_desc* desc, const void* Q_dec, const int32_t* q_idx,
+                          const int32_t* q_cnt, const float* Kbar, int n_units, double* score,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* (a4) Attention-sink detection by attention mass.  [F1 abstract: sinks are
+ * kept and their locations reused across layers]
+ * mass[b][t] = sum over all heads h and predicted positions i of
+ *   softmax over (context tokens t < L_ctx, and the L_q decode keys) of
+ *   scale * q_{h,i} . k_t, for context columns t.
+ * sink_pos[b] = the n_sinks columns of largest mass (ties -> lower index),
+ * ascending.  Computed once, at the first sparse layer, and passed unchanged
+ * to dl_select of every deeper layer.
+ *   sink_pos int32 [batch][n_sinks]  (out);  1 <= n_sinks <= 64 */
+dl_status dl_find_sinks(const dl_attn_desc* desc, const void* Q_dec, const int32_t* q_idx,
+                        const int32_t* q_cnt, const void* K_pool, const int32_t* page_table,
+                        const void* K_dec, int n_sinks, int32_t* sink_pos, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/* (a5) Sink-aware top-K block selection.  [F1 abstract; F2 summary]
+ * For each (b, g): the sink units SB = { sink_pos[b][s] / unit_size : s,
+ * sink_pos >= 0 } are always kept; the topK remaining units of largest score
+ * (ties -> lower index) are added; the result is written ascending.
+ *   score    fp64  [batch][H_kv][n_units]
+ *   sink_pos int32 [batch][n_sinks] or NULL (n_sinks == 0)
+ *   blk_idx  int32 [batch][H_kv][max_sel]  out: ascending units, -1 padding
+ *   blk_cnt  int32 [batch][H_kv]           out: min(topK, n_units-|SB|)+|SB|
+ * Requires max_sel >= min(topK, n_units) + n_sinks, n_units <= 16384. */
+dl_status dl_select(const double* score, int batch, int H_kv, int n_units, int unit_size,
+                    int topK, const int32_t* sink_pos, int n_sinks, int32_t* blk_idx,
+                    int32_t* blk_cnt, int max_sel, void* stream);
+
+/* (a6) Block-sparse bidirectional attention.  [F1 abstract; F2 summary]
+ * For every query head h (KV head g) and decode position i:
+ *   o_{h,i} = sum_{t in S} softmax_t(scale * q_{h,i} . k_t) v_t
+ * where S = valid tokens (< L_ctx) of the blocks blk_idx[b][g][0..blk_cnt)
+ * (read through the page table, possibly non-contiguous) plus all L_q
+ * decode keys; no causal mask.  bf16 in, fp32 accumulation, online softmax;
+ * O rounded to nearest-even in the input dtype; lse optional (NULL: not
+ * written).  blk_idx == NULL selects every block (dense shallow layers).
+ *   blk_idx int32 [batch][H_kv][max_sel], blk_cnt int32 [batch][H_kv]
+ * Q_dec/K_pool/V_pool/K_dec/V_dec/O must be 16-byte aligned. */
+dl_status dl_sparse_attn(const dl_attn_desc* desc, const void* Q_dec, const void* K_pool,
+                         const void* V_pool, const int32_t* page_table, const int32_t* blk_idx,
+                         const int32_t* blk_cnt, int max_sel, const void* K_dec,
+                         const void* V_dec, void* O, float* lse, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* (a7) Intra-chunk token selection for a chunked prefix.  [P1 abstract]
+ * For each (b, g) and each selected chunk c = chunk_idx[b][g][s]: rows r =
+ * every decode query of g's heads;
+ *   tau[t] = sum_r softmax_t(scale * q_r . k_t) over the chunk's content
+ *            tokens t = c*chunk_stride + 1 .. c*chunk_stride + chunk_content
+ * The topT tokens of largest tau (ties -> lower position) and the chunk's BOS
+ * anchor at c*chunk_stride are kept.  tok_pos[b][g] receives all kept
+ * logical positions of the n_sel selected chunks, ascending; tok_cnt[b][g]
+ * their number (n_sel * (min(topT, chunk_content) + 1)).
+ *   chunk_idx int32 [batch][H_kv][n_sel] (from dl_select over chunks)
+ *   tok_pos   int32 [batch][H_kv][n_sel*(topT+1)]  (out)
+ * Requires 1 <= chunk_content <= 1024, 0 <= topT <= chunk_content. */
+dl_status dl_token_select(const dl_attn_desc* desc, const void* Q_dec, const void* K_pool,
+                          const int32_t* page_table, const int32_t* chunk_idx, int n_sel,
+                          int chunk_stride, int chunk_content, int topT, int32_t* tok_pos,
+                          int32_t* tok_cnt, void* ws, size_t ws_bytes, void* stream);
+
+/* (a7) Attention over gathered, non-contiguous cached tokens plus the decode
+ * block.  [P1 abstract: a kernel that parallelises decoding over the
+ * non-contiguously cached chunk KV]
+ * As dl_sparse_attn with S = logical positions tok_pos[b][g][0..tok_cnt)
+ * (each < n_pages*page) plus the L_q decode keys.
+ *   tok_pos int32 [batch][H_kv][max_tok], tok_cnt int32 [batch][H_kv] */
+dl_status dl_sparse_attn_gather(const dl_attn_desc* desc, const void* Q_dec, const void* K_pool,
+                                const void* V_pool, const int32_t* page_table,
+                                const int32_t* tok_pos, const int32_t* tok_cnt, int max_tok,
+                                const void* K_dec, const void* V_dec, void* O, float* lse,
+                                void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DL_H */

@@ -1,0 +1,67 @@
+// Key tiles of one (sequence, KV head) for the attention kernels.
+//
+// The keys a decode block attends to are a sequence of 64-row tiles: first
+// the context tiles (a selected block, every block in dense mode, or 64
+// gathered tokens), then ceil(L_q/64) tiles of the decode block's own keys.
+// A row resolves to an element offset into the pool (through the page table)
+// or into K_dec/V_dec, or to "invalid" (past the context end, a padding row,
+// or an out-of-range index -- the latter also raises the device error word).
+#pragma once
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dl {
+
+__device__ __forceinline__ int n_blocks(const Shape& s) { return (s.L_ctx + s.page - 1) / s.page; }
+
+__device__ __forceinline__ int ctx_tile_count(const AttnArgs& a, int bg) {
+  if (a.mode == kDense) return n_blocks(a.s);
+  int c = a.cnt[bg];
+  c = c < 0 ? 0 : (c > a.max_idx ? a.max_idx : c);
+  return a.mode == kBlocks ? c : (c + kTile - 1) / kTile;
+}
+
+// Element offset of row r of context tile `tile` of (b, g) in the pool, or
+// -1 when the row holds no key.
+__device__ __forceinline__ long long ctx_row_offset(const AttnArgs& a, int b, int g, int bg,
+                                                    int tile, int r) {
+  const Shape& s = a.s;
+  long long pos;
+  if (a.mode == kDense) {
+    pos = (long long)tile * kTile + r;
+  } else if (a.mode == kBlocks) {
+    const int j = a.idx[(size_t)bg * a.max_idx + tile];
+    if (j < 0 || j >= n_blocks(s)) {
+      if (r == 0) flag_error(a.err, ERR_BAD_INDEX);
+      return -1;
+    }
+    pos = (long long)j * kTile + r;
+  } else {
+    const int e = tile * kTile + r;
+    int c = a.cnt[bg];
+    c = c > a.max_idx ? a.max_idx : c;
+    if (e >= c) return -1;
+    pos = a.idx[(size_t)bg * a.max_idx + e];
+    if (pos < 0 || pos >= s.L_ctx) {
+      flag_error(a.err, ERR_BAD_INDEX);
+      return -1;
+    }
+  }
+  if (pos >= s.L_ctx) return -1;
+  const int lp = (int)(pos / s.page);
+  const int slot = a.page_table[(size_t)b * s.n_pages + lp];
+  if (slot < 0 || slot >= s.n_slots) {
+    flag_error(a.err, ERR_BAD_INDEX);
+    return -1;
+  }
+  return (((long long)slot * s.H_kv + g) * s.page + (pos % s.page)) * s.d;
+}
+
+// Element offset of decode key i of (b, g) in K_dec/V_dec, or -1.
+__device__ __forceinline__ long long dec_row_offset(const Shape& s, int bg, int i) {
+  if (i >= s.L_q) return -1;
+  return ((long long)bg * s.L_q + i) * s.d;
+}
+
+}  // namespace dl

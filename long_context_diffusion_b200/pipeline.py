@@ -1,0 +1,181 @@
+"""Host-side sequencing of the library's entry points into one layer of a
+denoising step, the chunked-prefix step, and the multi-layer step.
+
+Focus-dLLM (research.elamur.ai summary): the queries are predicted once per
+step from the previous step's confidence; shallow layers attend densely; the
+first sparse layer finds the attention sinks, which every deeper layer reuses
+unchanged (abstract: sink locations reused across layers); each sparse layer
+scores blocks with the predicted queries, keeps the top-K plus the sinks and
+attends over them.  Prefilling-dLLM (abstract): chunk selection, then token
+selection inside the kept chunks, then attention over the gathered tokens.
+
+This module only allocates torch tensors for outputs and workspaces and calls
+the C ABI (`_abi`) in order on one stream; all arithmetic runs in the
+library's kernels.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import List, Optional
+
+import torch
+
+from . import _abi as A
+
+
+def _empty(shape, dtype, device):
+    return torch.empty(shape, dtype=dtype, device=device)
+
+
+def workspace(desc: A.dl_attn_desc, device) -> torch.Tensor:
+    n = A.dl_workspace_size(desc)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+@dataclasses.dataclass
+class LayerOutputs:
+    q_idx: Optional[torch.Tensor]
+    q_cnt: Optional[torch.Tensor]
+    Kbar: Optional[torch.Tensor]
+    score: Optional[torch.Tensor]
+    sink_pos: Optional[torch.Tensor]
+    blk_idx: Optional[torch.Tensor]
+    blk_cnt: Optional[torch.Tensor]
+    O: torch.Tensor
+    lse: torch.Tensor
+
+
+def layer_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec, v_dec, *,
+               topK: int, conf_prev=None, still_masked=None, k: int = 4, w: int = 2,
+               q_idx=None, q_cnt=None, sink_pos=None, detect_sinks: int = 0,
+               dense: bool = False, Kbar=None, ws=None, stream=None) -> LayerOutputs:
+    """One layer for a batch: (predict,) pool, score, (find sinks,) select,
+    attend -- or dense attention.  Mirrors the oracle's layer_step."""
+    dev = q_dec.device
+    B, L_q, d, H, H_kv = desc.batch, desc.L_q, desc.d, desc.H, desc.H_kv
+    n_blk = -(-desc.L_ctx // desc.page)
+    if ws is None:
+        ws = workspace(desc, dev)
+    if q_idx is None and conf_prev is not None:
+        q_idx = _empty((B, L_q), torch.int32, dev)
+        q_cnt = _empty((B,), torch.int32, dev)
+        A.dl_predict_queries(conf_prev, still_masked, k, w, q_idx, q_cnt, stream)
+    O = _empty((B, L_q, H, d), q_dec.dtype, dev)
+    lse = _empty((B, H, L_q), torch.float32, dev)
+    if dense:
+        A.dl_sparse_attn(desc, q_dec, k_pool, v_pool, page_table, None, None, k_dec, v_dec, O,
+                         lse, ws, stream)
+        return LayerOutputs(q_idx, q_cnt, None, None, sink_pos, None, None, O, lse)
+    if Kbar is None:
+        Kbar = _empty((B, H_kv, n_blk, d), torch.float32, dev)
+        A.dl_pool_keys(desc, k_pool, page_table, n_blk, desc.page, 0, desc.page, Kbar, stream)
+    score = _empty((B, H_kv, n_blk), torch.float64, dev)
+    A.dl_block_scores(desc, q_dec, q_idx, q_cnt, Kbar, n_blk, score, ws, stream)
+    if detect_sinks:
+        sink_pos = _empty((B, detect_sinks), torch.int32, dev)
+        A.dl_find_sinks(desc, q_dec, q_idx, q_cnt, k_pool, page_table, k_dec, detect_sinks,
+                        sink_pos, ws, stream)
+    n_s = 0 if sink_pos is None else sink_pos.shape[-1]
+    max_sel = min(topK, n_blk) + n_s
+    blk_idx = _empty((B, H_kv, max(max_sel, 1)), torch.int32, dev)
+    blk_cnt = _empty((B, H_kv), torch.int32, dev)
+    A.dl_select(score, desc.page, topK, sink_pos, blk_idx, blk_cnt, stream)
+    A.dl_sparse_attn(desc, q_dec, k_pool, v_pool, page_table, blk_idx, blk_cnt, k_dec, v_dec, O,
+                     lse, ws, stream)
+    return LayerOutputs(q_idx, q_cnt, Kbar, score, sink_pos, blk_idx, blk_cnt, O, lse)
+
+
+@dataclasses.dataclass
+class ChunkOutputs:
+    Kbar: torch.Tensor
+    score: torch.Tensor
+    chunk_idx: torch.Tensor
+    chunk_cnt: torch.Tensor
+    tok_pos: torch.Tensor
+    tok_cnt: torch.Tensor
+    O: torch.Tensor
+    lse: torch.Tensor
+
+
+def chunked_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec, v_dec, *,
+                 n_chunks: int, stride: int, content: int, topK_chunks: int, topT: int,
+                 Kbar=None, ws=None, stream=None) -> ChunkOutputs:
+    """Chunked-prefix step: chunk keys (BOS excluded), chunk scores from
+    every decode query, top-K chunks, top-T tokens per chunk plus its BOS,
+    attention over the gathered tokens and the decode block."""
+    dev = q_dec.device
+    B, L_q, d, H, H_kv = desc.batch, desc.L_q, desc.d, desc.H, desc.H_kv
+    if ws is None:
+        ws = workspace(desc, dev)
+    if Kbar is None:
+        Kbar = _empty((B, H_kv, n_chunks, d), torch.float32, dev)
+        A.dl_pool_keys(desc, k_pool, page_table, n_chunks, stride, 1, content, Kbar, stream)
+    score = _empty((B, H_kv, n_chunks), torch.float64, dev)
+    A.dl_block_scores(desc, q_dec, None, None, Kbar, n_chunks, score, ws, stream)
+    kc = min(topK_chunks, n_chunks)
+    chunk_idx = _empty((B, H_kv, kc), torch.int32, dev)
+    chunk_cnt = _empty((B, H_kv), torch.int32, dev)
+    A.dl_select(score, stride, kc, None, chunk_idx, chunk_cnt, stream)
+    tok_pos = _empty((B, H_kv, kc * (topT + 1)), torch.int32, dev)
+    tok_cnt = _empty((B, H_kv), torch.int32, dev)
+    A.dl_token_select(desc, q_dec, k_pool, page_table, chunk_idx, stride, content, topT, tok_pos,
+                      tok_cnt, ws, stream)
+    O = _empty((B, L_q, H, d), q_dec.dtype, dev)
+    lse = _empty((B, H, L_q), torch.float32, dev)
+    A.dl_sparse_attn_gather(desc, q_dec, k_pool, v_pool, page_table, tok_pos, tok_cnt, k_dec,
+                            v_dec, O, lse, ws, stream)
+    return ChunkOutputs(Kbar, score, chunk_idx, chunk_cnt, tok_pos, tok_cnt, O, lse)
+
+
+class DenoiseStep:
+    """One denoising step over n_layers layers sharing a page table.
+
+    Per step: predict the queries once; layers below first_sparse attend
+    densely; layer first_sparse finds n_sinks sinks and every sparse layer
+    selects topK blocks plus those sinks.  Pooled keys are an input (they are
+    built when the KV cache is refreshed: `refresh_pooled_keys`).  All output
+    buffers are allocated once, so `run` can be captured in a CUDA graph."""
+
+    def __init__(self, desc: A.dl_attn_desc, n_layers: int, first_sparse: int, topK: int,
+                 n_sinks: int, k: int, w: int, dtype: torch.dtype, device):
+        self.desc, self.n_layers, self.first_sparse = desc, n_layers, first_sparse
+        self.topK, self.n_sinks, self.k, self.w = topK, n_sinks, k, w
+        B, L_q, d, H, H_kv = desc.batch, desc.L_q, desc.d, desc.H, desc.H_kv
+        self.n_blk = -(-desc.L_ctx // desc.page)
+        self.max_sel = min(topK, self.n_blk) + n_sinks
+        self.device = device
+        self.ws = workspace(desc, device)
+        self.q_idx = _empty((B, L_q), torch.int32, device)
+        self.q_cnt = _empty((B,), torch.int32, device)
+        self.sink_pos = _empty((B, n_sinks), torch.int32, device)
+        self.score = _empty((B, H_kv, self.n_blk), torch.float64, device)
+        self.blk_idx = [_empty((B, H_kv, self.max_sel), torch.int32, device)
+                        for _ in range(n_layers)]
+        self.blk_cnt = [_empty((B, H_kv), torch.int32, device) for _ in range(n_layers)]
+        self.O = [_empty((B, L_q, H, d), dtype, device) for _ in range(n_layers)]
+        self.lse = [_empty((B, H, L_q), torch.float32, device) for _ in range(n_layers)]
+
+    def refresh_pooled_keys(self, layer: int, k_pool, page_table, Kbar, stream=None):
+        d = self.desc
+        A.dl_pool_keys(d, k_pool, page_table, self.n_blk, d.page, 0, d.page, Kbar, stream)
+
+    def run(self, conf_prev, still_masked, q_dec: List, k_pool: List, v_pool: List,
+            page_table, k_dec: List, v_dec: List, Kbar: List, stream=None):
+        d = self.desc
+        A.dl_predict_queries(conf_prev, still_masked, self.k, self.w, self.q_idx, self.q_cnt,
+                             stream)
+        for l in range(self.n_layers):
+            if l < self.first_sparse:
+                A.dl_sparse_attn(d, q_dec[l], k_pool[l], v_pool[l], page_table, None, None,
+                                 k_dec[l], v_dec[l], self.O[l], self.lse[l], self.ws, stream)
+                continue
+            if l == self.first_sparse:
+                A.dl_find_sinks(d, q_dec[l], self.q_idx, self.q_cnt, k_pool[l], page_table,
+                                k_dec[l], self.n_sinks, self.sink_pos, self.ws, stream)
+            A.dl_block_scores(d, q_dec[l], self.q_idx, self.q_cnt, Kbar[l], self.n_blk,
+                              self.score, self.ws, stream)
+            A.dl_select(self.score, d.page, self.topK, self.sink_pos, self.blk_idx[l],
+                        self.blk_cnt[l], stream)
+            A.dl_sparse_attn(d, q_dec[l], k_pool[l], v_pool[l], page_table, self.blk_idx[l],
+                             self.blk_cnt[l], k_dec[l], v_dec[l], self.O[l], self.lse[l],
+                             self.ws, stream)

@@ -99,7 +99,7 @@ def layer_step(q_dec, k_pool, v_pool, page_table, k_dec, v_dec, L_ctx: int, B: i
         sinks = np.zeros((batch, 0), dtype=np.int64)
 
     n_s = sinks.shape[1] if n_sinks_cap is None else n_sinks_cap
-    max_sel = n_blk if dense else min(n_blk, topK + n_s)
+    max_sel = n_blk if dense else min(topK, n_blk) + n_s
     blk_idx = np.full((batch, H_kv, max_sel), -1, dtype=np.int64)
     blk_cnt = np.zeros((batch, H_kv), dtype=np.int64)
     O = np.zeros((batch, L_q, H, d))

@@ -1,0 +1,83 @@
+"""The C-ABI library on a host without a GPU: it loads, exports every entry
+point include/dl.h declares, and rejects bad arguments before launching."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_diffusion_b200 as dl
+from long_context_diffusion_b200 import _abi
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "dl.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dl_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_path():
+    names = _declared()
+    for n in ("dl_predict_queries", "dl_pool_keys", "dl_block_scores", "dl_find_sinks",
+              "dl_select", "dl_sparse_attn", "dl_token_select", "dl_sparse_attn_gather",
+              "dl_workspace_size", "dl_get_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(_abi.LIB_PATH)
+    for n in _declared():
+        assert hasattr(lib, n), n
+
+
+def test_version():
+    assert dl.dl_version() >= 100
+
+
+def _desc(**kw):
+    base = dict(batch=2, H=28, H_kv=4, d=128, L_ctx=16384, L_q=32, page=64, n_pages=256,
+                n_slots=512, dtype=dl.DL_BF16)
+    base.update(kw)
+    return dl.make_desc(**base)
+
+
+def test_workspace_size_and_validation():
+    n = dl.dl_workspace_size(_desc())
+    assert n > 0 and n % 256 == 0
+    bad = [dict(d=96), dict(page=32), dict(H=30), dict(L_q=0), dict(L_q=300), dict(n_pages=10),
+           dict(dtype=7), dict(batch=0)]
+    for kw in bad:
+        with pytest.raises(dl.DLError) as e:
+            dl.dl_workspace_size(_desc(**kw))
+        assert e.value.status in (dl.DL_ERR_INVALID_ARG, dl.DL_ERR_UNSUPPORTED), kw
+
+
+def test_null_and_range_arguments_rejected_before_launch():
+    lib = _abi.lib
+    d = _desc()
+    assert lib.dl_predict_queries(None, None, 1, 32, 4, 2, None, None, None) == dl.DL_ERR_INVALID_ARG
+    fake = ctypes.c_void_p(0x1000)
+    assert lib.dl_predict_queries(fake, fake, 1, 2000, 4, 2, fake, fake, None) == \
+        dl.DL_ERR_INVALID_ARG
+    assert lib.dl_select(None, 1, 1, 8, 64, 2, None, 0, fake, fake, 4, None) == \
+        dl.DL_ERR_INVALID_ARG
+    # max_sel too small for topK + sinks
+    assert lib.dl_select(fake, 1, 1, 8, 64, 4, fake, 2, fake, fake, 5, None) == \
+        dl.DL_ERR_INVALID_ARG
+    assert "max_sel" in lib.dl_last_error_message().decode()
+    # misaligned attention pointers
+    odd = ctypes.c_void_p(0x1008)
+    st = lib.dl_sparse_attn(ctypes.byref(d), odd, fake, fake, fake, None, None, 0, fake, fake,
+                            fake, None, fake, 1 << 40, None)
+    assert st == dl.DL_ERR_INVALID_ARG
+    # workspace too small
+    st = lib.dl_sparse_attn(ctypes.byref(d), fake, fake, fake, fake, None, None, 0, fake, fake,
+                            fake, None, ctypes.c_void_p(0x10000), 256, None)
+    assert st == dl.DL_ERR_WORKSPACE
+    # unsupported token-select sizes
+    st = lib.dl_token_select(ctypes.byref(d), fake, fake, fake, fake, 8, 1088, 2048, 256, fake,
+                             fake, None, 0, None)
+    assert st == dl.DL_ERR_INVALID_ARG

@@ -1,0 +1,139 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the
+same seeded inputs.  Index outputs (predicted positions, pooled keys, block
+and token selections, sinks) must match exactly; attention outputs within
+the stated tolerances."""
+import numpy as np
+import pytest
+import torch
+
+import long_context_diffusion_b200 as dl
+import oracle
+import synth
+from long_context_diffusion_b200 import pipeline
+from oracle import steps as S
+from tests.helpers import check_attention, desc_for, np_
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_layer(wl, inp, **kw):
+    desc = desc_for(wl)
+    out = pipeline.layer_step(desc, inp.q_dec, inp.k_pool, inp.v_pool, inp.page_table,
+                              inp.k_dec, inp.v_dec, topK=wl.topK, k=wl.k, w=wl.w, **kw)
+    assert dl.dl_get_status() == dl.DL_OK, dl._abi.lib.dl_last_error_message()
+    return out
+
+
+def _oracle_layer(wl, inp, **kw):
+    return oracle.layer_step(inp.q_dec.cpu(), inp.k_pool.cpu(), inp.v_pool.cpu(),
+                             inp.page_table.cpu(), inp.k_dec.cpu(), inp.v_dec.cpu(), wl.L_ctx,
+                             wl.B, wl.topK, k=wl.k, w=wl.w, **kw)
+
+
+def _compare_layer(out, ref, fp32, what):
+    assert np.array_equal(np_(out.q_idx), ref.q_idx), f"{what}: q_idx"
+    assert np.array_equal(np_(out.q_cnt), ref.q_cnt), f"{what}: q_cnt"
+    assert np.array_equal(np_(out.Kbar), ref.Kbar), f"{what}: pooled keys"
+    assert np.allclose(np_(out.score), ref.score, rtol=1e-12, atol=1e-15), f"{what}: scores"
+    assert np.array_equal(np_(out.blk_cnt), ref.blk_cnt), f"{what}: blk_cnt"
+    assert np.array_equal(np_(out.blk_idx), ref.blk_idx), f"{what}: blk_idx"
+    return check_attention(out.O, out.lse, ref.O, ref.lse, fp32, what)
+
+
+@pytest.mark.parametrize("name", ["tiny", "llada8k", "dream16k"])
+def test_single_layer_workloads(name, cuda_device):
+    wl = synth.workload(name)
+    inp = synth.make_step_inputs(wl, device=cuda_device)
+    sinks = inp.sinks_planted[:, : wl.sinks_given].contiguous()
+    out = _gpu_layer(wl, inp, conf_prev=inp.conf_prev, still_masked=inp.still_masked,
+                     sink_pos=sinks)
+    ref = _oracle_layer(wl, inp, conf_prev=inp.conf_prev.cpu(),
+                        still_masked=inp.still_masked.cpu(), sink_pos=sinks.cpu())
+    _compare_layer(out, ref, wl.dtype == "fp32", name)
+
+
+@pytest.mark.parametrize("name", ["llada8k", "dream16k"])
+def test_find_sinks_recovers_planted(name, cuda_device):
+    wl = synth.workload(name)
+    inp = synth.make_step_inputs(wl, device=cuda_device)
+    desc = desc_for(wl)
+    q_idx = torch.empty((wl.batch, wl.L_q), dtype=torch.int32, device=cuda_device)
+    q_cnt = torch.empty((wl.batch,), dtype=torch.int32, device=cuda_device)
+    dl.dl_predict_queries(inp.conf_prev, inp.still_masked, wl.k, wl.w, q_idx, q_cnt)
+    ws = pipeline.workspace(desc, cuda_device)
+    sinks = torch.empty((wl.batch, 4), dtype=torch.int32, device=cuda_device)
+    dl.dl_find_sinks(desc, inp.q_dec, q_idx, q_cnt, inp.k_pool, inp.page_table, inp.k_dec, 4,
+                     sinks, ws)
+    assert dl.dl_get_status() == dl.DL_OK
+    qi, qc = np_(q_idx), np_(q_cnt)
+    for b in range(wl.batch):
+        Kc = np.stack([S.gather_context(np_(inp.k_pool), np_(inp.page_table)[b], g,
+                                        np.arange(wl.L_ctx), wl.B) for g in range(wl.H_kv)])
+        top, _ = S.find_sinks(np_(inp.q_dec)[b], Kc, np_(inp.k_dec)[b], qi[b, : qc[b]], 4,
+                              S.scale_for(wl.d))
+        assert np_(sinks)[b].tolist() == top.tolist()
+        assert top.tolist() == np_(inp.sinks_planted)[b].tolist()
+
+
+def test_chunked_prefix_workload(cuda_device):
+    wl = synth.workload("chunked32k")
+    inp = synth.make_step_inputs(wl, device=cuda_device)
+    desc = desc_for(wl)
+    out = pipeline.chunked_step(desc, inp.q_dec, inp.k_pool, inp.v_pool, inp.page_table,
+                                inp.k_dec, inp.v_dec, n_chunks=wl.n_chunks,
+                                stride=wl.chunk_stride, content=wl.chunk_content,
+                                topK_chunks=wl.topK_chunks, topT=wl.topT_tokens)
+    assert dl.dl_get_status() == dl.DL_OK
+    ref = oracle.chunked_step(inp.q_dec.cpu(), inp.k_pool.cpu(), inp.v_pool.cpu(),
+                              inp.page_table.cpu(), inp.k_dec.cpu(), inp.v_dec.cpu(),
+                              n_chunks=wl.n_chunks, stride=wl.chunk_stride,
+                              content=wl.chunk_content, B=wl.B, topK_chunks=wl.topK_chunks,
+                              topT=wl.topT_tokens)
+    assert np.array_equal(np_(out.Kbar), ref.Kbar)
+    assert np.allclose(np_(out.score), ref.score, rtol=1e-12)
+    assert np.array_equal(np_(out.chunk_idx), ref.chunk_idx)
+    tp = np_(out.tok_pos)
+    if not np.array_equal(tp, ref.tok_pos):
+        # report the oracle's margin at every differing cut before failing
+        msgs = []
+        for b, g in zip(*np.nonzero((tp != ref.tok_pos).any(-1))):
+            msgs.append(f"(b={b}, g={g}) differs")
+        pytest.fail("token selection differs: " + "; ".join(msgs[:8]))
+    check_attention(out.O, out.lse, ref.O, ref.lse, False, "chunked32k")
+
+
+def test_multilayer_step_reduced(cuda_device):
+    """The 32K step's structure (dense layers, sinks found at the first
+    sparse layer and reused) at a reduced size the oracle finishes quickly."""
+    wl = synth.workload("llada32k_step", batch=2, L_ctx=4096, n_layers=4, topK=16)
+    desc = desc_for(wl)
+    layers = [synth.make_step_inputs(wl, layer=l, device=cuda_device) for l in range(4)]
+    step = pipeline.DenoiseStep(desc, 4, wl.first_sparse_layer, wl.topK, wl.detect_sinks, wl.k,
+                                wl.w, torch.bfloat16, cuda_device)
+    Kbar = [torch.empty((wl.batch, wl.H_kv, wl.n_blk, wl.d), dtype=torch.float32,
+                        device=cuda_device) for _ in range(4)]
+    for l in range(4):
+        step.refresh_pooled_keys(l, layers[l].k_pool, layers[l].page_table, Kbar[l])
+    x0 = layers[0]
+    step.run(x0.conf_prev, x0.still_masked, [x.q_dec for x in layers],
+             [x.k_pool for x in layers], [x.v_pool for x in layers], x0.page_table,
+             [x.k_dec for x in layers], [x.v_dec for x in layers], Kbar)
+    assert dl.dl_get_status() == dl.DL_OK
+    q_idx, q_cnt = oracle.step.predict_all(x0.conf_prev.cpu(), x0.still_masked.cpu(), wl.k, wl.w)
+    assert np.array_equal(np_(step.q_idx), q_idx)
+    sinks = None
+    for l, x in enumerate(layers):
+        common = dict(q_idx=q_idx, q_cnt=q_cnt)
+        if l < wl.first_sparse_layer:
+            ref = _oracle_layer(wl, x, dense=True, **common)
+        elif l == wl.first_sparse_layer:
+            ref = _oracle_layer(wl, x, detect_sinks=wl.detect_sinks, **common)
+            sinks = ref.sink_pos
+            assert np.array_equal(np_(step.sink_pos), sinks)
+            assert sinks.tolist() == np_(x.sinks_planted).tolist()
+        else:
+            ref = _oracle_layer(wl, x, sink_pos=sinks, **common)
+        if l >= wl.first_sparse_layer:
+            assert np.array_equal(np_(step.blk_idx[l]), ref.blk_idx), f"layer {l} blk_idx"
+            assert np.array_equal(np_(step.blk_cnt[l]), ref.blk_cnt), f"layer {l} blk_cnt"
+        check_attention(step.O[l], step.lse[l], ref.O, ref.lse, False, f"layer {l}")
