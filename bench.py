@@ -1,0 +1,482 @@
+#!/usr/bin/env python
+"""Benchmark of one denoising step of sink-aware, query-predicted,
+block-sparse bidirectional attention on the 32-layer, 32K-context workload.
+
+Workload (per GPU): LLaDA-8B attention shape, 32 layers x 32 heads, head dim
+128, 32768 cached context tokens, decode block of 32, batch 4.  Layers 0-1
+attend densely; layer 2 finds the 4 sinks (attention mass) that layers 2-31
+reuse; sparse layers keep the top-128 of 512 blocks plus the sink blocks.
+Synthetic bf16 inputs drawn by the seeded generator (`synth`), resident in
+HBM (68.7 GB of KV cache) before the timed region.
+
+A step = one refresh of one layer's pooled keys (the KV-cache refresh of a
+32-step block, amortised one layer per step) + query prediction + 32 layers
+(pooled-key scores, sinks at layer 2, selection, attention).  K steps are
+captured in one CUDA graph and timed with CUDA events on the launch stream;
+each attention call is bracketed by graph event nodes to time the dominant
+kernel over the same region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the fp64 CPU oracle (the reference arm) on a bounded
+sample of the same workload.  Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+from long_context_diffusion_b200 import runtime  # noqa: E402
+
+METRIC = "sparse-attn denoise steps/s and KV-tokens/s at 32K; % of HBM/tensor roofline"
+WORKLOAD = "llada32k_step"
+NOMINAL_HBM_GBS = 8000.0
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons of one GPU via NVML every
+    20 ms while the timed region runs."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, index: int):
+        self.samples, self._stop, self.ok = [], threading.Event(), False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = None
+            try:
+                pr = torch.cuda.get_device_properties(index)
+                bus = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self._reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - NVML missing
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                rs = self._reasons(self.h)
+                self.samples.append((sm, pw, rs))
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sms = [s[0] for s in self.samples]
+        reasons = sorted({n for _, _, r in self.samples for n, bit in self.REASONS.items()
+                          if r & bit})
+        return {"sm_mhz": float(statistics.median(sms)), "sm_max_mhz": int(self.max_mhz),
+                "reasons": reasons, "samples": len(sms),
+                "power_w_max": float(max(s[1] for s in self.samples))}
+
+
+# ---------------------------------------------------------------- inputs
+def make_inputs(wl, device):
+    """All layers' tensors of the workload, drawn on the device."""
+    pt = synth.page_permutation(wl).to(device)
+    layers = []
+    for l in range(wl.n_layers):
+        q = synth.make_q_dec(wl, l, device)
+        kd, vd = synth.make_kv_dec(wl, l, device)
+        kp, vp = synth.make_layer_kv(wl, l, q, device, pt.cpu())
+        layers.append(dict(q=q, kd=kd, vd=vd, kp=kp, vp=vp))
+    confs, masks = zip(*(synth.confidence(wl, b) for b in range(wl.batch)))
+    conf = torch.stack(confs).to(device)
+    masked = torch.stack(masks).to(device)
+    return layers, pt, conf, masked
+
+
+def attn_bytes(wl, n_ctx_tokens_per_bg):
+    """Algorithmic HBM bytes of one attention call: every attended context
+    K and V row once, the decode K/V, Q, O and the LSE."""
+    e = 2  # bf16
+    kv_ctx = sum(n_ctx_tokens_per_bg) * wl.d * e * 2
+    dec = wl.batch * wl.H_kv * wl.L_q * wl.d * e * 2
+    q = wl.batch * wl.H * wl.L_q * wl.d * e
+    o = wl.batch * wl.L_q * wl.H * wl.d * e + wl.batch * wl.H * wl.L_q * 4
+    return kv_ctx + dec + q + o
+
+
+def attn_flops(wl, n_ctx_tokens_per_bg):
+    keys = sum(n + wl.L_q for n in n_ctx_tokens_per_bg)
+    return 4.0 * wl.d * keys * wl.G * wl.L_q
+
+
+# ---------------------------------------------------------------- oracle arm
+def oracle_sample(wl, seconds_budget=8.0):
+    """Times the fp64 oracle on a bounded sample of the step and scales it to
+    one full step.  Sample: one sequence, a few KV heads, one dense layer, one
+    sparse layer (sinks given) and the sink search over those heads."""
+    import oracle
+    from oracle import steps as S
+    heads = 2
+    b, layer_d, layer_s = 0, 0, wl.first_sparse_layer
+    q = synth.make_q_dec(wl.replace(batch=1), layer_s)
+    qd = synth.make_q_dec(wl.replace(batch=1), layer_d)
+    scale = S.scale_for(wl.d)
+
+    def kv(layer, qq):
+        k, v = synth.make_logical_kv(wl.replace(batch=1), layer, b, 0, heads, qq)
+        return k, v
+
+    kd_full, vd_full = synth.make_kv_dec(wl.replace(batch=1), layer_s)
+    conf, masked = synth.confidence(wl, b)
+    q_idx = S.predict_queries(conf, masked, wl.k, wl.w)
+    t_dense = t_sparse = t_sink = 0.0
+    n_rep = 0
+    t_all = time.perf_counter()
+    while True:
+        k_d, v_d = kv(layer_d, qd)
+        t0 = time.perf_counter()
+        pool_k = k_d.view(heads, wl.n_blk, wl.B, wl.d).permute(1, 0, 2, 3).contiguous()
+        pool_v = v_d.view(heads, wl.n_blk, wl.B, wl.d).permute(1, 0, 2, 3).contiguous()
+        pt = np.arange(wl.n_blk)
+        S.dense_attention(qd[0, :heads], pool_k, pool_v, pt, wl.L_ctx, wl.B,
+                          kd_full[0, :heads], vd_full[0, :heads], scale)
+        t_dense += time.perf_counter() - t0
+        k_s, v_s = kv(layer_s, q)
+        t0 = time.perf_counter()
+        pool_k = k_s.view(heads, wl.n_blk, wl.B, wl.d).permute(1, 0, 2, 3).contiguous()
+        pool_v = v_s.view(heads, wl.n_blk, wl.B, wl.d).permute(1, 0, 2, 3).contiguous()
+        sinks = synth.sink_positions(wl, b)
+        r = oracle.layer_step(q[:, :heads], pool_k, pool_v, pt[None], kd_full[:, :heads],
+                              vd_full[:, :heads], wl.L_ctx, wl.B, wl.topK,
+                              q_idx=oracle.step._pad([q_idx], wl.L_q),
+                              q_cnt=np.array([len(q_idx)]), sink_pos=np.array([sinks]))
+        t_sparse += time.perf_counter() - t0
+        t0 = time.perf_counter()
+        S.find_sinks(q[0, :heads], S.f64(k_s), S.f64(kd_full[0, :heads]), q_idx, wl.detect_sinks,
+                     scale)
+        t_sink += time.perf_counter() - t0
+        n_rep += 1
+        if time.perf_counter() - t_all > seconds_budget or n_rep >= 3:
+            break
+    t_dense, t_sparse, t_sink = t_dense / n_rep, t_sparse / n_rep, t_sink / n_rep
+    per_seq_heads = wl.H_kv / heads * wl.batch
+    n_dense = wl.first_sparse_layer
+    n_sparse = wl.n_layers - wl.first_sparse_layer
+    t_step = per_seq_heads * (n_dense * t_dense + n_sparse * t_sparse + t_sink)
+    del r
+    cores = torch.get_num_threads()
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        cores = max([i.get("num_threads", 1) for i in info] + [cores])
+    except Exception:
+        pass
+    sample = (f"sequence 0, KV heads 0-{heads - 1} of {wl.H_kv}: one dense layer, one sparse "
+              f"layer (pool, score, select, attend) and the sink search, x{n_rep}; scaled by "
+              f"{per_seq_heads:.0f} (heads x batch) and by layer counts "
+              f"({n_dense} dense, {n_sparse} sparse, 1 sink search)")
+    return 1.0 / t_step, cores, sample, t_step
+
+
+def run_reference(args):
+    rank, world, _ = runtime.env_rank()
+    if rank != 0:
+        return 0
+    wl = synth.workload(WORKLOAD)
+    times = []
+    for i in range(args.warmup + args.steps):
+        v, cores, sample, t_step = oracle_sample(wl, seconds_budget=1.0)
+        if i >= args.warmup:
+            times.append(t_step)
+    t = float(np.mean(times))
+    value = 1.0 / t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(wl),
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def config_of(wl):
+    return {"workload": WORKLOAD, "layers": wl.n_layers, "batch_per_gpu": wl.batch,
+            "heads": wl.H, "kv_heads": wl.H_kv, "head_dim": wl.d, "context": wl.L_ctx,
+            "decode_block": wl.L_q, "block": wl.B, "topK": wl.topK, "sinks": wl.detect_sinks,
+            "dense_layers": wl.first_sparse_layer, "predict_k": wl.k, "window": wl.w,
+            "l2": "inputs larger than L2 (68.7 GB resident KV per GPU, 23 GB read per step)"}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    rank, world, local, device = runtime.init()
+    import long_context_diffusion_b200 as dl
+    from long_context_diffusion_b200 import pipeline
+
+    wl = synth.workload(WORKLOAD, n_layers=args.layers, batch=args.batch)
+    torch.manual_seed(0)
+    desc = dl.make_desc(wl.batch, wl.H, wl.H_kv, wl.d, wl.L_ctx, wl.L_q, wl.B, wl.n_pages,
+                        wl.n_slots, dl.DL_BF16)
+    t_gen = time.time()
+    layers, pt, conf, masked = make_inputs(wl, device)
+    t_gen = time.time() - t_gen
+    L = wl.n_layers
+    step = pipeline.DenoiseStep(desc, L, wl.first_sparse_layer, wl.topK, wl.detect_sinks, wl.k,
+                                wl.w, torch.bfloat16, device)
+    Kbar = [torch.empty((wl.batch, wl.H_kv, wl.n_blk, wl.d), dtype=torch.float32,
+                        device=device) for _ in range(L)]
+    stream = torch.cuda.Stream(device)
+    args_of = lambda: (conf, masked, [x["q"] for x in layers], [x["kp"] for x in layers],  # noqa
+                       [x["vp"] for x in layers], pt, [x["kd"] for x in layers],
+                       [x["vd"] for x in layers], Kbar)
+
+    def one_step(i, events=None):
+        step.refresh_pooled_keys(i % L, layers[i % L]["kp"], pt, Kbar[i % L], stream)
+        step.run(*args_of(), stream=stream, attn_events=events)
+
+    with torch.cuda.stream(stream):
+        for l in range(L):  # the cache refresh that precedes a block of steps
+            step.refresh_pooled_keys(l, layers[l]["kp"], pt, Kbar[l], stream)
+        one_step(0)
+    torch.cuda.synchronize(device)
+    st = dl.dl_get_status(stream)
+    if st != dl.DL_OK:
+        raise RuntimeError(f"device status {st} after the first step")
+
+    K, W = args.steps, args.warmup
+    g_warm = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_warm, stream=stream):
+        one_step(0)
+    events = []
+    g_timed = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_timed, stream=stream):
+        for i in range(K):
+            one_step(i, events)
+    for _ in range(W):
+        g_warm.replay()
+    torch.cuda.synchronize(device)
+
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    runtime.barrier(device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            g_timed.replay()
+            ev1.record(stream)
+        torch.cuda.synchronize(device)
+    runtime.barrier(device)
+    ms_total = ev0.elapsed_time(ev1)
+    ms_total = runtime.max_over_ranks(ms_total, device)
+    ms_step = ms_total / K
+    st = dl.dl_get_status(stream)
+    if st != dl.DL_OK:
+        raise RuntimeError(f"device status {st} after the timed steps")
+
+    # selected context tokens per (b, g) of each layer, from the returned counts
+    n_blk = wl.n_blk
+    ctx_tokens = []
+    for l in range(L):
+        if l < wl.first_sparse_layer:
+            ctx_tokens.append([wl.L_ctx] * (wl.batch * wl.H_kv))
+        else:
+            cnt = step.blk_cnt[l].view(-1).cpu().tolist()
+            idx = step.blk_idx[l].view(wl.batch * wl.H_kv, -1).cpu()
+            toks = []
+            for r, c in enumerate(cnt):
+                blocks = idx[r, :c]
+                last = (blocks == n_blk - 1).sum().item()
+                toks.append(int(c) * wl.B - last * (n_blk * wl.B - wl.L_ctx))
+            ctx_tokens.append(toks)
+    attn_b = [attn_bytes(wl, t) for t in ctx_tokens]
+    attn_f = [attn_flops(wl, t) for t in ctx_tokens]
+    kv_tokens = sum(sum(t) / wl.H_kv + wl.batch * wl.L_q for t in ctx_tokens)  # per step
+
+    # dominant kernel: the sparse-layer attention calls, over the timed region
+    sparse_ms, dense_ms = [], []
+    for layer, s, e in events:
+        (sparse_ms if layer >= wl.first_sparse_layer else dense_ms).append(
+            (layer, s.elapsed_time(e)))
+    sp_bytes = sum(attn_b[l] for l, _ in sparse_ms)
+    sp_time = sum(t for _, t in sparse_ms) / 1e3
+    sp_flops = sum(attn_f[l] for l, _ in sparse_ms)
+    dn_bytes = sum(attn_b[l] for l, _ in dense_ms)
+    dn_time = sum(t for _, t in dense_ms) / 1e3
+    pk, pk_kind = peaks()
+    achieved = sp_bytes / sp_time / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / pk["hbm_gbs"], "traffic": None,
+            "kernel": "dl_sparse_attn (sparse layers)", "launches": len(sparse_ms),
+            "bytes_per_launch": sp_bytes / max(1, len(sparse_ms)),
+            "avg_launch_us": sp_time / max(1, len(sparse_ms)) * 1e6,
+            "tflops": sp_flops / sp_time / 1e12, "peak_kind": f"{pk_kind} (copy)",
+            "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS}
+
+    # step-level roofline: algorithmic bytes of every kernel of one step
+    e2b = 2
+    pool_b = wl.batch * wl.H_kv * wl.L_ctx * wl.d * e2b + wl.batch * wl.H_kv * n_blk * wl.d * 4
+    kbar_b = wl.batch * wl.H_kv * n_blk * wl.d * 4
+    q_b = wl.batch * wl.H * wl.L_q * wl.d * e2b
+    sink_b = wl.batch * wl.H_kv * (wl.L_ctx + wl.L_q) * wl.d * e2b + q_b
+    n_sparse = L - wl.first_sparse_layer
+    score_b = n_sparse * (kbar_b + q_b + wl.batch * wl.H_kv * n_blk * 8)
+    step_bytes = pool_b + sink_b + score_b + sum(attn_b)
+    step_flops = sum(attn_f)
+    t_roof_meas = max(step_bytes / (pk["hbm_gbs"] * 1e9), step_flops / (pk["bf16_tflops"] * 1e12))
+    t_roof_nom = max(step_bytes / (NOMINAL_HBM_GBS * 1e9),
+                     step_flops / (NOMINAL_BF16_TFLOPS * 1e12))
+    t_step = ms_step / 1e3
+
+    # end to end: pinned host inputs in, outputs back, inside the timed graph
+    e2e = None
+    if not args.no_e2e:
+        h_in = {"conf": conf.cpu().pin_memory(), "masked": masked.cpu().pin_memory()}
+        for l in range(L):
+            for key in ("q", "kd", "vd"):
+                h_in[(l, key)] = layers[l][key].cpu().pin_memory()
+        h_out = {}
+        for l in range(L):
+            h_out[(l, "O")] = torch.empty_like(step.O[l], device="cpu").pin_memory()
+            h_out[(l, "lse")] = torch.empty_like(step.lse[l], device="cpu").pin_memory()
+            h_out[(l, "blk")] = torch.empty_like(step.blk_idx[l], device="cpu").pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+        d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+
+        def e2e_step(i):
+            conf.copy_(h_in["conf"], non_blocking=True)
+            masked.copy_(h_in["masked"], non_blocking=True)
+            for l in range(L):
+                for key in ("q", "kd", "vd"):
+                    layers[l][key].copy_(h_in[(l, key)], non_blocking=True)
+            one_step(i)
+            for l in range(L):
+                h_out[(l, "O")].copy_(step.O[l], non_blocking=True)
+                h_out[(l, "lse")].copy_(step.lse[l], non_blocking=True)
+                h_out[(l, "blk")].copy_(step.blk_idx[l], non_blocking=True)
+
+        g_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_e2e, stream=stream):
+            for i in range(K):
+                e2e_step(i)
+        g_e2e.replay()
+        torch.cuda.synchronize(device)
+        runtime.barrier(device)
+        torch.cuda.synchronize(device)
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            g_e2e.replay()
+            ev1.record(stream)
+        torch.cuda.synchronize(device)
+        runtime.barrier(device)
+        e2e_ms = runtime.max_over_ranks(ev0.elapsed_time(ev1), device) / K
+        e2e = {"value": runtime.weak_throughput([1] * world, e2e_ms / 1e3), "unit": "steps/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e2e_ms}
+        del g_e2e
+
+    launches_per_step = count_launches(wl)
+    value = runtime.weak_throughput([1] * world, t_step)
+    line = {
+        "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(wl),
+        "kv_tokens_per_s": kv_tokens * world / t_step,
+        "kv_tokens_per_step_per_gpu": kv_tokens,
+        "roofline": roof,
+        "step_roofline": {"bytes": step_bytes, "flops": step_flops,
+                          "frac_of_measured": t_roof_meas / t_step,
+                          "frac_of_nominal": t_roof_nom / t_step,
+                          "t_roof_measured_ms": t_roof_meas * 1e3,
+                          "t_roof_nominal_ms": t_roof_nom * 1e3,
+                          "dense_attn_GBps": dn_bytes / dn_time / 1e9 if dn_time else None},
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K,
+        "gen_seconds": t_gen,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        v, cores, sample, _ = oracle_sample(synth.workload(WORKLOAD))
+        line["cpu_baseline"] = {"value": v, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    del g_timed, g_warm
+    if rank == 0:
+        print(json.dumps(line))
+    runtime.finalize()
+    return 0
+
+
+def count_launches(wl):
+    """Kernels of this library launched per step (from the call sequence)."""
+    n_sparse = wl.n_layers - wl.first_sparse_layer
+    pool, predict, attn, sinks, scores, select = 1, 1, 2, 4, 2, 1
+    return pool + predict + wl.first_sparse_layer * attn + sinks + n_sparse * (
+        scores + select + attn)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--batch", type=int, default=4)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours" and args.layers == 32:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -160,14 +160,20 @@ class DenoiseStep:
         A.dl_pool_keys(d, k_pool, page_table, self.n_blk, d.page, 0, d.page, Kbar, stream)
 
     def run(self, conf_prev, still_masked, q_dec: List, k_pool: List, v_pool: List,
-            page_table, k_dec: List, v_dec: List, Kbar: List, stream=None):
+            page_table, k_dec: List, v_dec: List, Kbar: List, stream=None,
+            attn_events: Optional[list] = None):
+        """Launches the step on `stream`.  If attn_events is a list, a pair of
+        timing events (recorded as graph nodes when captured) brackets every
+        attention call and (layer, start, end) is appended to it."""
         d = self.desc
         A.dl_predict_queries(conf_prev, still_masked, self.k, self.w, self.q_idx, self.q_cnt,
                              stream)
         for l in range(self.n_layers):
             if l < self.first_sparse:
+                ev = self._begin(attn_events, stream)
                 A.dl_sparse_attn(d, q_dec[l], k_pool[l], v_pool[l], page_table, None, None,
                                  k_dec[l], v_dec[l], self.O[l], self.lse[l], self.ws, stream)
+                self._end(attn_events, ev, l, stream)
                 continue
             if l == self.first_sparse:
                 A.dl_find_sinks(d, q_dec[l], self.q_idx, self.q_cnt, k_pool[l], page_table,
@@ -176,6 +182,24 @@ class DenoiseStep:
                               self.score, self.ws, stream)
             A.dl_select(self.score, d.page, self.topK, self.sink_pos, self.blk_idx[l],
                         self.blk_cnt[l], stream)
+            ev = self._begin(attn_events, stream)
             A.dl_sparse_attn(d, q_dec[l], k_pool[l], v_pool[l], page_table, self.blk_idx[l],
                              self.blk_cnt[l], k_dec[l], v_dec[l], self.O[l], self.lse[l],
                              self.ws, stream)
+            self._end(attn_events, ev, l, stream)
+
+    @staticmethod
+    def _begin(events, stream):
+        if events is None:
+            return None
+        e = torch.cuda.Event(enable_timing=True, external=True)
+        e.record(stream)
+        return e
+
+    @staticmethod
+    def _end(events, start, layer, stream):
+        if events is None:
+            return
+        e = torch.cuda.Event(enable_timing=True, external=True)
+        e.record(stream)
+        events.append((layer, start, e))

@@ -72,7 +72,11 @@ def test_find_sinks_recovers_planted(name, cuda_device):
         top, _ = S.find_sinks(np_(inp.q_dec)[b], Kc, np_(inp.k_dec)[b], qi[b, : qc[b]], 4,
                               S.scale_for(wl.d))
         assert np_(sinks)[b].tolist() == top.tolist()
-        assert top.tolist() == np_(inp.sinks_planted)[b].tolist()
+        if wl.G == 1:
+            # with one query head per KV head the planted boost (3 x the mean
+            # query) dominates; averaged over a GQA group of 7 it does not, so
+            # there only the match with the oracle is required
+            assert top.tolist() == np_(inp.sinks_planted)[b].tolist()
 
 
 def test_chunked_prefix_workload(cuda_device):
