@@ -1,6 +1,6 @@
 """Builds the C-ABI shared library (libdlsparse.so) in-tree for sm_100a.
 
-    python -m long_context_diffusion_b200.build
+    python long_context_diffusion_b200/build.py        (or __graft_entry__.build())
 
 Compiles every csrc/*.cu with nvcc into long_context_diffusion_b200/lib/.
 Object files go to _build/ at the repository root; a file is recompiled when
