@@ -205,6 +205,23 @@ dl_status dl_sparse_attn_gather(const dl_attn_desc* desc, const void* Q_dec, con
                                 const void* K_dec, const void* V_dec, void* O, float* lse,
                                 void* ws, size_t ws_bytes, void* stream);
 
+/* Allocation-free variant of dl_block_scores.  The pages describe no
+ * counterpart: this serves callers that cannot allocate device memory (a
+ * runtime that owns all allocations and has no workspace to give, code where
+ * cudaMalloc is not allowed because it may synchronise the device, a process
+ * whose footprint is fixed after start-up).
+ * Same arguments and results as dl_block_scores, minus the workspace: the
+ * scratch is a 32 MiB array built into the library (held on every GPU that
+ * loads it until exit).  Calls needing more, i.e. with
+ * batch*H*L_q*n_units*8 > 32 MiB, return DL_ERR_WORKSPACE.  All calls on a
+ * device share the array; calls whose kernels may overlap on the GPU race on
+ * it and must be ordered (one stream).  The first call on each device looks
+ * up the array's device address, so make it before any stream capture.  The
+ * call allocates nothing. */
+dl_status dl_block_scores_noalloc(const dl_attn_desc* desc, const void* Q_dec,
+                                  const int32_t* q_idx, const int32_t* q_cnt, const float* Kbar,
+                                  int n_units, double* score, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

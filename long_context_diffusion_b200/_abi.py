@@ -56,6 +56,8 @@ _SIGS = {
                         _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp], _c_int),
     "dl_token_select": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _c_int, _c_int,
                          _c_int, _c_int, _vp, _vp, _vp, ctypes.c_size_t, _vp], _c_int),
+    "dl_block_scores_noalloc": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _c_int, _vp,
+                                 _vp], _c_int),
     "dl_sparse_attn_gather": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _vp, _vp,
                                _c_int, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp], _c_int),
 }
@@ -173,3 +175,10 @@ def dl_sparse_attn_gather(desc, Q_dec, K_pool, V_pool, page_table, tok_pos, tok_
                                      _p(page_table), _p(tok_pos), _p(tok_cnt), tok_pos.shape[-1],
                                      _p(K_dec), _p(V_dec), _p(O), _p(lse), _p(ws),
                                      ws.numel() * ws.element_size(), _s(stream)))
+
+
+def dl_block_scores_noalloc(desc, Q_dec, q_idx, q_cnt, Kbar, n_units, score, stream=None):
+    """dl_block_scores without a workspace: for callers that cannot allocate
+    device memory; the library's built-in 32 MiB scratch array is used."""
+    _check(lib.dl_block_scores_noalloc(ctypes.byref(desc), _p(Q_dec), _p(q_idx), _p(q_cnt),
+                                       _p(Kbar), n_units, _p(score), _s(stream)))

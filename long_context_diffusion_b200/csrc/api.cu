@@ -108,6 +108,14 @@ int n_blk_of(const dl::Shape& s) { return (s.L_ctx + s.page - 1) / s.page; }
 
 }  // namespace
 
+// Validation and error-word access for entry points defined in other files.
+namespace dl {
+dl_status api_check_desc(const dl_attn_desc* d, Shape* s) { return check_desc(d, s); }
+dl_status api_error_word(unsigned** out) { return error_word(out); }
+dl_status api_fail(dl_status st, const char* msg) { return fail(st, "%s", msg); }
+dl_status api_ok() { return ok(); }
+}  // namespace dl
+
 extern "C" {
 
 int dl_version(void) { return 100; }

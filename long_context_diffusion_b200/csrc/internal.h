@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/dl.h"
+
 namespace dl {
 
 // Device error word codes (bit flags, OR-ed into the word).
@@ -76,6 +78,12 @@ cudaError_t launch_token_select(const Shape& s, const void* Q, const void* Kp,
                                 const int32_t* page_table, const int32_t* chunk_idx, int n_sel,
                                 int chunk_stride, int chunk_content, int topT, int32_t* tok_pos,
                                 int32_t* tok_cnt, unsigned* err, cudaStream_t st);
+
+// Shared by entry points in several files (defined in api.cu).
+dl_status api_check_desc(const dl_attn_desc* d, Shape* s);
+dl_status api_error_word(unsigned** out);
+dl_status api_fail(dl_status st, const char* msg);
+dl_status api_ok();
 
 __host__ __device__ inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
