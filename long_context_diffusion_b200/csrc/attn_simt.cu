@@ -30,20 +30,6 @@ __host__ __device__ constexpr size_t simt_smem_bytes() {
          sizeof(int) * kTile;
 }
 
-struct Partials {
-  float* o;    // [bg][split][R][d]
-  float2* ml;  // [bg][split][R]  (running max in natural-log units, sum)
-};
-
-__host__ __device__ inline Partials partials_of(void* ws, const Shape& s, int n_split) {
-  const size_t R = (size_t)s.G * s.L_q;
-  const size_t n = (size_t)s.batch * s.H_kv * n_split * R;
-  Partials p;
-  p.o = reinterpret_cast<float*>(ws);
-  p.ml = reinterpret_cast<float2*>(reinterpret_cast<char*>(ws) + round256(n * s.d * sizeof(float)));
-  return p;
-}
-
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 attn_simt_kernel(AttnArgs a, int n_split, int tps) {
@@ -218,6 +204,23 @@ int attn_splits(const Shape& s, int max_tiles) {
 }
 
 template <typename T, int D>
+static cudaError_t run_combine(const AttnArgs& a, int n_split, cudaStream_t st) {
+  const Shape& s = a.s;
+  const long long rows = (long long)s.batch * s.H_kv * s.G * s.L_q;
+  attn_combine_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+      s, n_split, a.ws, reinterpret_cast<T*>(a.O), a.lse);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const AttnArgs& a, int n_split, cudaStream_t st) {
+  if (a.s.dtype == 1)
+    return a.s.d == 128 ? run_combine<float, 128>(a, n_split, st)
+                        : run_combine<float, 64>(a, n_split, st);
+  return a.s.d == 128 ? run_combine<__nv_bfloat16, 128>(a, n_split, st)
+                      : run_combine<__nv_bfloat16, 64>(a, n_split, st);
+}
+
+template <typename T, int D>
 static cudaError_t run_simt(const AttnArgs& a, int max_tiles, cudaStream_t st) {
   const Shape& s = a.s;
   const int n_split = attn_splits(s, max_tiles);
@@ -230,10 +233,7 @@ static cudaError_t run_simt(const AttnArgs& a, int max_tiles, cudaStream_t st) {
   attn_simt_kernel<T, D><<<grid, 256, smem, st>>>(a, n_split, tps);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const long long rows = (long long)s.batch * s.H_kv * s.G * s.L_q;
-  attn_combine_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
-      s, n_split, a.ws, reinterpret_cast<T*>(a.O), a.lse);
-  return cudaGetLastError();
+  return launch_combine(a, n_split, st);
 }
 
 static int max_tiles_of(const AttnArgs& a) {
@@ -253,6 +253,15 @@ cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t st) {
                       : run_simt<__nv_bfloat16, 64>(a, mt, st);
 }
 
-cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) { return launch_attn_simt(a, st); }
+bool attn_tc_supported(const AttnArgs& a);
+cudaError_t launch_attn_tc(const AttnArgs& a, int max_tiles, cudaStream_t st);
+
+// bf16 block/dense attention runs on the tensor cores (attn_tc.cu); fp32
+// inputs (exact FMAs for the 1e-5 bar), gathered tokens and query groups of
+// more than 256 rows run on this kernel.
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
+  if (attn_tc_supported(a)) return launch_attn_tc(a, max_tiles_of(a), st);
+  return launch_attn_simt(a, st);
+}
 
 }  // namespace dl

@@ -64,4 +64,21 @@ __device__ __forceinline__ long long dec_row_offset(const Shape& s, int bg, int 
   return ((long long)bg * s.L_q + i) * s.d;
 }
 
+// Split-KV partials in the workspace: for each (b, g), split and query row
+// r = (h in the group, i), the unnormalised output row, and (running max in
+// natural-log units, running sum of exponentials).
+struct Partials {
+  float* o;    // [bg][split][R][d]
+  float2* ml;  // [bg][split][R]
+};
+
+__host__ __device__ inline Partials partials_of(void* ws, const Shape& s, int n_split) {
+  const size_t R = (size_t)s.G * s.L_q;
+  const size_t n = (size_t)s.batch * s.H_kv * n_split * R;
+  Partials p;
+  p.o = reinterpret_cast<float*>(ws);
+  p.ml = reinterpret_cast<float2*>(reinterpret_cast<char*>(ws) + round256(n * s.d * sizeof(float)));
+  return p;
+}
+
 }  // namespace dl
