@@ -406,8 +406,10 @@ EncodeTiled encoder() {
   return fn;
 }
 
+}  // namespace
+
 // bf16 rows of `inner` elements, boxes of 64 x box_rows, 128-byte swizzle.
-bool map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+bool tc_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
   EncodeTiled fn = encoder();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, rows};
@@ -418,6 +420,8 @@ bool map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uin
             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
 
 // decode block K/V: [bg][L_q][d], boxes of 64 x 64 x 1 (rows past L_q read 0)
 bool map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t L_q, uint64_t n_bg) {
@@ -432,12 +436,16 @@ bool map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t L_q, uint
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count() {
+}  // namespace
+
+int tc_sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n;
 }
+
+namespace {
 
 // Splits per (b, g): minimise waves x (tiles per CTA + fixed cost), one CTA
 // per SM resident.
@@ -470,11 +478,11 @@ static cudaError_t run_tc(const AttnArgs& a, int max_tiles, cudaStream_t st) {
   const uint64_t pool_rows = (uint64_t)s.n_slots * s.H_kv * 64;
   const uint64_t q_rows = (uint64_t)s.batch * s.H * s.L_q;
   const uint64_t n_bg = (uint64_t)s.batch * s.H_kv;
-  if (!map_2d(&mq, a.Q, D, q_rows, 128) || !map_2d(&mk, a.Kp, D, pool_rows, 64) ||
-      !map_2d(&mv, a.Vp, D, pool_rows, 64) || !map_3d(&mkd, a.Kd, D, s.L_q, n_bg) ||
+  if (!tc_map_2d(&mq, a.Q, D, q_rows, 128) || !tc_map_2d(&mk, a.Kp, D, pool_rows, 64) ||
+      !tc_map_2d(&mv, a.Vp, D, pool_rows, 64) || !map_3d(&mkd, a.Kd, D, s.L_q, n_bg) ||
       !map_3d(&mvd, a.Vd, D, s.L_q, n_bg))
     return cudaErrorInvalidValue;
-  const int n_split = tc_splits((int)n_bg, max_tiles, sm_count());
+  const int n_split = tc_splits((int)n_bg, max_tiles, tc_sm_count());
   const int tps = (max_tiles + n_split - 1) / n_split;
   auto kern = attn_tc_kernel<D, NM, ST, PB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);

@@ -9,10 +9,9 @@
 // the spacing of neighbouring scores, so the kept set equals the one an
 // exact computation gives.
 //
-// Two kernels.  (1) logits: grid (unit tiles, b*H_kv); each CTA stages 32
-// pooled keys and up to 32 query rows in shared memory (fp32, padded rows so
-// lanes hit distinct banks) and writes scale * q . Kbar in fp64 to the
-// workspace.  (2) softmax: one CTA per (b, g); a warp per row takes its max
+// Two kernels.  (1) logits: grid (64-unit tiles, b*H_kv); each thread owns
+// one pooled key and 8 query rows (staged in shared memory as fp64) and
+// writes scale * q . Kbar in fp64 to the workspace.  (2) softmax: one CTA per (b, g); a warp per row takes its max
 // and sum of exponentials by shuffles and writes the probabilities in place;
 // then one thread per unit sums its column over the rows in row order.
 #include "common.cuh"
@@ -20,53 +19,67 @@
 
 namespace dl {
 
-constexpr int kUT = 32;   // units per logits CTA
-constexpr int kRT = 32;   // query rows staged per pass
+constexpr int kUT = 64;   // units per logits CTA (one per thread column)
+constexpr int kRT = 32;   // query rows staged per pass (8 per thread)
 
+// Thread (u, rg): unit u0 + (tid % 64), rows rg*8 .. rg*8+7 of the pass.
+// Query rows are staged once as fp64 (exact) and read as broadcasts; the
+// pooled key is read 16 bytes at a time and converted once per element; the
+// 8 products per key element accumulate with fp64 FMAs.
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 scores_logits_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
                      const int32_t* __restrict__ q_cnt, const float* __restrict__ Kbar,
                      Shape s, int n_units, double* __restrict__ S, unsigned* err) {
-  __shared__ float sK[kUT][D + 1];
-  __shared__ float sQ[kRT][D];
+  __shared__ __align__(16) double sQ[kRT][D];
   const int bg = blockIdx.y;
   const int b = bg / s.H_kv, g = bg % s.H_kv;
-  const int u0 = blockIdx.x * kUT;
+  const int u = blockIdx.x * kUT + (threadIdx.x % kUT);
+  const int rg = threadIdx.x / kUT;  // 0..3
   const int nq = q_idx ? min(max(q_cnt[b], 0), s.L_q) : s.L_q;
   const int R = nq * s.G;
   const int R_max = s.L_q * s.G;
-  for (int e = threadIdx.x; e < kUT * D; e += blockDim.x) {
-    const int j = e / D, c = e % D;
-    sK[j][c] = (u0 + j < n_units) ? Kbar[(((size_t)b * s.H_kv + g) * n_units + u0 + j) * D + c]
-                                  : 0.0f;
-  }
-  const int j = threadIdx.x % kUT;
-  const int rl = threadIdx.x / kUT;  // 0..7
+  const bool u_ok = u < n_units;
+  const float* kb = Kbar + (((size_t)b * s.H_kv + g) * n_units + (u_ok ? u : 0)) * D;
   for (int r0 = 0; r0 < R; r0 += kRT) {
     __syncthreads();
     for (int e = threadIdx.x; e < kRT * D; e += blockDim.x) {
       const int rr = e / D, c = e % D;
       const int r = r0 + rr;
-      float v = 0.0f;
+      double v = 0.0;
       if (r < R) {
         const int h = g * s.G + r / nq;
         const int i = q_idx ? q_idx[(size_t)b * s.L_q + (r % nq)] : (r % nq);
         if (i >= 0 && i < s.L_q)
-          v = to_f32(Q[(((size_t)b * s.H + h) * s.L_q + i) * D + c]);
+          v = (double)to_f32(Q[(((size_t)b * s.H + h) * s.L_q + i) * D + c]);
         else if (c == 0)
           flag_error(err, ERR_BAD_INDEX);
       }
       sQ[rr][c] = v;
     }
     __syncthreads();
-    for (int rr = rl; rr < kRT; rr += 8) {
-      const int r = r0 + rr;
-      if (r >= R || u0 + j >= n_units) continue;
-      double acc = 0.0;
-#pragma unroll 16
-      for (int c = 0; c < D; ++c) acc = fma((double)sQ[rr][c], (double)sK[j][c], acc);
-      S[((size_t)bg * R_max + r) * n_units + u0 + j] = acc * s.scale;
+    if (!u_ok || r0 + rg * 8 >= R) continue;
+    double acc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = 0.0;
+#pragma unroll 2
+    for (int c0 = 0; c0 < D; c0 += 4) {
+      const float4 kv = __ldg(reinterpret_cast<const float4*>(kb + c0));
+      const double k0 = kv.x, k1 = kv.y, k2 = kv.z, k3 = kv.w;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const double2 qa = *reinterpret_cast<const double2*>(&sQ[rg * 8 + k][c0]);
+        const double2 qb = *reinterpret_cast<const double2*>(&sQ[rg * 8 + k][c0 + 2]);
+        acc[k] = fma(qa.x, k0, acc[k]);
+        acc[k] = fma(qa.y, k1, acc[k]);
+        acc[k] = fma(qb.x, k2, acc[k]);
+        acc[k] = fma(qb.y, k3, acc[k]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int r = r0 + rg * 8 + k;
+      if (r < R) S[((size_t)bg * R_max + r) * n_units + u] = acc[k] * s.scale;
     }
   }
 }

@@ -5,16 +5,102 @@
 // the topK other blocks of largest fp64 score are added (ties -> lower
 // index), and the union is written ascending.
 //
-// One CTA per (b, g).  Scores are staged in shared memory; a block's rank is
-// the number of candidates ordered before it by (score desc, index asc),
-// counted with an early exit once it reaches topK.  The ascending compaction
-// is a ballot/popc prefix count over the unit indices.
+// One CTA per (b, g).  Up to 4096 units: a bitonic sort in shared memory of
+// (score desc, index asc) keys -- the score's bits made order-preserving and
+// inverted, the index as the tie-break -- with sinks and padding sorted
+// last; the first topK entries are kept.  Larger unit counts use a rank
+// count (the number of candidates ordered before each unit).  The ascending
+// compaction is a ballot/popc prefix count over the unit indices.
 #include "common.cuh"
 #include "internal.h"
 
 namespace dl {
 
 constexpr int kSelThreads = 1024;
+constexpr int kBitonicMax = 4096;
+
+// Ascending order of the result equals descending order of x (IEEE bits made
+// monotone, then inverted).
+__device__ __forceinline__ uint64_t desc_key(double x) {
+  const uint64_t b = static_cast<uint64_t>(__double_as_longlong(x));
+  const uint64_t mono = (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+  return ~mono;
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+select_bitonic_kernel(const double* __restrict__ score, int H_kv, int n_units, int n2,
+                      int unit_size, int topK, const int32_t* __restrict__ sink_pos, int n_sinks,
+                      int32_t* __restrict__ blk_idx, int32_t* __restrict__ blk_cnt, int max_sel,
+                      unsigned* err) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint64_t* s_key = reinterpret_cast<uint64_t*>(smem);
+  int* s_idx = reinterpret_cast<int*>(s_key + n2);
+  uint8_t* s_sink = reinterpret_cast<uint8_t*>(s_idx + n2);
+  uint8_t* s_keep = s_sink + n2;
+  __shared__ int s_warp[33];
+  __shared__ int s_nsb;
+  __shared__ int s_base;
+  const int bg = blockIdx.x;
+  const int b = bg / H_kv;
+  const double* sc = score + (size_t)bg * n_units;
+  for (int u = threadIdx.x; u < n2; u += blockDim.x) {
+    s_sink[u] = 0;
+    s_keep[u] = 0;
+  }
+  if (threadIdx.x == 0) { s_nsb = 0; s_base = 0; }
+  __syncthreads();
+  for (int t = threadIdx.x; t < n_sinks; t += blockDim.x) {
+    const int p = sink_pos[(size_t)b * n_sinks + t];
+    if (p >= 0) {
+      const long long u = p / unit_size;
+      if (u < n_units) s_sink[u] = 1;
+      else flag_error(err, ERR_BAD_INDEX);
+    }
+  }
+  __syncthreads();
+  for (int u = threadIdx.x; u < n2; u += blockDim.x) {
+    const bool cand = u < n_units && !s_sink[u];
+    s_key[u] = cand ? desc_key(sc[u]) : ~0ull;
+    s_idx[u] = u;
+    if (u < n_units && s_sink[u]) atomicAdd(&s_nsb, 1);
+  }
+  __syncthreads();
+  for (int k = 2; k <= n2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+        const int l = i ^ j;
+        if (l > i) {
+          const uint64_t ki = s_key[i], kl = s_key[l];
+          const int ii = s_idx[i], il = s_idx[l];
+          const bool i_after = ki > kl || (ki == kl && ii > il);
+          if (((i & k) == 0) == i_after) {
+            s_key[i] = kl; s_key[l] = ki;
+            s_idx[i] = il; s_idx[l] = ii;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const int n_cand = n_units - s_nsb;
+  const int take = topK < n_cand ? topK : n_cand;
+  for (int t = threadIdx.x; t < take; t += blockDim.x) s_keep[s_idx[t]] = 1;
+  __syncthreads();
+  int32_t* out = blk_idx + (size_t)bg * max_sel;
+  for (int u0 = 0; u0 < n_units; u0 += blockDim.x) {
+    const int u = u0 + threadIdx.x;
+    const bool keep = u < n_units && (s_keep[u] || s_sink[u]);
+    int total = 0;
+    const int pos = block_exclusive_count(keep, s_warp, &total);
+    if (keep && s_base + pos < max_sel) out[s_base + pos] = u;
+    __syncthreads();
+    if (threadIdx.x == 0) s_base += total;
+    __syncthreads();
+  }
+  const int cnt = s_base;
+  for (int e = cnt + threadIdx.x; e < max_sel; e += blockDim.x) out[e] = -1;
+  if (threadIdx.x == 0) blk_cnt[bg] = cnt < max_sel ? cnt : max_sel;
+}
 
 __global__ void __launch_bounds__(kSelThreads)
 select_kernel(const double* __restrict__ score, int H_kv, int n_units, int unit_size, int topK,
@@ -73,6 +159,21 @@ select_kernel(const double* __restrict__ score, int H_kv, int n_units, int unit_
 cudaError_t launch_select(const double* score, int batch, int H_kv, int n_units, int unit_size,
                           int topK, const int32_t* sink_pos, int n_sinks, int32_t* blk_idx,
                           int32_t* blk_cnt, int max_sel, unsigned* err, cudaStream_t st) {
+  if (n_units <= kBitonicMax) {
+    int n2 = 2;
+    while (n2 < n_units) n2 <<= 1;
+    const size_t smem = (size_t)n2 * (sizeof(uint64_t) + sizeof(int) + 2);
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(select_bitonic_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    const int threads = n2 / 2 < 32 ? 32 : (n2 / 2 > kSelThreads ? kSelThreads : n2 / 2);
+    select_bitonic_kernel<<<batch * H_kv, threads, smem, st>>>(
+        score, H_kv, n_units, n2, unit_size, topK, sink_pos, n_sinks, blk_idx, blk_cnt, max_sel,
+        err);
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)n_units * (sizeof(double) + 1);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(select_kernel,

@@ -6,7 +6,9 @@
 // summed over every head; they are found once, at the first sparse layer.
 //
 // The softmax of each row runs over the whole context plus the decode block,
-// so its normaliser must be known before any column mass can be formed:
+// so its normaliser must be known before any column mass can be formed.
+// bf16 inputs take the tensor-core passes (sinks_tc.cu); the CUDA-core
+// passes below serve fp32 inputs and query groups of more than 256 rows:
 //   pass 1  grid (token tiles, b*H): per tile and predicted row, the max and
 //           the sum of exponentials of the tile's logits (one thread per
 //           token, key row in registers, query rows broadcast from shared
@@ -44,10 +46,35 @@ __host__ __device__ inline SinkWs sink_ws(void* ws, const Shape& s) {
   return w;
 }
 
+// Tensor-core path: [attention partials][O scratch][LSE of every row][mass]
+struct SinkTcWs {
+  void* attn;
+  void* O;
+  float* lse;
+  float* mass;
+};
+
+static SinkTcWs sink_tc_ws(void* ws, const Shape& s) {
+  char* p = reinterpret_cast<char*>(ws);
+  SinkTcWs w;
+  w.attn = p;
+  p += attn_workspace(s);
+  w.O = p;
+  p += round256((size_t)s.batch * s.L_q * s.H * s.d * 2);
+  w.lse = reinterpret_cast<float*>(p);
+  p += round256((size_t)s.batch * s.H * s.L_q * sizeof(float));
+  w.mass = reinterpret_cast<float*>(p);
+  return w;
+}
+
 size_t sinks_workspace(const Shape& s) {
-  return round256((size_t)s.batch * s.H * sink_tiles(s) * s.L_q * sizeof(float2)) +
-         round256((size_t)s.batch * s.H * s.L_q * sizeof(float)) +
-         round256((size_t)s.batch * s.L_ctx * sizeof(float));
+  const size_t simt = round256((size_t)s.batch * s.H * sink_tiles(s) * s.L_q * sizeof(float2)) +
+                      round256((size_t)s.batch * s.H * s.L_q * sizeof(float)) +
+                      round256((size_t)s.batch * s.L_ctx * sizeof(float));
+  const size_t tc = attn_workspace(s) + round256((size_t)s.batch * s.L_q * s.H * s.d * 2) +
+                    round256((size_t)s.batch * s.H * s.L_q * sizeof(float)) +
+                    round256((size_t)s.batch * s.L_ctx * sizeof(float));
+  return simt > tc ? simt : tc;
 }
 
 // Loads key row `t` of KV head g (context t < L_ctx, else decode key t-L_ctx)
@@ -251,10 +278,34 @@ static cudaError_t run_sinks(const Shape& s, const void* Q, const int32_t* q_idx
   return cudaGetLastError();
 }
 
+bool attn_tc_supported(const AttnArgs& a);
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_sink_mass_tc(const Shape& s, const void* Q, const int32_t* q_idx,
+                                const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
+                                const float* lse, float* mass, unsigned* err, cudaStream_t st);
+
+// bf16 with at most 256 query rows per KV group: tensor cores (pass 1 = dense
+// attention with V = K for the row LSEs, pass 2 = sinks_tc.cu); otherwise
+// the CUDA-core passes above.
 cudaError_t launch_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
                          const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
                          const void* Kd, int n_sinks, int32_t* sink_pos, void* ws,
                          unsigned* err, cudaStream_t st) {
+  SinkTcWs tw = sink_tc_ws(ws, s);
+  AttnArgs a{};
+  a.s = s; a.Q = Q; a.Kp = Kp; a.Vp = Kp; a.page_table = page_table; a.mode = kDense;
+  a.idx = nullptr; a.cnt = nullptr; a.max_idx = 0; a.Kd = Kd; a.Vd = Kd; a.O = tw.O;
+  a.lse = tw.lse; a.ws = tw.attn; a.ws_bytes = attn_workspace(s); a.err = err;
+  if (s.dtype == 0 && s.G * s.L_q <= 256 && attn_tc_supported(a)) {
+    cudaError_t e = launch_attn(a, st);
+    if (e != cudaSuccess) return e;
+    e = launch_sink_mass_tc(s, Q, q_idx, q_cnt, Kp, page_table, tw.lse, tw.mass, err, st);
+    if (e != cudaSuccess) return e;
+    SinkWs w = sink_ws(ws, s);
+    w.mass = tw.mass;
+    sink_topn_kernel<<<s.batch, 1024, 0, st>>>(s, n_sinks, w, sink_pos);
+    return cudaGetLastError();
+  }
   if (s.dtype == 0)
     return s.d == 128 ? run_sinks<__nv_bfloat16, 128>(s, Q, q_idx, q_cnt, Kp, page_table, Kd,
                                                       n_sinks, sink_pos, ws, err, st)
