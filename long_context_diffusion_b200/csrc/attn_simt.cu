@@ -150,10 +150,13 @@ attn_simt_kernel(AttnArgs a, int n_split, int tps) {
 
 // Merge the split partials of each (b, g, row): O = sum_s acc_s e^{m_s-M} / L,
 // L = sum_s l_s e^{m_s-M}, lse = M + ln L.  One warp per row.
+// Partials of (b, g) occupy slots [0, n_valid): all n_split slots for the
+// CUDA-core kernel (P == 0); for the persistent tensor-core kernel (S tile
+// slots per (b, g) split over P CTAs) the CTAs sharing the (b, g).
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 attn_combine_kernel(Shape s, int n_split, const void* ws, T* __restrict__ O,
-                    float* __restrict__ lse) {
+                    float* __restrict__ lse, int S, int P) {
   const int R = s.G * s.L_q;
   const long long n_rows = (long long)s.batch * s.H_kv * R;
   const long long gw = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -163,8 +166,17 @@ attn_combine_kernel(Shape s, int n_split, const void* ws, T* __restrict__ O,
   const int b = bg / s.H_kv, g = bg % s.H_kv;
   const int h = g * s.G + r / s.L_q, i = r % s.L_q;
   Partials part = partials_of(const_cast<void*>(ws), s, n_split);
+  int n_valid = n_split;
+  if (P > 0) {
+    const long long U = (long long)s.batch * s.H_kv * S;
+    const long long base = (long long)bg * S;
+    const long long c0 = ((base + 1) * P + U - 1) / U - 1;
+    const long long c1 = ((base + S) * P + U - 1) / U - 1;
+    n_valid = (int)(c1 - c0 + 1);
+    n_valid = n_valid < n_split ? n_valid : n_split;
+  }
   float M = -INFINITY;
-  for (int sp = 0; sp < n_split; ++sp)
+  for (int sp = 0; sp < n_valid; ++sp)
     M = fmaxf(M, part.ml[((size_t)bg * n_split + sp) * R + r].x);
   constexpr int CPL = D / 32;
   float o[CPL];
@@ -172,7 +184,7 @@ attn_combine_kernel(Shape s, int n_split, const void* ws, T* __restrict__ O,
   for (int c = 0; c < CPL; ++c) o[c] = 0.0f;
   float L = 0.0f;
   if (M != -INFINITY) {
-    for (int sp = 0; sp < n_split; ++sp) {
+    for (int sp = 0; sp < n_valid; ++sp) {
       const size_t row = ((size_t)bg * n_split + sp) * R + r;
       const float2 ml = part.ml[row];
       if (ml.x == -INFINITY) continue;
@@ -204,20 +216,21 @@ int attn_splits(const Shape& s, int max_tiles) {
 }
 
 template <typename T, int D>
-static cudaError_t run_combine(const AttnArgs& a, int n_split, cudaStream_t st) {
+static cudaError_t run_combine(const AttnArgs& a, int n_split, cudaStream_t st, int S, int P) {
   const Shape& s = a.s;
   const long long rows = (long long)s.batch * s.H_kv * s.G * s.L_q;
   attn_combine_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
-      s, n_split, a.ws, reinterpret_cast<T*>(a.O), a.lse);
+      s, n_split, a.ws, reinterpret_cast<T*>(a.O), a.lse, S, P);
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const AttnArgs& a, int n_split, cudaStream_t st) {
+cudaError_t launch_combine(const AttnArgs& a, int n_split, cudaStream_t st, int S = 0,
+                           int P = 0) {
   if (a.s.dtype == 1)
-    return a.s.d == 128 ? run_combine<float, 128>(a, n_split, st)
-                        : run_combine<float, 64>(a, n_split, st);
-  return a.s.d == 128 ? run_combine<__nv_bfloat16, 128>(a, n_split, st)
-                      : run_combine<__nv_bfloat16, 64>(a, n_split, st);
+    return a.s.d == 128 ? run_combine<float, 128>(a, n_split, st, S, P)
+                        : run_combine<float, 64>(a, n_split, st, S, P);
+  return a.s.d == 128 ? run_combine<__nv_bfloat16, 128>(a, n_split, st, S, P)
+                      : run_combine<__nv_bfloat16, 64>(a, n_split, st, S, P);
 }
 
 template <typename T, int D>

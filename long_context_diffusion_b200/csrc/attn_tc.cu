@@ -6,14 +6,23 @@
 //
 // One CTA per (split, b, g).  Its tiles are 64-key pages: the selected
 // context blocks (through the page table) and then the decode block.  Roles:
-//   warp 0, one thread : TMA producer -- Q once, then K and V of each tile
-//                        into a ring of ST shared-memory stages (128-byte
-//                        swizzle; the pool is a 2-D tensor map of 64-row
-//                        pages, so a gathered block is just a coordinate);
+//   warp 0, one thread : TMA producer of Q (per segment) and of the K ring;
+//   warp 2, one thread : TMA producer of the V ring (128-byte swizzle; the
+//                        pool is a 2-D tensor map of 64-row pages, so a
+//                        gathered block is just a coordinate; a K slot is
+//                        freed when its S is done, a V slot when its P V is);
 //   warp 1, one thread : tcgen05.mma issuer -- S = Q K^T into TMEM (two
 //                        buffers), then O += P V into TMEM;
-//   warps 4.. (128 per M-tile of 128 query rows): softmax -- one thread per
-//                        query row reads its S row from TMEM, keeps a running
+//   warps 4.. (4 per M-tile of 128 rows): softmax -- one thread per TMEM
+//                        lane.  With at most 32 (64) query rows, the M-tile
+//                        holds 4 (2) replicas of them, one per lane quadrant
+//                        (pair), so that all four SM sub-partitions work:
+//                        replica c takes columns [c*64/REP, (c+1)*64/REP) of
+//                        each tile, the row maximum is exchanged through
+//                        shared memory, and each replica writes its P columns
+//                        into every replica block, so every replica's O row
+//                        is complete; replica c rescales and writes out only
+//                        its share of O's columns.  Each thread keeps a running
 //                        max (lazy rescale: O and l are rescaled only when the
 //                        max grows by more than 2^8) and sum, writes P (bf16)
 //                        to shared memory in the MMA's K-major swizzled
@@ -39,25 +48,46 @@ namespace dl {
 using namespace sm100;
 
 constexpr int kTcMaxTiles = 1024;  // tiles of one CTA (tile table in shared memory)
+constexpr int kMaxSegs = 64;       // (b, g) segments of one CTA
 
-template <int D, int NM, int ST, int PB>
+// D head dim, NM M-tiles of 128 rows, REP replicas of the query rows in an
+// M-tile (4: at most 32 rows, 2: at most 64, 1 otherwise), ST K/V stages, QB
+// Q buffers and OB O accumulators (2 = the next segment starts while the
+// previous one is written out).
+template <int D, int NM, int REP, int ST, int QB, int OB>
 struct TcCfg {
+  static constexpr int PB = 2;                             // P buffers
   static constexpr int HALVES = D / 64;                    // 128-byte column chunks
-  static constexpr int Q_BYTES = NM * HALVES * 128 * 128;  // [m][half][128 rows][128 B]
+  static constexpr int Q_TILE = NM * HALVES * 128 * 128;   // [m][half][128 rows][128 B]
   static constexpr int KT_BYTES = HALVES * 64 * 128;       // [half][64 rows][128 B]
-  static constexpr int STAGE_BYTES = 2 * KT_BYTES;         // K tile, then V tile
+  static constexpr int RING_BYTES = ST * KT_BYTES;         // one ring of K (or V) tiles
   static constexpr int P_TILE = 128 * 128;                 // [128 rows][64 keys bf16]
-  static constexpr int P_BYTES = PB * NM * P_TILE;
-  static constexpr int BAR_OFF = Q_BYTES + ST * STAGE_BYTES + P_BYTES;
-  static constexpr int N_BARS = 2 * ST + 1 + 2 + 2 + 2;
-  static constexpr int MISC_OFF = BAR_OFF + N_BARS * 8;
-  static constexpr int TILE_OFF = MISC_OFF + 16;
-  static constexpr int SMEM = TILE_OFF + 2 * kTcMaxTiles * 4 + 1024;  // + alignment slack
-  static constexpr int THREADS = 128 + 128 * NM;
-  static constexpr uint32_t TMEM_NEED = NM * D + 2 * NM * 64;
+  static constexpr int RB = 128 / REP;                     // rows per replica block
+  static constexpr int NC = 64 / REP;                      // S columns per softmax thread
+  static constexpr int OC = D / REP;                       // O columns per softmax thread
+  static constexpr int SOFTMAX_THREADS = 128 * NM;
+  static constexpr int KV_OFF = QB * Q_TILE;
+  static constexpr int P_OFF = KV_OFF + 2 * RING_BYTES;    // K ring, then V ring
+  static constexpr int RED_OFF = P_OFF + PB * NM * P_TILE;
+  static constexpr int RED_BYTES = 3 * 128 * 4;            // tile maxima x2, final sums
+  static constexpr int BAR_OFF = RED_OFF + RED_BYTES;
+  // full_k, empty_k, full_v, empty_v [ST]; q_full, q_free [2]; s_full,
+  // p_ready [2]; pv_done [2]; o_free [2]; xbar [2][NM][4]; lbar [NM][4]
+  static constexpr int N_BARS = 4 * ST + 2 + 2 + 2 + 2 + 2 + 2 + 3 * NM * 4;
+  static constexpr int MISC_OFF = (BAR_OFF + N_BARS * 8 + 15) / 16 * 16;
+  static constexpr int TILE_OFF = MISC_OFF + 16;                   // int2 [kTcMaxTiles]
+  static constexpr int SEG_OFF = TILE_OFF + kTcMaxTiles * 8;       // int4 [kMaxSegs]
+  static constexpr int SEGLO_OFF = SEG_OFF + kMaxSegs * 16;        // int [kMaxSegs]
+  static constexpr int MARK_OFF = SEGLO_OFF + kMaxSegs * 4;        // int2 [kMaxSegs]
+  static_assert(BAR_OFF % 16 == 0 && TILE_OFF % 16 == 0 && SEG_OFF % 16 == 0, "alignment");
+  static constexpr int SMEM = MARK_OFF + kMaxSegs * 8 + 1024;      // + alignment slack
+  static constexpr int THREADS = 128 + SOFTMAX_THREADS;
+  static constexpr uint32_t TMEM_NEED = OB * NM * D + 2 * NM * 64;
   static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(TMEM_NEED <= 512, "tensor memory budget");
+  static_assert(NC >= 16 && OC >= 16, "column split");
+  static_assert(REP == 1 || NM == 1, "replicas only within one M-tile");
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -76,75 +106,140 @@ __device__ __forceinline__ int ctx_tile_block(const AttnArgs& a, int bg, int til
   return j;
 }
 
-template <int D, int NM, int ST, int PB>
+// Persistent work split over tile slots: slot u = (bg, t) = (u / S, u % S)
+// with S = the largest tile count of any (b, g); the slot holds a tile when
+// t < n_tiles(bg).  CTA c owns slots [c*U/P, (c+1)*U/P) of U = n_bg*S, so the
+// CTAs share the work within one tile.  The run of one (b, g) inside a CTA is
+// a segment: one accumulator and one partial, at partial slot c - first(bg),
+// where first(bg) is the CTA owning slot (bg, 0); a CTA whose run of a (b, g)
+// holds no tile writes an empty marker (m = -inf) there instead.
+struct TcPlan {
+  int S;      // tile slots per (b, g)
+  int nslot;  // partial slots per (b, g) (at most ceil(P / n_bg) + 1)
+};
+
+// CTA owning tile slot u when U slots are split over P CTAs.
+__host__ __device__ inline int tc_owner(long long u, long long U, int P) {
+  return (int)(((u + 1) * P + U - 1) / U) - 1;
+}
+
+template <int D, int NM, int REP, int ST, int QB, int OB>
 __global__ void __launch_bounds__(128 + 128 * NM, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kd,
-               const __grid_constant__ CUtensorMap tm_vd, const AttnArgs a, const int n_split,
-               const int tps) {
-  using C = TcCfg<D, NM, ST, PB>;
+               const __grid_constant__ CUtensorMap tm_vd, const AttnArgs a, const TcPlan plan) {
+  using C = TcCfg<D, NM, REP, ST, QB, OB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sQ = smem;
-  uint8_t* sKV = smem + C::Q_BYTES;
-  uint8_t* sP = sKV + ST * C::STAGE_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
-  uint64_t* empty = full + ST;
-  uint64_t* qbar = empty + ST;
-  uint64_t* s_full = qbar + 1;     // [2]  S buffer written
-  uint64_t* p_ready = s_full + 2;  // [2]  P written, O rescaled (128*NM arrivals)
-  uint64_t* pv_done = p_ready + 2; // [PB] P V of the buffer's last tile done
+  uint8_t* sK = smem + C::KV_OFF;               // K ring [ST][KT_BYTES]
+  uint8_t* sV = sK + C::RING_BYTES;              // V ring [ST][KT_BYTES]
+  uint8_t* sP = smem + C::P_OFF;
+  float* s_red = reinterpret_cast<float*>(smem + C::RED_OFF);  // [2][RB][REP]
+  float* s_lsum = s_red + 2 * 128;                             // [RB][REP]
+  // K and V travel in separate rings: a K slot is free once its S = Q K^T is
+  // done, a V slot once its P V is done, so neither waits for the softmax
+  uint64_t* full_k = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* empty_k = full_k + ST;
+  uint64_t* full_v = empty_k + ST;
+  uint64_t* empty_v = full_v + ST;
+  uint64_t* q_full = empty_v + ST;   // [2] Q of a segment landed
+  uint64_t* q_free = q_full + 2;     // [2] every MMA of a segment done (Q reusable)
+  uint64_t* s_full = q_free + 2;     // [2] S buffer written
+  uint64_t* p_ready = s_full + 2;    // [2] P written, O rescaled
+  uint64_t* pv_done = p_ready + 2;   // [2] P V of the tiles of that parity done
+  uint64_t* o_free = pv_done + 2;    // [2] segment's O read out
+  uint64_t* xbar = o_free + 2;       // [2][NM][4] tile-max exchange
+  uint64_t* lbar = xbar + 2 * NM * 4;  // [NM][4] final-sum exchange
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
-  int* t_y = reinterpret_cast<int*>(smem + C::TILE_OFF);
-  int* t_valid = t_y + kTcMaxTiles;
+  int* s_nt = reinterpret_cast<int*>(smem + C::MISC_OFF + 8);
+  int* s_nseg = s_nt + 1;
+  int2* t_info = reinterpret_cast<int2*>(smem + C::TILE_OFF);  // (y, valid | seg << 16)
+  int4* seg = reinterpret_cast<int4*>(smem + C::SEG_OFF);      // (bg, slot, first, n)
+  int* seg_lo = reinterpret_cast<int*>(smem + C::SEGLO_OFF);   // first tile index in (b, g)
+  int2* mark = reinterpret_cast<int2*>(smem + C::MARK_OFF);    // (bg, slot) of empty runs
+  int* s_nmark = s_nt + 2;
 
   const Shape& s = a.s;
-  const int bg = blockIdx.y, sp = blockIdx.x;
-  const int b = bg / s.H_kv, g = bg % s.H_kv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_ctx = ctx_tile_count(a, bg);
-  const int n_tiles = n_ctx + (s.L_q + 63) / 64;
-  const int t0 = sp * tps;
-  const int nt = max(0, min(t0 + tps, n_tiles) - t0);
   const int R = s.G * s.L_q;
+  const int n_dec = (s.L_q + 63) / 64;
+  const long long U = (long long)s.batch * s.H_kv * plan.S;
+  const long long u0 = (long long)blockIdx.x * U / gridDim.x;
+  const long long u1 = (long long)(blockIdx.x + 1) * U / gridDim.x;
+  Partials part = partials_of(a.ws, s, plan.nslot);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < ST; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
-    }
-    mbar_init(qbar, 1);
+    for (int i = 0; i < 4 * ST; ++i) mbar_init(&full_k[i], 1);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_free[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_ready[i], 128 * NM);
+      mbar_init(&p_ready[i], C::SOFTMAX_THREADS);
+      mbar_init(&o_free[i], C::SOFTMAX_THREADS);
       mbar_init(&pv_done[i], 1);
     }
+    for (int i = 0; i < 3 * NM * 4; ++i) mbar_init(&xbar[i], 128);
     *abort_flag = 0;
     fence_mbar_init();
-  }
-  // Tile table: TMA row coordinate and number of valid keys of every tile.
-  for (int t = threadIdx.x; t < nt; t += blockDim.x) {
-    const int tile = t0 + t;
-    int y = 0, valid = 0;
-    if (tile < n_ctx) {
-      const int j = ctx_tile_block(a, bg, tile);
-      if (j >= 0) {
-        const int slot = a.page_table[(size_t)b * s.n_pages + j];
-        if (slot < 0 || slot >= s.n_slots) {
-          flag_error(a.err, ERR_BAD_INDEX);
+    // runs of (b, g) in this CTA's slots: segments (with tiles) and markers
+    int nseg = 0, nmark = 0, ntile = 0;
+    if (u1 > u0) {
+      for (int bg = (int)(u0 / plan.S); bg <= (int)((u1 - 1) / plan.S); ++bg) {
+        const long long base = (long long)bg * plan.S;
+        const int lo = (int)max(u0 - base, 0ll);
+        const int hi = (int)min(u1 - base, (long long)plan.S);
+        const int n_tiles = ctx_tile_count(a, bg) + n_dec;
+        const int thi = min(hi, n_tiles);
+        const int slot = (int)blockIdx.x - tc_owner(base, U, gridDim.x);
+        if (thi > lo) {
+          seg[nseg] = make_int4(bg, slot, ntile, thi - lo);
+          seg_lo[nseg] = lo;
+          ++nseg;
+          ntile += thi - lo;
         } else {
-          valid = min(64, s.L_ctx - j * 64);
-          y = (slot * s.H_kv + g) * 64;
+          mark[nmark++] = make_int2(bg, slot);
         }
       }
-    } else {
-      const int td = tile - n_ctx;
-      valid = min(64, s.L_q - td * 64);
-      y = td * 64;
     }
-    t_y[t] = y;
-    t_valid[t] = valid;
+    *s_nt = ntile;
+    *s_nseg = nseg;
+    *s_nmark = nmark;
+  }
+  __syncthreads();
+  const int nt = *s_nt, nseg = *s_nseg, nmark = *s_nmark;
+  for (int e = threadIdx.x; e < nmark * R; e += blockDim.x) {
+    const int2 mk = mark[e / R];
+    part.ml[((size_t)mk.x * plan.nslot + mk.y) * R + e % R] = make_float2(-INFINITY, 0.0f);
+  }
+  // tile table: TMA row coordinate, valid keys, segment
+  for (int k = 0; k < nseg; ++k) {
+    const int bg = seg[k].x;
+    const int b = bg / s.H_kv, g = bg % s.H_kv;
+    const int n_ctx = ctx_tile_count(a, bg);
+    const int lo = seg_lo[k];
+    for (int t = threadIdx.x; t < seg[k].w; t += blockDim.x) {
+      const int tile = lo + t;
+      int y = 0, valid = 0;
+      if (tile < n_ctx) {
+        const int j = ctx_tile_block(a, bg, tile);
+        if (j >= 0) {
+          const int slot = a.page_table[(size_t)b * s.n_pages + j];
+          if (slot < 0 || slot >= s.n_slots) {
+            flag_error(a.err, ERR_BAD_INDEX);
+          } else {
+            valid = min(64, s.L_ctx - j * 64);
+            y = (slot * s.H_kv + g) * 64;
+          }
+        }
+      } else {
+        const int td = tile - n_ctx;
+        valid = min(64, s.L_q - td * 64) | (1 << 15);  // bit 15: decode tile
+        y = td * 64;
+      }
+      t_info[seg[k].z + t] = make_int2(y, valid | (k << 16));
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -154,43 +249,70 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  auto tile_seg = [&](int i) { return t_info[i].y >> 16; };
+  auto tile_valid = [&](int i) { return t_info[i].y & 0x7F; };
+  auto tile_dec = [&](int i) { return (t_info[i].y >> 15) & 1; };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------ producers
+    // warp 0: Q of every segment and the K ring; warp 2: the V ring
+    const bool is_k = warp == 0;
+    uint64_t* full = is_k ? full_k : full_v;
+    uint64_t* empty = is_k ? empty_k : empty_v;
+    uint8_t* ring = is_k ? sK : sV;
+    const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+    const CUtensorMap* map_dec = is_k ? &tm_kd : &tm_vd;
     if (lane == 0 && nt > 0) {
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(qbar, C::Q_BYTES);
-      const int q_row0 = (b * s.H + g * s.G) * s.L_q;
-      for (int m = 0; m < NM; ++m)
-        for (int h = 0; h < C::HALVES; ++h)
-          tma_load_2d(sQ + (m * C::HALVES + h) * 16384, &tm_q, h * 64, q_row0 + m * 128, qbar);
-      for (int i = 0; i < nt; ++i) {
+      prefetch_tmap(map);
+      prefetch_tmap(map_dec);
+      auto load_q = [&](int k) -> bool {
+        const int qb = QB == 2 ? (k & 1) : 0;
+        if (k >= QB) {  // the buffer's previous segment must be done with it
+          const int prev = k - QB;
+          if (!mbar_wait(&q_free[qb], (QB == 2 ? (prev >> 1) : prev) & 1, abort_flag))
+            return false;
+        }
+        const int bg = seg[k].x;
+        const int b = bg / s.H_kv, g = bg % s.H_kv;
+        const int q_row0 = (b * s.H + g * s.G) * s.L_q;
+        mbar_arrive_expect_tx(&q_full[qb], C::Q_TILE);
+        for (int m = 0; m < NM; ++m)
+          for (int h = 0; h < C::HALVES; ++h)
+            for (int c = 0; c < REP; ++c)  // replica c at rows [c*RB, (c+1)*RB)
+              tma_load_2d(sQ + qb * C::Q_TILE + (m * C::HALVES + h) * 16384 + c * C::RB * 128,
+                          &tm_q, h * 64, q_row0 + m * 128, &q_full[qb]);
+        return true;
+      };
+      int next_q = 0;  // next segment whose Q is to be loaded
+      bool ok = true;
+      for (int i = 0; ok && i < nt; ++i) {
+        const int k = tile_seg(i);
+        // a segment's Q is loaded with its first K tile
+        while (is_k && ok && next_q < nseg && next_q <= k) {
+          ok = load_q(next_q);
+          ++next_q;
+        }
+        if (!ok) break;
         const int st = i % ST;
         if (i >= ST && !mbar_wait(&empty[st], ((i / ST) - 1) & 1, abort_flag)) break;
-        uint8_t* sK = sKV + st * C::STAGE_BYTES;
-        uint8_t* sV = sK + C::KT_BYTES;
-        if (t_valid[i] > 0) {
-          mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
-          if (t0 + i < n_ctx) {
-            for (int h = 0; h < C::HALVES; ++h) {
-              tma_load_2d(sK + h * 8192, &tm_k, h * 64, t_y[i], &full[st]);
-              tma_load_2d(sV + h * 8192, &tm_v, h * 64, t_y[i], &full[st]);
-            }
+        uint8_t* dst = ring + st * C::KT_BYTES;
+        if (tile_valid(i) > 0) {
+          mbar_arrive_expect_tx(&full[st], C::KT_BYTES);
+          if (!tile_dec(i)) {
+            for (int h = 0; h < C::HALVES; ++h)
+              tma_load_2d(dst + h * 8192, map, h * 64, t_info[i].x, &full[st]);
           } else {
-            for (int h = 0; h < C::HALVES; ++h) {
-              tma_load_3d(sK + h * 8192, &tm_kd, h * 64, t_y[i], bg, &full[st]);
-              tma_load_3d(sV + h * 8192, &tm_vd, h * 64, t_y[i], bg, &full[st]);
-            }
+            const int bg = seg[k].x;
+            for (int h = 0; h < C::HALVES; ++h)
+              tma_load_3d(dst + h * 8192, map_dec, h * 64, t_info[i].x, bg, &full[st]);
           }
         } else {
           mbar_arrive(&full[st]);  // nothing to load: the tile is fully masked
         }
       }
-      // do not leave with copies in flight: wait for the last stages' loads
-      if (*abort_flag) {
+      if (*abort_flag) {  // do not leave with copies in flight
         for (int i = max(0, nt - ST); i < nt; ++i)
-          for (uint32_t k = 0; k < (1u << 20) && !mbar_try_wait(&full[i % ST], (i / ST) & 1); ++k) {
+          for (uint32_t t = 0; t < (1u << 20) && !mbar_try_wait(&full[i % ST], (i / ST) & 1); ++t) {
           }
       }
     }
@@ -199,95 +321,132 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (lane == 0 && nt > 0) {
       constexpr uint32_t IS = idesc_bf16_f32(128, 64, false);
       constexpr uint32_t IP = idesc_bf16_f32(128, D, true);
-      const uint32_t q_base = smem_u32(sQ), kv_base = smem_u32(sKV), p_base = smem_u32(sP);
-      bool ok = mbar_wait(qbar, 0, abort_flag);
-      tc_fence_after();
+      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
+      const uint32_t p_base = smem_u32(sP);
+      bool ok = true;
+      auto is_first = [&](int i) { return i == 0 || tile_seg(i - 1) != tile_seg(i); };
+      auto is_last = [&](int i) { return i == nt - 1 || tile_seg(i + 1) != tile_seg(i); };
       auto issue_s = [&](int i) -> bool {
+        const int k = tile_seg(i);
+        const int qb = QB == 2 ? (k & 1) : 0;
+        if (is_first(i) &&
+            !mbar_wait(&q_full[qb], (QB == 2 ? (k >> 1) : k) & 1, abort_flag))
+          return false;
         const int st = i % ST;
-        if (!mbar_wait(&full[st], (i / ST) & 1, abort_flag)) return false;
+        if (!mbar_wait(&full_k[st], (i / ST) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t kb = kv_base + st * C::STAGE_BYTES;
+        const uint32_t kb = k_base + st * C::KT_BYTES;
+        const uint32_t qbase = q_base + qb * C::Q_TILE;
         const int buf = i & 1;
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
-          const uint32_t d_t = tmem + NM * D + (buf * NM + m) * 64;
+          const uint32_t d_t = tmem + OB * NM * D + (buf * NM + m) * 64;
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const int h = k >> 2, kk = k & 3;
-            const uint64_t ad =
-                sdesc_sw128(q_base + (m * C::HALVES + h) * 16384 + kk * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(kb + h * 8192 + kk * 32, 16, 1024);
-            mma_f16_ss(d_t, ad, bd, IS, k > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int h = kk >> 2, k4 = kk & 3;
+            const uint64_t ad = sdesc_sw128(qbase + (m * C::HALVES + h) * 16384 + k4 * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(kb + h * 8192 + k4 * 32, 16, 1024);
+            mma_f16_ss(d_t, ad, bd, IS, kk > 0 ? 1u : 0u);
           }
         }
         mma_commit(&s_full[buf]);
+        mma_commit(&empty_k[st]);  // K is no longer needed once S is done
         return true;
       };
-      if (ok) ok = issue_s(0);
+      ok = issue_s(0);
       for (int i = 0; ok && i < nt; ++i) {
-        if (i + 1 < nt && !issue_s(i + 1)) break;
+        const int k = tile_seg(i);
+        // S of the next tile is issued ahead, unless it belongs to the next
+        // segment and both segments share the single Q buffer
+        const bool ahead = i + 1 < nt && (QB == 2 || !is_first(i + 1));
+        if (ahead && !(ok = issue_s(i + 1))) break;
         const int buf = i & 1;
-        if (!mbar_wait(&p_ready[buf], (i >> 1) & 1, abort_flag)) break;
-        tc_fence_after();
+        if (!(ok = mbar_wait(&p_ready[buf], (i >> 1) & 1, abort_flag))) break;
+        const bool first = is_first(i);
+        const int ob = OB == 2 ? (k & 1) : 0;
+        if (first && k >= OB &&
+            !(ok = mbar_wait(&o_free[ob], (OB == 2 ? ((k - OB) >> 1) : (k - OB)) & 1, abort_flag)))
+          break;
         const int st = i % ST;
-        const uint32_t vb = kv_base + st * C::STAGE_BYTES + C::KT_BYTES;
-        const int pbuf = PB == 2 ? buf : 0;
+        if (!(ok = mbar_wait(&full_v[st], (i / ST) & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t vb = v_base + st * C::KT_BYTES;
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
-          const uint32_t d_t = tmem + m * D;
-          const uint32_t pb = p_base + (pbuf * NM + m) * C::P_TILE;
+          const uint32_t d_t = tmem + (ob * NM + m) * D;
+          const uint32_t pb = p_base + (buf * NM + m) * C::P_TILE;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = sdesc_sw128(pb + k * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(vb + k * 2048, 8192, 1024);
-            mma_f16_ss(d_t, ad, bd, IP, (i > 0 || k > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = sdesc_sw128(pb + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(vb + kk * 2048, 8192, 1024);
+            mma_f16_ss(d_t, ad, bd, IP, (!first || kk > 0) ? 1u : 0u);
           }
         }
-        mma_commit(&empty[st]);
-        mma_commit(&pv_done[pbuf]);
+        mma_commit(&empty_v[st]);
+        mma_commit(&pv_done[buf]);
+        if (is_last(i)) mma_commit(&q_free[QB == 2 ? (k & 1) : 0]);
+        if (i + 1 < nt && !ahead && !(ok = issue_s(i + 1))) break;
       }
       if (*abort_flag) {  // give issued MMAs time to finish before TMEM is freed
-        for (uint32_t k = 0; k < (1u << 16); ++k) __nanosleep(1000);
+        for (uint32_t t = 0; t < (1u << 16); ++t) __nanosleep(1000);
       }
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
+    // thread -> TMEM lane `row` of M-tile m; replica `rp` of query row `qr`
     const int m = (warp - 4) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    const int r = m * 128 + row;
+    const int rp = row / C::RB;
+    const int qr = row % C::RB;
+    const int r = m * 128 + qr;
     const bool active = r < R;
+    const int col0 = rp * C::NC;
+    const int ocol0 = rp * C::OC;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t s_col = NM * D;
+    const uint32_t s_col = OB * NM * D;
     const float c2 = static_cast<float>(s.scale * 1.4426950408889634);
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = nt > 0;
-    // completion index of pv_done[x] for tile t is t / PB (PB buffers share tiles)
+    // pv_done[t & 1] completes once per tile of that parity: tile t is its
+    // completion t >> 1
     auto wait_pv = [&](int t) -> bool {
-      const bool w = mbar_wait(&pv_done[PB == 2 ? (t & 1) : 0], (PB == 2 ? (t >> 1) : t) & 1,
-                               abort_flag);
-      return __all_sync(0xffffffffu, w);
+      return __all_sync(0xffffffffu, mbar_wait(&pv_done[t & 1], (t >> 1) & 1, abort_flag));
     };
     for (int i = 0; ok && i < nt; ++i) {
+      const int k = tile_seg(i);
+      const int ob = OB == 2 ? (k & 1) : 0;
+      const uint32_t o_col = (ob * NM + m) * D;
+      const bool first = i == 0 || tile_seg(i - 1) != k;
+      const bool last = i == nt - 1 || tile_seg(i + 1) != k;
+      if (first) {
+        m_run = -INFINITY;
+        l_run = 0.0f;
+      }
       const int buf = i & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[buf], (i >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sv[64];
-      {
-        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
-        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
-        tmem_ld32(tmem + lane_base + s_col + (buf * NM + m) * 64, lo);
-        tmem_ld32(tmem + lane_base + s_col + (buf * NM + m) * 64 + 32, hi);
-        tmem_ld_wait();
-      }
-      const int valid = t_valid[i];
+      uint32_t sv[C::NC];
+      tmem_ld<C::NC>(tmem + lane_base + s_col + (buf * NM + m) * 64 + col0, sv);
+      tmem_ld_wait();
+      const int valid = tile_valid(i);
       float tmax = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float x = (active && c < valid) ? __uint_as_float(sv[c]) * c2 : -INFINITY;
+      for (int c = 0; c < C::NC; ++c) {
+        const float x = (active && col0 + c < valid) ? __uint_as_float(sv[c]) * c2 : -INFINITY;
         sv[c] = __float_as_uint(x);
         tmax = fmaxf(tmax, x);
+      }
+      if constexpr (REP > 1) {
+        // the row's maximum over the whole tile: exchange between replicas
+        float* red = s_red + buf * 128 + qr * REP;
+        red[rp] = tmax;
+        mbar_arrive(&xbar[buf]);
+        ok = __all_sync(0xffffffffu, mbar_wait(&xbar[buf], (i >> 1) & 1, abort_flag));
+        if (!ok) break;
+#pragma unroll
+        for (int q = 0; q < REP; ++q) tmax = fmaxf(tmax, red[q]);
       }
       const float m_new = fmaxf(m_run, tmax);
       const bool grow = m_new > m_run + 8.0f;
@@ -297,14 +456,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (!ok) break;
         tc_fence_after();
         const float alpha = live ? exp2f(m_run - m_new) : 1.0f;
+        constexpr int CH = C::OC < 32 ? C::OC : 32;
 #pragma unroll 1
-        for (int cc = 0; cc < D; cc += 32) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_base + m * D + cc, o);
+        for (int cc = 0; cc < C::OC; cc += CH) {
+          uint32_t o[CH];
+          tmem_ld<CH>(tmem + lane_base + o_col + ocol0 + cc, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st32(tmem + lane_base + m * D + cc, o);
+          for (int q = 0; q < CH; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+          tmem_st<CH>(tmem + lane_base + o_col + ocol0 + cc, o);
         }
         tmem_st_wait();
       }
@@ -312,10 +472,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         l_run = (m_run == -INFINITY) ? 0.0f : l_run * exp2f(m_run - m_new);
         m_run = m_new;
       }
-      uint32_t packed[32];
+      uint32_t packed[C::NC / 2];
       float psum = 0.0f;
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
+      for (int c = 0; c < C::NC; c += 2) {
         const float x0 = __uint_as_float(sv[c]), x1 = __uint_as_float(sv[c + 1]);
         const float p0 = (m_run == -INFINITY) ? 0.0f : ex2_approx(x0 - m_run);
         const float p1 = (m_run == -INFINITY) ? 0.0f : ex2_approx(x1 - m_run);
@@ -323,56 +483,79 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         packed[c >> 1] = pack_bf16x2(p0, p1);
       }
       l_run += psum;
-      // the P buffer is free once the P V that last read it is done
-      if (i >= PB) {
-        ok = wait_pv(i - PB);
+      // the P buffer is free once the P V that last read it (tile i-2) is done
+      if (i >= 2) {
+        ok = wait_pv(i - 2);
         if (!ok) break;
       }
-      uint8_t* prow = sP + ((PB == 2 ? buf : 0) * NM + m) * C::P_TILE + row * 128;
+      // this replica's columns, into the P row of every replica block
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) =
-            make_uint4(packed[4 * ch], packed[4 * ch + 1], packed[4 * ch + 2], packed[4 * ch + 3]);
+      for (int blk = 0; blk < REP; ++blk) {
+        const int prow_idx = blk * C::RB + qr;
+        uint8_t* prow = sP + (buf * NM + m) * C::P_TILE + prow_idx * 128;
+#pragma unroll
+        for (int q = 0; q < C::NC / 8; ++q) {
+          const int ch = col0 / 8 + q;
+          *reinterpret_cast<uint4*>(prow + ((ch ^ (prow_idx & 7)) << 4)) =
+              make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+        }
       }
       if (m == 0 && valid < 64) {
         // rows past the valid keys may hold anything (even NaN): zero V there
-        uint8_t* sV = sKV + (i % ST) * C::STAGE_BYTES + C::KT_BYTES;
+        // once it has landed
+        ok = __all_sync(0xffffffffu, mbar_wait(&full_v[i % ST], (i / ST) & 1, abort_flag));
+        if (!ok) break;
+        uint8_t* sVt = sV + (i % ST) * C::KT_BYTES;
         const int per_row = C::HALVES * 8;
         const int nz = (64 - valid) * per_row;
         for (int e = row; e < nz; e += 128) {
           const int rr = valid + e / per_row, rem = e % per_row;
-          *reinterpret_cast<uint4*>(sV + (rem >> 3) * 8192 + rr * 128 + (rem & 7) * 16) =
+          *reinterpret_cast<uint4*>(sVt + (rem >> 3) * 8192 + rr * 128 + (rem & 7) * 16) =
               make_uint4(0u, 0u, 0u, 0u);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_ready[buf]);
-    }
-    // epilogue: unnormalised partial O, running max (natural log) and sum
-    Partials part = partials_of(a.ws, s, n_split);
-    const size_t prow = ((size_t)bg * n_split + sp) * R + r;
-    if (ok) ok = wait_pv(nt - 1);
-    if (ok) {
+      if (!last) continue;
+      // ---- segment epilogue: unnormalised partial O, running max and sum
+      ok = wait_pv(i);
+      if (!ok) break;
       tc_fence_after();
+      const int bg = seg[k].x;
+      const size_t prow_i = ((size_t)bg * plan.nslot + seg[k].y) * R + r;
+      constexpr int CH = C::OC < 32 ? C::OC : 32;
 #pragma unroll 1
-      for (int cc = 0; cc < D; cc += 32) {
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_base + m * D + cc, o);
+      for (int cc = 0; cc < C::OC; cc += CH) {
+        uint32_t o[CH];
+        tmem_ld<CH>(tmem + lane_base + o_col + ocol0 + cc, o);
         tmem_ld_wait();
         if (active) {
-          float4* dst = reinterpret_cast<float4*>(part.o + prow * D + cc);
+          float4* dst = reinterpret_cast<float4*>(part.o + prow_i * D + ocol0 + cc);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            dst[k] = make_float4(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]),
-                                 __uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3]));
+          for (int q = 0; q < CH / 4; ++q)
+            dst[q] = make_float4(__uint_as_float(o[4 * q]), __uint_as_float(o[4 * q + 1]),
+                                 __uint_as_float(o[4 * q + 2]), __uint_as_float(o[4 * q + 3]));
         }
       }
-    }
-    if (active) {
-      const bool any = ok && m_run != -INFINITY;
-      part.ml[prow] = make_float2(any ? m_run * 0.69314718055994531f : -INFINITY,
-                                  any ? l_run : 0.0f);
+      tc_fence_before();
+      mbar_arrive(&o_free[ob]);
+      float l_tot = l_run;
+      if constexpr (REP > 1) {
+        float* ls = s_lsum + qr * REP;
+        ls[rp] = l_run;
+        mbar_arrive(lbar);
+        ok = __all_sync(0xffffffffu, mbar_wait(lbar, k & 1, abort_flag));
+        if (!ok) break;
+        l_tot = 0.0f;
+#pragma unroll
+        for (int q = 0; q < REP; ++q) l_tot += ls[q];
+        // the sums are read before the next segment writes them: the next
+        // write follows at least one tile-maximum exchange of every replica
+      }
+      if (active && rp == 0)
+        part.ml[prow_i] = make_float2(m_run == -INFINITY ? -INFINITY : m_run * 0.69314718055994531f,
+                                      m_run == -INFINITY ? 0.0f : l_tot);
     }
   }
   if (threadIdx.x == 0 && *abort_flag) flag_error(a.err, ERR_TIMEOUT);
@@ -447,50 +630,62 @@ int tc_sm_count() {
 
 namespace {
 
-// Splits per (b, g): minimise waves x (tiles per CTA + fixed cost), one CTA
-// per SM resident.
-int tc_splits(int bgs, int max_tiles, int sms) {
-  int best = 1;
-  double best_cost = 1e30;
-  for (int n = 1; n <= kMaxSplits && n <= max_tiles; ++n) {
-    const int tps = (max_tiles + n - 1) / n;
-    if (tps > kTcMaxTiles) continue;
-    const long long ctas = (long long)bgs * n;
-    const long long waves = (ctas + sms - 1) / sms;
-    const double cost = (double)waves * (tps + 6.0);
-    if (cost < best_cost - 1e-9) {
-      best_cost = cost;
-      best = n;
-    }
+// Work split of the persistent kernel: one CTA per SM (more when the tile
+// table of a CTA would overflow), S = the largest tile count of a (b, g).
+struct TcLaunch {
+  TcPlan plan;
+  int grid;
+};
+
+TcLaunch tc_plan(int n_bg, int max_tiles, int sms) {
+  TcLaunch L;
+  L.plan.S = max_tiles;
+  const long long U = (long long)n_bg * max_tiles;
+  long long grid = U < sms ? U : sms;
+  // partial slots per (b, g) stay within the workspace's kMaxSplits
+  const long long cap = (long long)n_bg * (kMaxSplits - 2);
+  grid = grid < cap ? grid : cap;
+  // a CTA's tile table and its (b, g) runs must fit in shared memory
+  if ((U + grid - 1) / grid > kTcMaxTiles) grid = (U + kTcMaxTiles - 1) / kTcMaxTiles;
+  const long long per_seg = (long long)(kMaxSegs - 1) * max_tiles;
+  if ((U + grid - 1) / grid > per_seg) grid = (U + per_seg - 1) / per_seg;
+  L.grid = (int)grid;
+  // CTAs that share one (b, g): those owning its first and last slots
+  int nslot = 1;
+  for (int bg = 0; bg < n_bg; ++bg) {
+    const int n = tc_owner((long long)bg * max_tiles + max_tiles - 1, U, L.grid) -
+                  tc_owner((long long)bg * max_tiles, U, L.grid) + 1;
+    nslot = n > nslot ? n : nslot;
   }
-  return best;
+  L.plan.nslot = nslot;
+  return L;
 }
 
 }  // namespace
 
-cudaError_t launch_combine(const AttnArgs& a, int n_split, cudaStream_t st);
+cudaError_t launch_combine(const AttnArgs& a, int n_split, cudaStream_t st, int S = 0,
+                           int P = 0);
 
-template <int D, int NM, int ST, int PB>
+template <int D, int NM, int REP, int ST, int QB, int OB>
 static cudaError_t run_tc(const AttnArgs& a, int max_tiles, cudaStream_t st) {
-  using C = TcCfg<D, NM, ST, PB>;
+  using C = TcCfg<D, NM, REP, ST, QB, OB>;
   const Shape& s = a.s;
   CUtensorMap mq, mk, mv, mkd, mvd;
   const uint64_t pool_rows = (uint64_t)s.n_slots * s.H_kv * 64;
   const uint64_t q_rows = (uint64_t)s.batch * s.H * s.L_q;
   const uint64_t n_bg = (uint64_t)s.batch * s.H_kv;
-  if (!tc_map_2d(&mq, a.Q, D, q_rows, 128) || !tc_map_2d(&mk, a.Kp, D, pool_rows, 64) ||
+  if (!tc_map_2d(&mq, a.Q, D, q_rows, C::RB) || !tc_map_2d(&mk, a.Kp, D, pool_rows, 64) ||
       !tc_map_2d(&mv, a.Vp, D, pool_rows, 64) || !map_3d(&mkd, a.Kd, D, s.L_q, n_bg) ||
       !map_3d(&mvd, a.Vd, D, s.L_q, n_bg))
     return cudaErrorInvalidValue;
-  const int n_split = tc_splits((int)n_bg, max_tiles, tc_sm_count());
-  const int tps = (max_tiles + n_split - 1) / n_split;
-  auto kern = attn_tc_kernel<D, NM, ST, PB>;
+  const TcLaunch L = tc_plan((int)n_bg, max_tiles, tc_sm_count());
+  if (L.plan.nslot > kMaxSplits) return cudaErrorInvalidValue;  // workspace bound
+  auto kern = attn_tc_kernel<D, NM, REP, ST, QB, OB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(n_split, (unsigned)n_bg), C::THREADS, C::SMEM, st>>>(mq, mk, mv, mkd, mvd, a,
-                                                                   n_split, tps);
+  kern<<<L.grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mkd, mvd, a, L.plan);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  return launch_combine(a, n_split, st);
+  return launch_combine(a, L.plan.nslot, st, L.plan.S, L.grid);
 }
 
 // Whether the tensor-core kernel takes this call (bf16, block or dense keys,
@@ -504,10 +699,17 @@ bool attn_tc_supported(const AttnArgs& a) {
 
 cudaError_t launch_attn_tc(const AttnArgs& a, int max_tiles, cudaStream_t st) {
   const Shape& s = a.s;
-  const int nm = (s.G * s.L_q + 127) / 128;
-  if (s.d == 128)
-    return nm == 1 ? run_tc<128, 1, 4, 2>(a, max_tiles, st) : run_tc<128, 2, 3, 1>(a, max_tiles, st);
-  return nm == 1 ? run_tc<64, 1, 6, 2>(a, max_tiles, st) : run_tc<64, 2, 4, 2>(a, max_tiles, st);
+  const int R = s.G * s.L_q;
+  if (s.d == 128) {
+    if (R > 128) return run_tc<128, 2, 1, 2, 1, 1>(a, max_tiles, st);
+    if (R > 64) return run_tc<128, 1, 1, 4, 1, 2>(a, max_tiles, st);
+    if (R > 32) return run_tc<128, 1, 2, 4, 1, 2>(a, max_tiles, st);
+    return run_tc<128, 1, 4, 4, 1, 2>(a, max_tiles, st);
+  }
+  if (R > 128) return run_tc<64, 2, 1, 4, 1, 2>(a, max_tiles, st);
+  if (R > 64) return run_tc<64, 1, 1, 6, 1, 2>(a, max_tiles, st);
+  if (R > 32) return run_tc<64, 1, 2, 6, 1, 2>(a, max_tiles, st);
+  return run_tc<64, 1, 4, 6, 1, 2>(a, max_tiles, st);
 }
 
 }  // namespace dl
