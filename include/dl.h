@@ -212,8 +212,9 @@ dl_status dl_sparse_attn_gather(const dl_attn_desc* desc, const void* Q_dec, con
  * whose footprint is fixed after start-up).
  * Same arguments and results as dl_block_scores, minus the workspace: the
  * scratch is a 32 MiB array built into the library (held on every GPU that
- * loads it until exit).  Calls needing more, i.e. with
- * batch*H*L_q*n_units*8 > 32 MiB, return DL_ERR_WORKSPACE.  All calls on a
+ * loads it until exit).  Calls needing more return DL_ERR_WORKSPACE; the
+ * need is batch*H*L_q*(8*n128 + 16*n128/128) bytes, n128 = n_units rounded
+ * up to a multiple of 128.  All calls on a
  * device share the array; calls whose kernels may overlap on the GPU race on
  * it and must be ordered (one stream).  The first call on each device looks
  * up the array's device address, so make it before any stream capture.  The

@@ -11,8 +11,12 @@
 //                        pool is a 2-D tensor map of 64-row pages, so a
 //                        gathered block is just a coordinate; a K slot is
 //                        freed when its S is done, a V slot when its P V is);
-//   warp 1, one thread : tcgen05.mma issuer -- S = Q K^T into TMEM (two
-//                        buffers), then O += P V into TMEM;
+//   warp 1, one thread : tcgen05.mma issuer of S = Q K^T into TMEM (two
+//                        buffers; a buffer is reused once the softmax of the
+//                        tile two back has read it);
+//   warp 3, one thread : tcgen05.mma issuer of O += P V into TMEM (each
+//                        issuer has its own chain of waits, so the two
+//                        streams of MMAs overlap);
 //   warps 4.. (4 per M-tile of 128 rows): softmax -- one thread per TMEM
 //                        lane.  With at most 32 (64) query rows, the M-tile
 //                        holds 4 (2) replicas of them, one per lane quadrant
@@ -34,21 +38,14 @@
 // Every wait is bounded: a role that gives up raises the shared abort flag
 // and the device error word (ERR_TIMEOUT) and leaves its loop; the CTA then
 // frees its TMEM and returns.
-#include <cudaTypedefs.h>
-
 #include <mutex>
 
-#include "common.cuh"
-#include "internal.h"
 #include "sm100.cuh"
-#include "tiles.cuh"
+#include "tc_common.cuh"
 
 namespace dl {
 
 using namespace sm100;
-
-constexpr int kTcMaxTiles = 1024;  // tiles of one CTA (tile table in shared memory)
-constexpr int kMaxSegs = 64;       // (b, g) segments of one CTA
 
 // D head dim, NM M-tiles of 128 rows, REP replicas of the query rows in an
 // M-tile (4: at most 32 rows, 2: at most 64, 1 otherwise), ST K/V stages, QB
@@ -90,39 +87,6 @@ struct TcCfg {
   static_assert(REP == 1 || NM == 1, "replicas only within one M-tile");
 };
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Block index of context tile `tile` of (b, g), or -1 (bad index, flagged).
-__device__ __forceinline__ int ctx_tile_block(const AttnArgs& a, int bg, int tile) {
-  if (a.mode == kDense) return tile;
-  const int j = a.idx[(size_t)bg * a.max_idx + tile];
-  if (j < 0 || j >= n_blocks(a.s)) {
-    flag_error(a.err, ERR_BAD_INDEX);
-    return -1;
-  }
-  return j;
-}
-
-// Persistent work split over tile slots: slot u = (bg, t) = (u / S, u % S)
-// with S = the largest tile count of any (b, g); the slot holds a tile when
-// t < n_tiles(bg).  CTA c owns slots [c*U/P, (c+1)*U/P) of U = n_bg*S, so the
-// CTAs share the work within one tile.  The run of one (b, g) inside a CTA is
-// a segment: one accumulator and one partial, at partial slot c - first(bg),
-// where first(bg) is the CTA owning slot (bg, 0); a CTA whose run of a (b, g)
-// holds no tile writes an empty marker (m = -inf) there instead.
-struct TcPlan {
-  int S;      // tile slots per (b, g)
-  int nslot;  // partial slots per (b, g) (at most ceil(P / n_bg) + 1)
-};
-
-// CTA owning tile slot u when U slots are split over P CTAs.
-__host__ __device__ inline int tc_owner(long long u, long long U, int P) {
-  return (int)(((u + 1) * P + U - 1) / U) - 1;
-}
-
 template <int D, int NM, int REP, int ST, int QB, int OB>
 __global__ void __launch_bounds__(128 + 128 * NM, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -144,7 +108,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint64_t* full_v = empty_k + ST;
   uint64_t* empty_v = full_v + ST;
   uint64_t* q_full = empty_v + ST;   // [2] Q of a segment landed
-  uint64_t* q_free = q_full + 2;     // [2] every MMA of a segment done (Q reusable)
+  uint64_t* q_free = q_full + 2;     // [2] every S of a segment done (Q reusable)
   uint64_t* s_full = q_free + 2;     // [2] S buffer written
   uint64_t* p_ready = s_full + 2;    // [2] P written, O rescaled
   uint64_t* pv_done = p_ready + 2;   // [2] P V of the tiles of that parity done
@@ -216,29 +180,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   // tile table: TMA row coordinate, valid keys, segment
   for (int k = 0; k < nseg; ++k) {
     const int bg = seg[k].x;
-    const int b = bg / s.H_kv, g = bg % s.H_kv;
     const int n_ctx = ctx_tile_count(a, bg);
     const int lo = seg_lo[k];
     for (int t = threadIdx.x; t < seg[k].w; t += blockDim.x) {
-      const int tile = lo + t;
-      int y = 0, valid = 0;
-      if (tile < n_ctx) {
-        const int j = ctx_tile_block(a, bg, tile);
-        if (j >= 0) {
-          const int slot = a.page_table[(size_t)b * s.n_pages + j];
-          if (slot < 0 || slot >= s.n_slots) {
-            flag_error(a.err, ERR_BAD_INDEX);
-          } else {
-            valid = min(64, s.L_ctx - j * 64);
-            y = (slot * s.H_kv + g) * 64;
-          }
-        }
-      } else {
-        const int td = tile - n_ctx;
-        valid = min(64, s.L_q - td * 64) | (1 << 15);  // bit 15: decode tile
-        y = td * 64;
-      }
-      t_info[seg[k].z + t] = make_int2(y, valid | (k << 16));
+      const int2 ti = tc_tile_info(a, bg, lo + t, n_ctx);
+      t_info[seg[k].z + t] = make_int2(ti.x, ti.y | (k << 16));
     }
   }
   if (warp == 1) {
@@ -316,76 +262,80 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------------ MMA issuers
+    // warp 1 issues S = Q K^T, warp 3 issues O += P V: two single-thread
+    // issue chains, each with its own waits, so neither waits on the other
     if (lane == 0 && nt > 0) {
-      constexpr uint32_t IS = idesc_bf16_f32(128, 64, false);
-      constexpr uint32_t IP = idesc_bf16_f32(128, D, true);
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
       const uint32_t p_base = smem_u32(sP);
+      // base descriptors (128-byte swizzle): Q and K K-major (LBO 16, SBO
+      // 1024 B), P K-major, V MN-major (LBO = the 64-column half, 8 KB); the
+      // descriptor of an offset address differs by the address field only
+      const uint64_t q_desc0 = sdesc_sw128(q_base, 16, 1024);
+      const uint64_t k_desc0 = sdesc_sw128(k_base, 16, 1024);
+      const uint64_t p_desc0 = sdesc_sw128(p_base, 16, 1024);
+      const uint64_t v_desc0 = sdesc_sw128(v_base, 8192, 1024);
       bool ok = true;
       auto is_first = [&](int i) { return i == 0 || tile_seg(i - 1) != tile_seg(i); };
       auto is_last = [&](int i) { return i == nt - 1 || tile_seg(i + 1) != tile_seg(i); };
-      auto issue_s = [&](int i) -> bool {
-        const int k = tile_seg(i);
-        const int qb = QB == 2 ? (k & 1) : 0;
-        if (is_first(i) &&
-            !mbar_wait(&q_full[qb], (QB == 2 ? (k >> 1) : k) & 1, abort_flag))
-          return false;
-        const int st = i % ST;
-        if (!mbar_wait(&full_k[st], (i / ST) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t kb = k_base + st * C::KT_BYTES;
-        const uint32_t qbase = q_base + qb * C::Q_TILE;
-        const int buf = i & 1;
+      if (warp == 1) {
+        constexpr uint32_t IS = idesc_bf16_f32(128, 64, false);
+        for (int i = 0; ok && i < nt; ++i) {
+          const int k = tile_seg(i);
+          const int qb = QB == 2 ? (k & 1) : 0;
+          if (is_first(i) &&
+              !(ok = mbar_wait(&q_full[qb], (QB == 2 ? (k >> 1) : k) & 1, abort_flag)))
+            break;
+          const int buf = i & 1;
+          // the S buffer is free once the softmax of tile i-2 has read it
+          if (i >= 2 && !(ok = mbar_wait(&p_ready[buf], ((i - 2) >> 1) & 1, abort_flag))) break;
+          const int st = i % ST;
+          if (!(ok = mbar_wait(&full_k[st], (i / ST) & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint64_t ad0 = q_desc0 + (uint64_t)((qb * C::Q_TILE) >> 4);
+          const uint64_t bd0 = k_desc0 + (uint64_t)((st * C::KT_BYTES) >> 4);
 #pragma unroll
-        for (int m = 0; m < NM; ++m) {
-          const uint32_t d_t = tmem + OB * NM * D + (buf * NM + m) * 64;
+          for (int m = 0; m < NM; ++m) {
+            const uint32_t d_t = tmem + OB * NM * D + (buf * NM + m) * 64;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const int h = kk >> 2, k4 = kk & 3;
-            const uint64_t ad = sdesc_sw128(qbase + (m * C::HALVES + h) * 16384 + k4 * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(kb + h * 8192 + k4 * 32, 16, 1024);
-            mma_f16_ss(d_t, ad, bd, IS, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const int h = kk >> 2, k4 = kk & 3;
+              mma_f16_ss(d_t, ad0 + (uint64_t)(((m * C::HALVES + h) * 16384 + k4 * 32) >> 4),
+                         bd0 + (uint64_t)((h * 8192 + k4 * 32) >> 4), IS, kk > 0 ? 1u : 0u);
+            }
           }
+          mma_commit(&s_full[buf]);
+          mma_commit(&empty_k[st]);  // K is no longer needed once S is done
+          if (is_last(i)) mma_commit(&q_free[qb]);  // only S reads Q
         }
-        mma_commit(&s_full[buf]);
-        mma_commit(&empty_k[st]);  // K is no longer needed once S is done
-        return true;
-      };
-      ok = issue_s(0);
-      for (int i = 0; ok && i < nt; ++i) {
-        const int k = tile_seg(i);
-        // S of the next tile is issued ahead, unless it belongs to the next
-        // segment and both segments share the single Q buffer
-        const bool ahead = i + 1 < nt && (QB == 2 || !is_first(i + 1));
-        if (ahead && !(ok = issue_s(i + 1))) break;
-        const int buf = i & 1;
-        if (!(ok = mbar_wait(&p_ready[buf], (i >> 1) & 1, abort_flag))) break;
-        const bool first = is_first(i);
-        const int ob = OB == 2 ? (k & 1) : 0;
-        if (first && k >= OB &&
-            !(ok = mbar_wait(&o_free[ob], (OB == 2 ? ((k - OB) >> 1) : (k - OB)) & 1, abort_flag)))
-          break;
-        const int st = i % ST;
-        if (!(ok = mbar_wait(&full_v[st], (i / ST) & 1, abort_flag))) break;
-        tc_fence_after();
-        const uint32_t vb = v_base + st * C::KT_BYTES;
+      } else {
+        constexpr uint32_t IP = idesc_bf16_f32(128, D, true);
+        for (int i = 0; ok && i < nt; ++i) {
+          const int k = tile_seg(i);
+          const int buf = i & 1;
+          if (!(ok = mbar_wait(&p_ready[buf], (i >> 1) & 1, abort_flag))) break;
+          const bool first = is_first(i);
+          const int ob = OB == 2 ? (k & 1) : 0;
+          if (first && k >= OB &&
+              !(ok = mbar_wait(&o_free[ob], (OB == 2 ? ((k - OB) >> 1) : (k - OB)) & 1, abort_flag)))
+            break;
+          const int st = i % ST;
+          if (!(ok = mbar_wait(&full_v[st], (i / ST) & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint64_t vd0 = v_desc0 + (uint64_t)((st * C::KT_BYTES) >> 4);
 #pragma unroll
-        for (int m = 0; m < NM; ++m) {
-          const uint32_t d_t = tmem + (ob * NM + m) * D;
-          const uint32_t pb = p_base + (buf * NM + m) * C::P_TILE;
+          for (int m = 0; m < NM; ++m) {
+            const uint32_t d_t = tmem + (ob * NM + m) * D;
+            const uint64_t pd0 = p_desc0 + (uint64_t)(((buf * NM + m) * C::P_TILE) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = sdesc_sw128(pb + kk * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(vb + kk * 2048, 8192, 1024);
-            mma_f16_ss(d_t, ad, bd, IP, (!first || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ss(d_t, pd0 + (uint64_t)((kk * 32) >> 4),
+                         vd0 + (uint64_t)((kk * 2048) >> 4), IP, (!first || kk > 0) ? 1u : 0u);
           }
+          mma_commit(&empty_v[st]);
+          mma_commit(&pv_done[buf]);
         }
-        mma_commit(&empty_v[st]);
-        mma_commit(&pv_done[buf]);
-        if (is_last(i)) mma_commit(&q_free[QB == 2 ? (k & 1) : 0]);
-        if (i + 1 < nt && !ahead && !(ok = issue_s(i + 1))) break;
       }
       if (*abort_flag) {  // give issued MMAs time to finish before TMEM is freed
         for (uint32_t t = 0; t < (1u << 16); ++t) __nanosleep(1000);
@@ -604,10 +554,7 @@ bool tc_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-namespace {
-
-// decode block K/V: [bg][L_q][d], boxes of 64 x 64 x 1 (rows past L_q read 0)
-bool map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t L_q, uint64_t n_bg) {
+bool tc_map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t L_q, uint64_t n_bg) {
   EncodeTiled fn = encoder();
   if (!fn) return false;
   cuuint64_t dims[3] = {inner, L_q, n_bg};
@@ -619,7 +566,6 @@ bool map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t L_q, uint
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
 
 int tc_sm_count() {
   int dev = 0, n = 148;
@@ -628,15 +574,8 @@ int tc_sm_count() {
   return n;
 }
 
-namespace {
-
 // Work split of the persistent kernel: one CTA per SM (more when the tile
 // table of a CTA would overflow), S = the largest tile count of a (b, g).
-struct TcLaunch {
-  TcPlan plan;
-  int grid;
-};
-
 TcLaunch tc_plan(int n_bg, int max_tiles, int sms) {
   TcLaunch L;
   L.plan.S = max_tiles;
@@ -661,10 +600,6 @@ TcLaunch tc_plan(int n_bg, int max_tiles, int sms) {
   return L;
 }
 
-}  // namespace
-
-cudaError_t launch_combine(const AttnArgs& a, int n_split, cudaStream_t st, int S = 0,
-                           int P = 0);
 
 template <int D, int NM, int REP, int ST, int QB, int OB>
 static cudaError_t run_tc(const AttnArgs& a, int max_tiles, cudaStream_t st) {
@@ -675,8 +610,8 @@ static cudaError_t run_tc(const AttnArgs& a, int max_tiles, cudaStream_t st) {
   const uint64_t q_rows = (uint64_t)s.batch * s.H * s.L_q;
   const uint64_t n_bg = (uint64_t)s.batch * s.H_kv;
   if (!tc_map_2d(&mq, a.Q, D, q_rows, C::RB) || !tc_map_2d(&mk, a.Kp, D, pool_rows, 64) ||
-      !tc_map_2d(&mv, a.Vp, D, pool_rows, 64) || !map_3d(&mkd, a.Kd, D, s.L_q, n_bg) ||
-      !map_3d(&mvd, a.Vd, D, s.L_q, n_bg))
+      !tc_map_2d(&mv, a.Vp, D, pool_rows, 64) || !tc_map_3d(&mkd, a.Kd, D, s.L_q, n_bg) ||
+      !tc_map_3d(&mvd, a.Vd, D, s.L_q, n_bg))
     return cudaErrorInvalidValue;
   const TcLaunch L = tc_plan((int)n_bg, max_tiles, tc_sm_count());
   if (L.plan.nslot > kMaxSplits) return cudaErrorInvalidValue;  // workspace bound
@@ -697,7 +632,11 @@ bool attn_tc_supported(const AttnArgs& a) {
          (uint64_t)s.batch * s.H * s.L_q < (1ull << 31);
 }
 
+bool attn_tc_kt_supported(const AttnArgs& a);
+cudaError_t launch_attn_tc_kt(const AttnArgs& a, int max_tiles, cudaStream_t st);
+
 cudaError_t launch_attn_tc(const AttnArgs& a, int max_tiles, cudaStream_t st) {
+  if (attn_tc_kt_supported(a)) return launch_attn_tc_kt(a, max_tiles, st);
   const Shape& s = a.s;
   const int R = s.G * s.L_q;
   if (s.d == 128) {

@@ -9,136 +9,279 @@
 // the spacing of neighbouring scores, so the kept set equals the one an
 // exact computation gives.
 //
-// Two kernels.  (1) logits: grid (64-unit tiles, b*H_kv); each thread owns
-// one pooled key and 8 query rows (staged in shared memory as fp64) and
-// writes scale * q . Kbar in fp64 to the workspace.  (2) softmax: one CTA per (b, g); a warp per row takes its max
-// and sum of exponentials by shuffles and writes the probabilities in place;
-// then one thread per unit sums its column over the rows in row order.
+// Two kernels.  (1) tile: grid (128-unit tiles, b*H_kv).  Each warp owns
+// 16 pooled keys and multiplies them with every query row on the fp64
+// tensor-core MMA (m8n8k4; products of bf16 or fp32 inputs are exact in
+// fp64).  The CTA then takes, per row, the max over its 128 units, writes
+// e = exp(l - m_tile) and records (m_tile, z_tile = sum e).  (2) reduce: one
+// CTA per (b, g) merges the tile statistics of each row into the factors
+// f = exp(m_tile - M) / Z, the row's softmax being e * f, and sums the
+// columns over the rows in row order.  This is the two-pass softmax of the
+// definition with its max and sum taken tile by tile (online-softmax
+// merging), equal to it up to fp64 rounding.
 #include "common.cuh"
 #include "internal.h"
 
 namespace dl {
 
-constexpr int kUT = 64;   // units per logits CTA (one per thread column)
-constexpr int kRT = 32;   // query rows staged per pass (8 per thread)
+constexpr int kWarps = 8;              // warps per tile CTA
+constexpr int kNT = 2;                 // 8-unit MMA tiles per warp
+constexpr int kUT = kWarps * kNT * 8;  // 128 units per CTA
+constexpr int kRT = 32;                // query rows per pass (4 MMA row tiles)
 
-// Thread (u, rg): unit u0 + (tid % 64), rows rg*8 .. rg*8+7 of the pass.
-// Query rows are staged once as fp64 (exact) and read as broadcasts; the
-// pooled key is read 16 bytes at a time and converted once per element; the
-// 8 products per key element accumulate with fp64 FMAs.
+// D (8x8) += A (8x4, row-major) * B (4x8, column-major) in fp64.  Lane l
+// holds A[l/4][l%4], B[l%4][l/4] and D[l/4][2(l%4) .. 2(l%4)+1].
+__device__ __forceinline__ void dmma_m8n8k4(double (&d)[2], double a, double b) {
+  asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(d[0]), "+d"(d[1])
+               : "d"(a), "d"(b));
+}
+
+__device__ __forceinline__ float2 load_pair(const __nv_bfloat16* p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+__device__ __forceinline__ float2 load_pair(const float* p) {
+  return *reinterpret_cast<const float2*>(p);
+}
+__device__ __forceinline__ float4 load_key4(const float* p, bool ok) {
+  return ok ? __ldg(reinterpret_cast<const float4*>(p)) : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+__host__ __device__ inline int score_tiles(int n_units) { return (n_units + kUT - 1) / kUT; }
+
+// Lane (gi = lane/4, t = lane%4) of warp w: pooled keys u_w + 8nt + gi as
+// MMA B columns, query rows 8m + gi as A rows.  The four k-slots of one MMA
+// step take, for k-group kg and step i, the model dimensions
+// 16kg + 4t + i (t = the k-slot): A and B use the same assignment, so each
+// dot product still runs over every dimension once.  The lane then reads its
+// four dimensions as one float4 of the pooled key (from global memory, each
+// read once per row pass) and two double2 of the staged query row.
 template <typename T, int D>
-__global__ void __launch_bounds__(256)
-scores_logits_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
-                     const int32_t* __restrict__ q_cnt, const float* __restrict__ Kbar,
-                     Shape s, int n_units, double* __restrict__ S, unsigned* err) {
-  __shared__ __align__(16) double sQ[kRT][D];
+__global__ void __launch_bounds__(kWarps * 32, 2)
+scores_tile_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
+                   const int32_t* __restrict__ q_cnt, const float* __restrict__ Kbar, Shape s,
+                   int n_units, double* __restrict__ E, double2* __restrict__ stats,
+                   unsigned* err) {
+  constexpr int QP = D + 2;       // staged row pitch (doubles): conflict-free A loads
+  constexpr int KG = D / 16;      // k-groups of 16 dimensions
+  __shared__ __align__(16) double sQ[kRT * QP];
+  __shared__ double s_red[kWarps][kRT];
+  __shared__ double s_row[kRT];
   const int bg = blockIdx.y;
   const int b = bg / s.H_kv, g = bg % s.H_kv;
-  const int u = blockIdx.x * kUT + (threadIdx.x % kUT);
-  const int rg = threadIdx.x / kUT;  // 0..3
+  const int tile = blockIdx.x, n_tiles = gridDim.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gi = lane >> 2, t = lane & 3;
   const int nq = q_idx ? min(max(q_cnt[b], 0), s.L_q) : s.L_q;
   const int R = nq * s.G;
   const int R_max = s.L_q * s.G;
-  const bool u_ok = u < n_units;
-  const float* kb = Kbar + (((size_t)b * s.H_kv + g) * n_units + (u_ok ? u : 0)) * D;
+  if (R == 0) return;
+  const size_t pitch = (size_t)n_tiles * kUT;
+  const int u_w = tile * kUT + warp * (kNT * 8);
+
+  const float* kb[kNT];
+  bool kok[kNT];
+#pragma unroll
+  for (int nt = 0; nt < kNT; ++nt) {
+    const int u = u_w + nt * 8 + gi;
+    kok[nt] = u < n_units;
+    kb[nt] = Kbar + ((size_t)bg * n_units + (kok[nt] ? u : 0)) * D + 4 * t;
+  }
+
   for (int r0 = 0; r0 < R; r0 += kRT) {
     __syncthreads();
-    for (int e = threadIdx.x; e < kRT * D; e += blockDim.x) {
-      const int rr = e / D, c = e % D;
+    for (int c = threadIdx.x; c < kRT * (D / 2); c += blockDim.x) {
+      const int rr = c / (D / 2), col = (c % (D / 2)) * 2;
       const int r = r0 + rr;
-      double v = 0.0;
+      float2 v = make_float2(0.f, 0.f);
       if (r < R) {
         const int h = g * s.G + r / nq;
         const int i = q_idx ? q_idx[(size_t)b * s.L_q + (r % nq)] : (r % nq);
         if (i >= 0 && i < s.L_q)
-          v = (double)to_f32(Q[(((size_t)b * s.H + h) * s.L_q + i) * D + c]);
-        else if (c == 0)
+          v = load_pair(Q + (((size_t)b * s.H + h) * s.L_q + i) * D + col);
+        else if (col == 0)
           flag_error(err, ERR_BAD_INDEX);
       }
-      sQ[rr][c] = v;
+      *reinterpret_cast<double2*>(sQ + rr * QP + col) = make_double2(v.x, v.y);
     }
     __syncthreads();
-    if (!u_ok || r0 + rg * 8 >= R) continue;
-    double acc[8];
+    const int mt = min(kRT / 8, (R - r0 + 7) / 8);  // row tiles holding valid rows
+    double acc[kRT / 8][kNT][2];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) acc[k] = 0.0;
-#pragma unroll 2
-    for (int c0 = 0; c0 < D; c0 += 4) {
-      const float4 kv = __ldg(reinterpret_cast<const float4*>(kb + c0));
-      const double k0 = kv.x, k1 = kv.y, k2 = kv.z, k3 = kv.w;
+    for (int m = 0; m < kRT / 8; ++m)
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const double2 qa = *reinterpret_cast<const double2*>(&sQ[rg * 8 + k][c0]);
-        const double2 qb = *reinterpret_cast<const double2*>(&sQ[rg * 8 + k][c0 + 2]);
-        acc[k] = fma(qa.x, k0, acc[k]);
-        acc[k] = fma(qa.y, k1, acc[k]);
-        acc[k] = fma(qb.x, k2, acc[k]);
-        acc[k] = fma(qb.y, k3, acc[k]);
+      for (int nt = 0; nt < kNT; ++nt) acc[m][nt][0] = acc[m][nt][1] = 0.0;
+    float4 bv[2][kNT];
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) bv[0][nt] = load_key4(kb[nt], kok[nt]);
+#pragma unroll
+    for (int kg = 0; kg < KG; ++kg) {
+      const int cur = kg & 1;
+      if (kg + 1 < KG) {
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) bv[cur ^ 1][nt] = load_key4(kb[nt] + 16 * (kg + 1), kok[nt]);
+      }
+      double a[kRT / 8][4];
+#pragma unroll
+      for (int m = 0; m < kRT / 8; ++m) {
+        if (m < mt) {
+          const double* qa = sQ + (8 * m + gi) * QP + 16 * kg + 4 * t;
+          const double2 a01 = *reinterpret_cast<const double2*>(qa);
+          const double2 a23 = *reinterpret_cast<const double2*>(qa + 2);
+          a[m][0] = a01.x; a[m][1] = a01.y; a[m][2] = a23.x; a[m][3] = a23.y;
+        }
+      }
+      // k-step outermost: the kRT/8 x kNT accumulator chains advance in turn.
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int m = 0; m < kRT / 8; ++m) {
+          if (m < mt) {
+#pragma unroll
+            for (int nt = 0; nt < kNT; ++nt) {
+              const float bk = i == 0 ? bv[cur][nt].x : i == 1 ? bv[cur][nt].y
+                             : i == 2 ? bv[cur][nt].z : bv[cur][nt].w;
+              dmma_m8n8k4(acc[m][nt], a[m][i], (double)bk);
+            }
+          }
+        }
       }
     }
+    // Scale; units past the end take -inf so that they drop out of max and sum.
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int r = r0 + rg * 8 + k;
-      if (r < R) S[((size_t)bg * R_max + r) * n_units + u] = acc[k] * s.scale;
+    for (int m = 0; m < kRT / 8; ++m)
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+          acc[m][nt][i] = u_w + nt * 8 + 2 * t + i < n_units ? acc[m][nt][i] * s.scale : -INFINITY;
+    // Row max over the tile's 128 units: lanes t, then warps.
+#pragma unroll
+    for (int m = 0; m < kRT / 8; ++m) {
+      double v = fmax(fmax(acc[m][0][0], acc[m][0][1]), fmax(acc[m][1][0], acc[m][1][1]));
+      v = fmax(v, __shfl_xor_sync(0xffffffffu, v, 1));
+      v = fmax(v, __shfl_xor_sync(0xffffffffu, v, 2));
+      if (t == 0) s_red[warp][8 * m + gi] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < kRT) {
+      double v = s_red[0][threadIdx.x];
+#pragma unroll
+      for (int w = 1; w < kWarps; ++w) v = fmax(v, s_red[w][threadIdx.x]);
+      s_row[threadIdx.x] = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < kRT / 8; ++m) {
+      const int rr = 8 * m + gi;
+      const double mx = s_row[rr];
+      double z = 0.0;
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          acc[m][nt][i] = m < mt ? exp(acc[m][nt][i] - mx) : 0.0;
+          z += acc[m][nt][i];
+        }
+      z += __shfl_xor_sync(0xffffffffu, z, 1);
+      z += __shfl_xor_sync(0xffffffffu, z, 2);
+      if (t == 0) s_red[warp][rr] = z;
+      if (r0 + rr < R) {
+        double* row = E + ((size_t)bg * R_max + r0 + rr) * pitch + u_w + 2 * t;
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt)
+          *reinterpret_cast<double2*>(row + nt * 8) = make_double2(acc[m][nt][0], acc[m][nt][1]);
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < kRT && r0 + threadIdx.x < R) {
+      double z = 0.0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) z += s_red[w][threadIdx.x];
+      stats[((size_t)bg * R_max + r0 + threadIdx.x) * n_tiles + tile] =
+          make_double2(s_row[threadIdx.x], z);
     }
   }
 }
 
+// One CTA per (b, g).  Warp per row: M = max of the tile maxima,
+// Z = sum_t z_t exp(m_t - M); the tile factors f_t = exp(m_t - M) / Z
+// replace the statistics in place.  Then thread per unit: score[u] =
+// sum over rows, in row order, of e[r][u] * f[r][tile of u].
 __global__ void __launch_bounds__(512)
-scores_softmax_kernel(const int32_t* __restrict__ q_idx, const int32_t* __restrict__ q_cnt,
-                      Shape s, int n_units, double* __restrict__ S, double* __restrict__ score) {
+scores_reduce_kernel(const int32_t* __restrict__ q_idx, const int32_t* __restrict__ q_cnt,
+                     Shape s, int n_units, const double* __restrict__ E,
+                     double2* __restrict__ stats, double* __restrict__ score) {
   const int bg = blockIdx.x;
   const int b = bg / s.H_kv;
   const int nq = q_idx ? min(max(q_cnt[b], 0), s.L_q) : s.L_q;
   const int R = nq * s.G;
   const int R_max = s.L_q * s.G;
+  const int n_tiles = score_tiles(n_units);
+  const size_t pitch = (size_t)n_tiles * kUT;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  double* Sb = S + (size_t)bg * R_max * n_units;
+  double2* st = stats + (size_t)bg * R_max * n_tiles;
   for (int r = warp; r < R; r += nw) {
-    double* row = Sb + (size_t)r * n_units;
-    double m = -INFINITY;
-    for (int u = lane; u < n_units; u += 32) m = fmax(m, row[u]);
-    m = warp_max_d(m);
-    double z = 0.0;
-    for (int u = lane; u < n_units; u += 32) z += exp(row[u] - m);
-    z = warp_sum_d(z);
-    for (int u = lane; u < n_units; u += 32) row[u] = exp(row[u] - m) / z;
+    double2* row = st + (size_t)r * n_tiles;
+    double M = -INFINITY;
+    for (int t = lane; t < n_tiles; t += 32) M = fmax(M, row[t].x);
+    M = warp_max_d(M);
+    double Z = 0.0;
+    for (int t = lane; t < n_tiles; t += 32) Z += row[t].y * exp(row[t].x - M);
+    Z = warp_sum_d(Z);
+    __syncwarp();
+    for (int t = lane; t < n_tiles; t += 32) row[t].x = exp(row[t].x - M) / Z;
   }
   __syncthreads();
+  const double* Eb = E + (size_t)bg * R_max * pitch;
   for (int u = threadIdx.x; u < n_units; u += blockDim.x) {
+    const int t = u / kUT;
     double acc = 0.0;
-    for (int r = 0; r < R; ++r) acc += Sb[(size_t)r * n_units + u];
+    for (int r = 0; r < R; ++r) acc += Eb[(size_t)r * pitch + u] * st[(size_t)r * n_tiles + t].x;
     score[(size_t)bg * n_units + u] = acc;
   }
 }
 
+static size_t scores_e_bytes(const Shape& s, int n_units) {
+  return round256((size_t)s.batch * s.H_kv * s.G * s.L_q * (size_t)score_tiles(n_units) * kUT *
+                  sizeof(double));
+}
+
 size_t scores_workspace(const Shape& s, int n_units) {
-  return round256((size_t)s.batch * s.H_kv * s.G * s.L_q * (size_t)n_units * sizeof(double));
+  return scores_e_bytes(s, n_units) +
+         round256((size_t)s.batch * s.H_kv * s.G * s.L_q * (size_t)score_tiles(n_units) *
+                  sizeof(double2));
 }
 
 cudaError_t launch_scores(const Shape& s, const void* Q, const int32_t* q_idx,
                           const int32_t* q_cnt, const float* Kbar, int n_units, double* score,
                           void* ws, unsigned* err, cudaStream_t st) {
-  double* S = reinterpret_cast<double*>(ws);
-  dim3 grid((n_units + kUT - 1) / kUT, s.batch * s.H_kv);
+  double* E = reinterpret_cast<double*>(ws);
+  double2* stats =
+      reinterpret_cast<double2*>(reinterpret_cast<char*>(ws) + scores_e_bytes(s, n_units));
+  dim3 grid(score_tiles(n_units), s.batch * s.H_kv);
+  const dim3 block(kWarps * 32);
   if (s.dtype == 0) {
     auto* q = reinterpret_cast<const __nv_bfloat16*>(Q);
     if (s.d == 128)
-      scores_logits_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(q, q_idx, q_cnt, Kbar, s,
-                                                                     n_units, S, err);
+      scores_tile_kernel<__nv_bfloat16, 128><<<grid, block, 0, st>>>(q, q_idx, q_cnt, Kbar, s,
+                                                                     n_units, E, stats, err);
     else
-      scores_logits_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(q, q_idx, q_cnt, Kbar, s,
-                                                                    n_units, S, err);
+      scores_tile_kernel<__nv_bfloat16, 64><<<grid, block, 0, st>>>(q, q_idx, q_cnt, Kbar, s,
+                                                                    n_units, E, stats, err);
   } else {
     auto* q = reinterpret_cast<const float*>(Q);
     if (s.d == 128)
-      scores_logits_kernel<float, 128><<<grid, 256, 0, st>>>(q, q_idx, q_cnt, Kbar, s, n_units, S, err);
+      scores_tile_kernel<float, 128><<<grid, block, 0, st>>>(q, q_idx, q_cnt, Kbar, s, n_units,
+                                                             E, stats, err);
     else
-      scores_logits_kernel<float, 64><<<grid, 256, 0, st>>>(q, q_idx, q_cnt, Kbar, s, n_units, S, err);
+      scores_tile_kernel<float, 64><<<grid, block, 0, st>>>(q, q_idx, q_cnt, Kbar, s, n_units, E,
+                                                            stats, err);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  scores_softmax_kernel<<<s.batch * s.H_kv, 512, 0, st>>>(q_idx, q_cnt, s, n_units, S, score);
+  scores_reduce_kernel<<<s.batch * s.H_kv, 512, 0, st>>>(q_idx, q_cnt, s, n_units, E, stats,
+                                                         score);
   return cudaGetLastError();
 }
 

@@ -64,7 +64,7 @@ extern "C" dl_status dl_block_scores_noalloc(const dl_attn_desc* desc, const voi
     return dl::api_fail(DL_ERR_INVALID_ARG, "dl_block_scores_noalloc: n_units out of range");
   if (dl::scores_workspace(s, n_units) > kScratchBytes)
     return dl::api_fail(DL_ERR_WORKSPACE,
-                        "dl_block_scores_noalloc: batch*H*L_q*n_units*8 bytes exceeds the "
+                        "dl_block_scores_noalloc: the block-score scratch for these sizes exceeds the "
                         "built-in 32 MiB scratch; use dl_block_scores with a workspace");
   void* scratch = nullptr;
   if ((st = scratch_address(&scratch)) != DL_OK) return st;

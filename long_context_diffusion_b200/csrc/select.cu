@@ -5,18 +5,22 @@
 // the topK other blocks of largest fp64 score are added (ties -> lower
 // index), and the union is written ascending.
 //
-// One CTA per (b, g).  Up to 4096 units: a bitonic sort in shared memory of
-// (score desc, index asc) keys -- the score's bits made order-preserving and
-// inverted, the index as the tie-break -- with sinks and padding sorted
-// last; the first topK entries are kept.  Larger unit counts use a rank
-// count (the number of candidates ordered before each unit).  The ascending
-// compaction is a ballot/popc prefix count over the unit indices.
+// One CTA per (b, g).  The candidates are sorted by (score desc, index asc)
+// -- the score's bits made order-preserving and inverted, the index as the
+// tie-break -- with sinks and padding sorted last; the first topK entries
+// are kept.  Up to 1024 units: a bitonic sort with one key per thread held
+// in registers, partners at distance < 32 exchanged by warp shuffles and
+// farther ones through shared memory.  Up to 4096: the same network entirely
+// in shared memory.  Larger unit counts use a rank count (the number of
+// candidates ordered before each unit).  The ascending compaction is a
+// ballot/popc prefix count over the unit indices.
 #include "common.cuh"
 #include "internal.h"
 
 namespace dl {
 
 constexpr int kSelThreads = 1024;
+constexpr int kShflMax = 1024;
 constexpr int kBitonicMax = 4096;
 
 // Ascending order of the result equals descending order of x (IEEE bits made
@@ -25,6 +29,76 @@ __device__ __forceinline__ uint64_t desc_key(double x) {
   const uint64_t b = static_cast<uint64_t>(__double_as_longlong(x));
   const uint64_t mono = (b >> 63) ? ~b : (b | 0x8000000000000000ull);
   return ~mono;
+}
+
+// blockDim.x = n2, a power of two in [32, 1024] with n2 >= n_units; thread
+// i holds the key at position i of the network.
+__global__ void __launch_bounds__(kShflMax)
+select_shfl_kernel(const double* __restrict__ score, int H_kv, int n_units, int unit_size,
+                   int topK, const int32_t* __restrict__ sink_pos, int n_sinks,
+                   int32_t* __restrict__ blk_idx, int32_t* __restrict__ blk_cnt, int max_sel,
+                   unsigned* err) {
+  __shared__ uint64_t s_key[kShflMax];
+  __shared__ int s_idx[kShflMax];
+  __shared__ uint8_t s_sink[kShflMax];
+  __shared__ uint8_t s_keep[kShflMax];
+  __shared__ int s_warp[33];
+  const int n2 = blockDim.x;
+  const int i = threadIdx.x;
+  const int bg = blockIdx.x;
+  const int b = bg / H_kv;
+  s_sink[i] = 0;
+  s_keep[i] = 0;
+  __syncthreads();
+  for (int t = i; t < n_sinks; t += n2) {
+    const int p = sink_pos[(size_t)b * n_sinks + t];
+    if (p >= 0) {
+      const long long u = p / unit_size;
+      if (u < n_units) s_sink[u] = 1;
+      else flag_error(err, ERR_BAD_INDEX);
+    }
+  }
+  __syncthreads();
+  const bool is_sink = i < n_units && s_sink[i];
+  const int n_sb = __syncthreads_count(is_sink);
+  uint64_t key = (i < n_units && !is_sink) ? desc_key(score[(size_t)bg * n_units + i]) : ~0ull;
+  int idx = i;
+  for (int k = 2; k <= n2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      uint64_t pk;
+      int px;
+      if (j >= 32) {
+        s_key[i] = key;
+        s_idx[i] = idx;
+        __syncthreads();
+        pk = s_key[i ^ j];
+        px = s_idx[i ^ j];
+        __syncthreads();
+      } else {
+        pk = __shfl_xor_sync(0xffffffffu, key, j);
+        px = __shfl_xor_sync(0xffffffffu, idx, j);
+      }
+      // Ascending runs where (i & k) == 0; the lower position of a pair
+      // keeps the smaller key there and the larger one elsewhere.
+      const bool keep_min = ((i & j) == 0) == ((i & k) == 0);
+      const bool p_less = pk < key || (pk == key && px < idx);
+      if (keep_min == p_less) {
+        key = pk;
+        idx = px;
+      }
+    }
+  }
+  const int n_cand = n_units - n_sb;
+  const int take = topK < n_cand ? topK : n_cand;
+  if (i < take) s_keep[idx] = 1;
+  __syncthreads();
+  const bool keep = i < n_units && (s_keep[i] || s_sink[i]);
+  int total = 0;
+  const int pos = block_exclusive_count(keep, s_warp, &total);
+  int32_t* out = blk_idx + (size_t)bg * max_sel;
+  if (keep && pos < max_sel) out[pos] = i;
+  for (int e = total + i; e < max_sel; e += n2) out[e] = -1;
+  if (i == 0) blk_cnt[bg] = total < max_sel ? total : max_sel;
 }
 
 __global__ void __launch_bounds__(kSelThreads)
@@ -159,6 +233,14 @@ select_kernel(const double* __restrict__ score, int H_kv, int n_units, int unit_
 cudaError_t launch_select(const double* score, int batch, int H_kv, int n_units, int unit_size,
                           int topK, const int32_t* sink_pos, int n_sinks, int32_t* blk_idx,
                           int32_t* blk_cnt, int max_sel, unsigned* err, cudaStream_t st) {
+  if (n_units <= kShflMax) {
+    int n2 = 32;
+    while (n2 < n_units) n2 <<= 1;
+    select_shfl_kernel<<<batch * H_kv, n2, 0, st>>>(score, H_kv, n_units, unit_size, topK,
+                                                     sink_pos, n_sinks, blk_idx, blk_cnt, max_sel,
+                                                     err);
+    return cudaGetLastError();
+  }
   if (n_units <= kBitonicMax) {
     int n2 = 2;
     while (n2 < n_units) n2 <<= 1;

@@ -1,0 +1,101 @@
+"""GPU parity of block scores (a3) and top-K selection (a5) called directly
+through the C ABI, at unit counts that span several 128-unit score tiles
+with a ragged tail, query-row counts that need several 32-row passes, and
+selection sizes that reach each of the selection kernels (one key per
+thread up to 1024 units, the shared-memory network up to 4096, the rank
+count beyond), with tied scores and duplicate sinks."""
+import numpy as np
+import pytest
+import torch
+
+import long_context_diffusion_b200 as dl
+import oracle
+import synth
+from tests.helpers import np_
+
+pytestmark = pytest.mark.gpu
+
+SEED = 20260520
+
+
+def _desc(batch, H, H_kv, d, L_q, n_units, dtype):
+    return dl.make_desc(batch=batch, H=H, H_kv=H_kv, d=d, L_ctx=n_units * 64, L_q=L_q, page=64,
+                        n_pages=n_units, n_slots=batch * n_units,
+                        dtype=dl.DL_BF16 if dtype == "bf16" else dl.DL_FP32)
+
+
+@pytest.mark.parametrize("n_units,H,H_kv,d,L_q,cnts,dtype", [
+    (1, 4, 4, 128, 32, [32, 7], "bf16"),
+    (129, 8, 2, 128, 32, [20, 32], "bf16"),
+    (300, 4, 1, 64, 16, [16, 3], "bf16"),
+    (513, 8, 8, 128, 32, [0, 19], "bf16"),
+    (1100, 4, 2, 128, 40, [40, 1], "fp32"),
+])
+def test_block_scores_tiles_and_passes(n_units, H, H_kv, d, L_q, cnts, dtype, cuda_device):
+    batch = len(cnts)
+    G = H // H_kv
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    sid = 9000 + n_units
+    q = synth.normals(SEED, sid, 0, batch * H * L_q * d).reshape(batch, H, L_q, d)
+    q = (q * 0.7).to(tdt)
+    kbar = synth.normals(SEED, sid + 1, 0, batch * H_kv * n_units * d)
+    kbar = (kbar * 0.5).to(torch.float32).reshape(batch, H_kv, n_units, d)
+    # predicted query rows: a seeded subset of positions, ascending, cnt each
+    q_idx = torch.full((batch, L_q), -1, dtype=torch.int32)
+    for b, c in enumerate(cnts):
+        keys = synth.uniforms(SEED, sid + 2 + b, 0, L_q)
+        q_idx[b, :c] = torch.sort(torch.argsort(keys)[:c]).values.to(torch.int32)
+    q_cnt = torch.tensor(cnts, dtype=torch.int32)
+    desc = _desc(batch, H, H_kv, d, L_q, n_units, dtype)
+    ws = torch.empty(max(dl.dl_workspace_size(desc), 256), dtype=torch.uint8, device=cuda_device)
+    score = torch.full((batch, H_kv, n_units), float("nan"), dtype=torch.float64,
+                       device=cuda_device)
+    dl.dl_block_scores(desc, q.to(cuda_device), q_idx.to(cuda_device), q_cnt.to(cuda_device),
+                       kbar.to(cuda_device), n_units, score, ws)
+    torch.cuda.synchronize()
+    assert dl.dl_get_status() == dl.DL_OK
+    got = np_(score)
+    scale = oracle.scale_for(d)
+    for b, c in enumerate(cnts):
+        for g in range(H_kv):
+            rows = [q[b, g * G + j, int(q_idx[b, i])] for j in range(G) for i in range(c)]
+            Q_rows = torch.stack(rows) if rows else torch.zeros(0, d, dtype=tdt)
+            ref = oracle.block_scores(Q_rows, kbar[b, g], scale)
+            np.testing.assert_allclose(got[b, g], ref, rtol=1e-12, atol=1e-15)
+
+
+def _scores_with_ties(n_units, n_bg, sid):
+    u = synth.uniforms(SEED, sid, 0, n_bg * n_units).reshape(n_bg, n_units)
+    # a third of the units take one of four shared values: many exact ties
+    tie = synth.uniforms(SEED, sid + 1, 0, n_bg * n_units).reshape(n_bg, n_units) < 1 / 3
+    level = torch.floor(u * 4) / 4 + 0.125
+    return torch.where(tie, level, u)
+
+
+@pytest.mark.parametrize("n_units,topK", [
+    (5, 2), (31, 40), (32, 0), (33, 8), (512, 128), (1000, 64), (1024, 1023),
+    (1025, 100), (3000, 128), (4097, 300), (5000, 128),
+])
+def test_select_all_paths(n_units, topK, cuda_device):
+    batch, H_kv, unit_size, n_sinks = 2, 3, 64, 5
+    score = _scores_with_ties(n_units, batch * H_kv, 7000 + n_units)
+    sp = synth.uniforms(SEED, 7500 + n_units, 0, batch * n_sinks).reshape(batch, n_sinks)
+    sink_pos = (sp * n_units * unit_size).to(torch.int64).clamp(max=n_units * unit_size - 1)
+    sink_pos[0, 1] = sink_pos[0, 0]           # duplicate position
+    sink_pos[1, 2] = -1                       # unused slot
+    sink_pos[1, 3] = (sink_pos[1, 4] // unit_size) * unit_size + 1  # same block
+    sink_pos = sink_pos.to(torch.int32)
+    max_sel = min(topK, n_units) + n_sinks
+    blk_idx = torch.full((batch, H_kv, max_sel), -7, dtype=torch.int32, device=cuda_device)
+    blk_cnt = torch.full((batch, H_kv), -7, dtype=torch.int32, device=cuda_device)
+    dl.dl_select(score.reshape(batch, H_kv, n_units).to(cuda_device), unit_size, topK,
+                 sink_pos.to(cuda_device), blk_idx, blk_cnt)
+    torch.cuda.synchronize()
+    assert dl.dl_get_status() == dl.DL_OK
+    got_idx, got_cnt = np_(blk_idx), np_(blk_cnt)
+    for b in range(batch):
+        for g in range(H_kv):
+            ref = oracle.select_blocks(score[b * H_kv + g], sink_pos[b], unit_size, topK)
+            assert got_cnt[b, g] == len(ref)
+            assert np.array_equal(got_idx[b, g, :len(ref)], ref)
+            assert (got_idx[b, g, len(ref):] == -1).all()
