@@ -18,6 +18,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "tiles.cuh"
+#include "launch.cuh"
 
 namespace dl {
 
@@ -33,6 +34,8 @@ __host__ __device__ constexpr size_t simt_smem_bytes() {
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 attn_simt_kernel(AttnArgs a, int n_split, int tps) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float smem[];
   float* sK = smem;                              // [64][D+1]
   float* sV = sK + kTile * (D + 1);              // [64][D]
@@ -157,6 +160,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256)
 attn_combine_kernel(Shape s, int n_split, const void* ws, T* __restrict__ O,
                     float* __restrict__ lse, int S, int P) {
+  pdl_trigger();
+  pdl_wait();
   const int R = s.G * s.L_q;
   const long long n_rows = (long long)s.batch * s.H_kv * R;
   const long long gw = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -190,14 +195,18 @@ attn_combine_kernel(Shape s, int n_split, const void* ws, T* __restrict__ O,
       if (ml.x == -INFINITY) continue;
       const float wgt = expf(ml.x - M);
       L += ml.y * wgt;
+      if (O) {
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) o[c] = fmaf(part.o[row * D + lane + 32 * c], wgt, o[c]);
+        for (int c = 0; c < CPL; ++c) o[c] = fmaf(part.o[row * D + lane + 32 * c], wgt, o[c]);
+      }
     }
   }
-  const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-  T* dst = O + (((size_t)b * s.L_q + i) * s.H + h) * D;
+  if (O) {  // O == nullptr: the row LSEs only
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    T* dst = O + (((size_t)b * s.L_q + i) * s.H + h) * D;
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) dst[lane + 32 * c] = from_f32<T>(o[c] * inv);
+    for (int c = 0; c < CPL; ++c) dst[lane + 32 * c] = from_f32<T>(o[c] * inv);
+  }
   if (lse && lane == 0) lse[((size_t)b * s.H + h) * s.L_q + i] = L > 0.0f ? M + logf(L) : -INFINITY;
 }
 
@@ -219,7 +228,7 @@ template <typename T, int D>
 static cudaError_t run_combine(const AttnArgs& a, int n_split, cudaStream_t st, int S, int P) {
   const Shape& s = a.s;
   const long long rows = (long long)s.batch * s.H_kv * s.G * s.L_q;
-  attn_combine_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+  DL_LAUNCH(attn_combine_kernel<T, D>, (unsigned)((rows + 7) / 8), 256, 0, st, 
       s, n_split, a.ws, reinterpret_cast<T*>(a.O), a.lse, S, P);
   return cudaGetLastError();
 }
@@ -243,7 +252,7 @@ static cudaError_t run_simt(const AttnArgs& a, int max_tiles, cudaStream_t st) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(n_split, s.batch * s.H_kv);
-  attn_simt_kernel<T, D><<<grid, 256, smem, st>>>(a, n_split, tps);
+  DL_LAUNCH(attn_simt_kernel<T, D>, grid, 256, smem, st, a, n_split, tps);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_combine(a, n_split, st);

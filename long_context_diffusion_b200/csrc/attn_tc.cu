@@ -42,6 +42,7 @@
 
 #include "sm100.cuh"
 #include "tc_common.cuh"
+#include "launch.cuh"
 
 namespace dl {
 
@@ -127,6 +128,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
   const Shape& s = a.s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // tensor memory first; the successor may be scheduled only after that
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+    pdl_trigger();
+  }
+  pdl_wait();
   const int R = s.G * s.L_q;
   const int n_dec = (s.L_q + 63) / 64;
   const long long U = (long long)s.batch * s.H_kv * plan.S;
@@ -186,10 +194,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const int2 ti = tc_tile_info(a, bg, lo + t, n_ctx);
       t_info[seg[k].z + t] = make_int2(ti.x, ti.y | (k << 16));
     }
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
@@ -618,7 +622,7 @@ static cudaError_t run_tc(const AttnArgs& a, int max_tiles, cudaStream_t st) {
   auto kern = attn_tc_kernel<D, NM, REP, ST, QB, OB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<L.grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mkd, mvd, a, L.plan);
+  DL_LAUNCH(kern, L.grid, C::THREADS, C::SMEM, st, mq, mk, mv, mkd, mvd, a, L.plan);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return launch_combine(a, L.plan.nslot, st, L.plan.S, L.grid);
 }

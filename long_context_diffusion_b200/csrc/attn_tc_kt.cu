@@ -35,10 +35,13 @@
 // slots exactly as in attn_tc.cu; partials go to the same combine kernel.
 // Every wait is bounded and the softmax warps exchange through mbarriers (no
 // named barriers), so a role that gives up cannot leave another waiting.
+// With O == nullptr only the row LSEs are produced (the first pass of the
+// sink search): the V ring, the O^T MMAs and all O work are skipped.
 #include <mutex>
 
 #include "sm100.cuh"
 #include "tc_common.cuh"
+#include "launch.cuh"
 
 namespace dl {
 
@@ -143,6 +146,14 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   const Shape& s = a.s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool lse_only = a.O == nullptr;  // row LSEs only: no V, no P V, no O
+  // tensor memory first; the successor may be scheduled only after that
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+    pdl_trigger();
+  }
+  pdl_wait();
   const int R = s.G * s.L_q;
   const int n_dec = (s.L_q + 63) / 64;
   const long long U = (long long)s.batch * s.H_kv * plan.S;
@@ -213,10 +224,6 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       steps[seg[k].z + t] = make_int4(p0.x, p1.x, p0.y | (k << 16), p1.y);
     }
   }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -232,7 +239,7 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint8_t* ring = is_k ? sK : sV;
     const CUtensorMap* map = is_k ? &tm_k : &tm_v;
     const CUtensorMap* map_dec = is_k ? &tm_kd : &tm_vd;
-    if (lane == 0 && nst > 0) {
+    if (lane == 0 && nst > 0 && (is_k || !lse_only)) {
       prefetch_tmap(map);
       prefetch_tmap(map_dec);
       int next_q = 0;
@@ -285,7 +292,7 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   } else if (warp == 1 || warp == 3) {
     // ------------------------------------------------------------ MMA issuers
-    if (lane == 0 && nst > 0) {
+    if (lane == 0 && nst > 0 && (warp == 1 || !lse_only)) {
       // K and Q K-major (LBO 16, SBO 1024 B); V^T and P^T MN-major (LBO =
       // the 64-column half, SBO = 1024 B per 8 keys)
       const uint64_t q_desc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
@@ -362,6 +369,29 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
     };
+    // end of segment k: the row sums over the 128 lanes, (max, sum) of each
+    // row to the partial, and a fresh reference for the next segment
+    auto segment_sums = [&](int k) -> bool {
+      s_sum[quad * NQ + lane] = xreduce32<false>(l_sum, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(lbar);
+      if (!wait_all(lbar, n_segdone & 1)) return false;
+      ++n_segdone;
+      if (quad == 0 && lane < R) {
+        const size_t prow0 = ((size_t)seg[k].x * plan.nslot + seg[k].y) * R;
+        const float lt = s_sum[lane] + s_sum[NQ + lane] + s_sum[2 * NQ + lane] + s_sum[3 * NQ + lane];
+        part.ml[prow0 + lane] = make_float2(
+            m_mine == -INFINITY ? -INFINITY : m_mine * 0.69314718055994531f,
+            m_mine == -INFINITY ? 0.0f : lt);
+      }
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        m_ref[q] = -INFINITY;
+        l_sum[q] = 0.0f;
+      }
+      m_mine = -INFINITY;
+      return true;
+    };
     for (int j = 0; ok && j < nst; ++j) {
       const int4 e = steps[j];
       const int k = step_seg(e);
@@ -414,7 +444,7 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         m_mine = fmaxf(m_mine, fmaxf(fmaxf(s_max[lane], s_max[NQ + lane]),
                                      fmaxf(s_max[2 * NQ + lane], s_max[3 * NQ + lane])));
-        if (!first) {
+        if (!first && !lse_only) {
           // O^T holds every step before j: rescale this thread's row
           if (!(ok = wait_all(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1))) break;
           tc_fence_after();
@@ -436,6 +466,12 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         l_sum[q] += p0;
         l_sum[q + 1] += p1;
         pk[q >> 1] = pack_bf16x2(p0, p1);
+      }
+      if (lse_only) {  // the row sums are all that is kept
+        tc_fence_before();
+        mbar_arrive(&p_ready[buf]);
+        if (last && !(ok = segment_sums(k))) break;
+        continue;
       }
       // the P^T buffer is free once the O^T MMAs of step j-2 are done
       if (j >= 2 && !(ok = wait_all(&pv_done[buf], ((j - 2) >> 1) & 1))) break;
@@ -475,23 +511,7 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (q < R) part.o[(prow0 + q) * D + key] = __uint_as_float(o[q]);
       tc_fence_before();
       mbar_arrive(&o_free[ob]);
-      s_sum[quad * NQ + lane] = xreduce32<false>(l_sum, lane);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(lbar);
-      if (!(ok = wait_all(lbar, n_segdone & 1))) break;
-      ++n_segdone;
-      if (quad == 0 && lane < R) {
-        const float lt = s_sum[lane] + s_sum[NQ + lane] + s_sum[2 * NQ + lane] + s_sum[3 * NQ + lane];
-        part.ml[prow0 + lane] = make_float2(
-            m_mine == -INFINITY ? -INFINITY : m_mine * 0.69314718055994531f,
-            m_mine == -INFINITY ? 0.0f : lt);
-      }
-#pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        m_ref[q] = -INFINITY;
-        l_sum[q] = 0.0f;
-      }
-      m_mine = -INFINITY;
+      if (!(ok = segment_sums(k))) break;
     }
   }
   if (threadIdx.x == 0 && *abort_flag) flag_error(a.err, ERR_TIMEOUT);
@@ -527,7 +547,7 @@ cudaError_t launch_attn_tc_kt(const AttnArgs& a, int max_tiles, cudaStream_t st)
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kt_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kt::SMEM);
   if (e != cudaSuccess) return e;
-  attn_tc_kt_kernel<<<L.grid, kt::THREADS, kt::SMEM, st>>>(mq, mk, mv, mkd, mvd, a, L.plan);
+  DL_LAUNCH(attn_tc_kt_kernel, L.grid, kt::THREADS, kt::SMEM, st, mq, mk, mv, mkd, mvd, a, L.plan);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return launch_combine(a, L.plan.nslot, st, L.plan.S, L.grid);
 }

@@ -11,6 +11,7 @@
 // divided by the token count and rounded once to fp32.
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace dl {
 
@@ -23,6 +24,8 @@ __global__ void __launch_bounds__(256)
 pool_kernel(const T* __restrict__ Kp, const int32_t* __restrict__ page_table, Shape s,
             int n_units, int stride, int offset, int len, float* __restrict__ Kbar,
             unsigned* err) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int EPT = Vec16<T>::N;          // elements per 16-byte load
   constexpr int TPR = D / EPT;              // threads per K row
   constexpr int UPC = 256 / TPR;            // units per CTA
@@ -78,18 +81,18 @@ cudaError_t launch_pool(const Shape& s, const void* Kp, const int32_t* page_tabl
   if (s.dtype == 0) {
     auto* k = reinterpret_cast<const __nv_bfloat16*>(Kp);
     if (s.d == 128)
-      pool_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(k, page_table, s, n_units, stride,
+      DL_LAUNCH(pool_kernel<__nv_bfloat16, 128>, grid, 256, 0, st, k, page_table, s, n_units, stride,
                                                             offset, len, Kbar, err);
     else
-      pool_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(k, page_table, s, n_units, stride,
+      DL_LAUNCH(pool_kernel<__nv_bfloat16, 64>, grid, 256, 0, st, k, page_table, s, n_units, stride,
                                                            offset, len, Kbar, err);
   } else {
     auto* k = reinterpret_cast<const float*>(Kp);
     if (s.d == 128)
-      pool_kernel<float, 128><<<grid, 256, 0, st>>>(k, page_table, s, n_units, stride, offset,
+      DL_LAUNCH(pool_kernel<float, 128>, grid, 256, 0, st, k, page_table, s, n_units, stride, offset,
                                                     len, Kbar, err);
     else
-      pool_kernel<float, 64><<<grid, 256, 0, st>>>(k, page_table, s, n_units, stride, offset,
+      DL_LAUNCH(pool_kernel<float, 64>, grid, 256, 0, st, k, page_table, s, n_units, stride, offset,
                                                    len, Kbar, err);
   }
   return cudaGetLastError();

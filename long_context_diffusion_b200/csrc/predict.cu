@@ -9,12 +9,15 @@
 // popc prefix count.
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace dl {
 
 __global__ void __launch_bounds__(1024)
 predict_kernel(const float* __restrict__ conf, const uint8_t* __restrict__ masked, int L_q,
                int k, int w, int32_t* __restrict__ q_idx, int32_t* __restrict__ q_cnt) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float s_conf[1024];
   __shared__ uint8_t s_mask[1024];
   __shared__ uint8_t s_chosen[1024];
@@ -56,7 +59,7 @@ predict_kernel(const float* __restrict__ conf, const uint8_t* __restrict__ maske
 cudaError_t launch_predict(const float* conf, const uint8_t* masked, int batch, int L_q, int k,
                            int w, int32_t* q_idx, int32_t* q_cnt, cudaStream_t st) {
   const int threads = ((L_q + 31) / 32) * 32;
-  predict_kernel<<<batch, threads, 0, st>>>(conf, masked, L_q, k, w, q_idx, q_cnt);
+  DL_LAUNCH(predict_kernel, batch, threads, 0, st, conf, masked, L_q, k, w, q_idx, q_cnt);
   return cudaGetLastError();
 }
 

@@ -21,6 +21,7 @@
 // merging), equal to it up to fp64 rounding.
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace dl {
 
@@ -43,9 +44,6 @@ __device__ __forceinline__ float2 load_pair(const __nv_bfloat16* p) {
 __device__ __forceinline__ float2 load_pair(const float* p) {
   return *reinterpret_cast<const float2*>(p);
 }
-__device__ __forceinline__ float4 load_key4(const float* p, bool ok) {
-  return ok ? __ldg(reinterpret_cast<const float4*>(p)) : make_float4(0.f, 0.f, 0.f, 0.f);
-}
 
 __host__ __device__ inline int score_tiles(int n_units) { return (n_units + kUT - 1) / kUT; }
 
@@ -54,17 +52,49 @@ __host__ __device__ inline int score_tiles(int n_units) { return (n_units + kUT 
 // step take, for k-group kg and step i, the model dimensions
 // 16kg + 4t + i (t = the k-slot): A and B use the same assignment, so each
 // dot product still runs over every dimension once.  The lane then reads its
-// four dimensions as one float4 of the pooled key (from global memory, each
-// read once per row pass) and two double2 of the staged query row.
+// four dimensions as one float4 of the staged pooled key and two double2 of
+// the staged query row.  The CTA's 128 pooled keys are copied to shared
+// memory once (cp.async, overlapping the query staging); query rows are
+// staged 32 at a time as fp64.
+// Pooled keys: fp32 rows of D, the 16-byte chunk index XOR-ed with
+// 4 * (row & 1) so that the float4 loads of two rows in one quarter-warp hit
+// distinct banks.  Query rows: fp64, pitch D + 2 (rows 16 B apart mod 128).
+// The rows as copied (bf16 or fp32) sit in the tail of the fp64 area and are
+// converted through registers.
+template <typename T, int D>
+struct TileSmem {
+  static constexpr int QP = D + 2;
+  static constexpr int K_BYTES = kUT * D * 4;
+  static constexpr int Q_BYTES = kRT * QP * 8;
+  static constexpr int RAW_BYTES = kRT * D * (int)sizeof(T);
+  static constexpr int RAW_OFF = K_BYTES + Q_BYTES - RAW_BYTES;
+  static constexpr int BYTES = K_BYTES + Q_BYTES;
+  static_assert(RAW_BYTES <= Q_BYTES && RAW_OFF % 16 == 0, "raw query rows inside the fp64 area");
+};
+__device__ __forceinline__ int key_chunk(int j, int chunk) { return chunk ^ ((j & 1) << 2); }
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src, bool ok) {
+  const uint32_t sp = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sp), "l"(src),
+               "r"(ok ? 16 : 0)
+               : "memory");
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kWarps * 32, 2)
 scores_tile_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
                    const int32_t* __restrict__ q_cnt, const float* __restrict__ Kbar, Shape s,
                    int n_units, double* __restrict__ E, double2* __restrict__ stats,
                    unsigned* err) {
-  constexpr int QP = D + 2;       // staged row pitch (doubles): conflict-free A loads
-  constexpr int KG = D / 16;      // k-groups of 16 dimensions
-  __shared__ __align__(16) double sQ[kRT * QP];
+  pdl_trigger();
+  pdl_wait();
+  using L = TileSmem<T, D>;
+  constexpr int KG = D / 16;               // k-groups of 16 dimensions
+  constexpr int CPR = D * sizeof(T) / 16;  // 16-byte chunks per query row
+  extern __shared__ __align__(16) uint8_t smem_s[];
+  float* sK = reinterpret_cast<float*>(smem_s);                   // [kUT][D], swizzled
+  double* sQ = reinterpret_cast<double*>(smem_s + L::K_BYTES);    // [kRT][QP]
+  T* sRaw = reinterpret_cast<T*>(smem_s + L::RAW_OFF);            // [kRT][D]
   __shared__ double s_red[kWarps][kRT];
   __shared__ double s_row[kRT];
   const int bg = blockIdx.y;
@@ -72,37 +102,63 @@ scores_tile_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
   const int tile = blockIdx.x, n_tiles = gridDim.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gi = lane >> 2, t = lane & 3;
+  const size_t pitch = (size_t)n_tiles * kUT;
+  const int u_t = tile * kUT;
+  const int u_w = u_t + warp * (kNT * 8);
+
+  {  // the tile's pooled keys (zeros past the last unit), in flight from the start
+    const float* src = Kbar + ((size_t)bg * n_units + u_t) * D;
+    for (int c = threadIdx.x; c < kUT * (D / 4); c += blockDim.x) {
+      const int j = c / (D / 4), col = (c % (D / 4)) * 4;
+      const bool ok = u_t + j < n_units;
+      cp_async16(sK + j * D + key_chunk(j, col >> 2) * 4, ok ? src + (size_t)j * D + col : Kbar,
+                 ok);
+    }
+  }
   const int nq = q_idx ? min(max(q_cnt[b], 0), s.L_q) : s.L_q;
   const int R = nq * s.G;
   const int R_max = s.L_q * s.G;
-  if (R == 0) return;
-  const size_t pitch = (size_t)n_tiles * kUT;
-  const int u_w = tile * kUT + warp * (kNT * 8);
-
-  const float* kb[kNT];
-  bool kok[kNT];
-#pragma unroll
-  for (int nt = 0; nt < kNT; ++nt) {
-    const int u = u_w + nt * 8 + gi;
-    kok[nt] = u < n_units;
-    kb[nt] = Kbar + ((size_t)bg * n_units + (kok[nt] ? u : 0)) * D + 4 * t;
+  if (R == 0) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    return;
   }
 
   for (int r0 = 0; r0 < R; r0 += kRT) {
-    __syncthreads();
-    for (int c = threadIdx.x; c < kRT * (D / 2); c += blockDim.x) {
-      const int rr = c / (D / 2), col = (c % (D / 2)) * 2;
+    __syncthreads();  // the previous pass is done with sQ and sRaw
+    // query rows r0 .. r0+31 as copied (zeros past R or for a bad index)
+    for (int c = threadIdx.x; c < kRT * CPR; c += blockDim.x) {
+      const int rr = c / CPR, ch = c % CPR;
       const int r = r0 + rr;
-      float2 v = make_float2(0.f, 0.f);
+      const T* src = Q;
+      bool ok = false;
       if (r < R) {
         const int h = g * s.G + r / nq;
         const int i = q_idx ? q_idx[(size_t)b * s.L_q + (r % nq)] : (r % nq);
-        if (i >= 0 && i < s.L_q)
-          v = load_pair(Q + (((size_t)b * s.H + h) * s.L_q + i) * D + col);
-        else if (col == 0)
+        if (i >= 0 && i < s.L_q) {
+          src = Q + (((size_t)b * s.H + h) * s.L_q + i) * D + ch * (16 / sizeof(T));
+          ok = true;
+        } else if (ch == 0) {
           flag_error(err, ERR_BAD_INDEX);
+        }
       }
-      *reinterpret_cast<double2*>(sQ + rr * QP + col) = make_double2(v.x, v.y);
+      cp_async16(sRaw + rr * D + ch * (16 / sizeof(T)), src, ok);
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    // to fp64 (the copied rows share the area: read all, sync, then write)
+    constexpr int NP = kRT * (D / 2) / (kWarps * 32);
+    float2 v[NP];
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+      const int c = threadIdx.x + q * kWarps * 32;
+      v[q] = load_pair(sRaw + (c / (D / 2)) * D + (c % (D / 2)) * 2);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+      const int c = threadIdx.x + q * kWarps * 32;
+      *reinterpret_cast<double2*>(sQ + (c / (D / 2)) * L::QP + (c % (D / 2)) * 2) =
+          make_double2(v[q].x, v[q].y);
     }
     __syncthreads();
     const int mt = min(kRT / 8, (R - r0 + 7) / 8);  // row tiles holding valid rows
@@ -111,21 +167,18 @@ scores_tile_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
     for (int m = 0; m < kRT / 8; ++m)
 #pragma unroll
       for (int nt = 0; nt < kNT; ++nt) acc[m][nt][0] = acc[m][nt][1] = 0.0;
-    float4 bv[2][kNT];
-#pragma unroll
-    for (int nt = 0; nt < kNT; ++nt) bv[0][nt] = load_key4(kb[nt], kok[nt]);
-#pragma unroll
+#pragma unroll 2
     for (int kg = 0; kg < KG; ++kg) {
-      const int cur = kg & 1;
-      if (kg + 1 < KG) {
+      float4 bv[kNT];
 #pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) bv[cur ^ 1][nt] = load_key4(kb[nt] + 16 * (kg + 1), kok[nt]);
-      }
+      for (int nt = 0; nt < kNT; ++nt)
+        bv[nt] = *reinterpret_cast<const float4*>(
+            sK + (warp * (kNT * 8) + nt * 8 + gi) * D + key_chunk(gi, 4 * kg + t) * 4);
       double a[kRT / 8][4];
 #pragma unroll
       for (int m = 0; m < kRT / 8; ++m) {
         if (m < mt) {
-          const double* qa = sQ + (8 * m + gi) * QP + 16 * kg + 4 * t;
+          const double* qa = sQ + (8 * m + gi) * L::QP + 16 * kg + 4 * t;
           const double2 a01 = *reinterpret_cast<const double2*>(qa);
           const double2 a23 = *reinterpret_cast<const double2*>(qa + 2);
           a[m][0] = a01.x; a[m][1] = a01.y; a[m][2] = a23.x; a[m][3] = a23.y;
@@ -139,8 +192,7 @@ scores_tile_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
           if (m < mt) {
 #pragma unroll
             for (int nt = 0; nt < kNT; ++nt) {
-              const float bk = i == 0 ? bv[cur][nt].x : i == 1 ? bv[cur][nt].y
-                             : i == 2 ? bv[cur][nt].z : bv[cur][nt].w;
+              const float bk = i == 0 ? bv[nt].x : i == 1 ? bv[nt].y : i == 2 ? bv[nt].z : bv[nt].w;
               dmma_m8n8k4(acc[m][nt], a[m][i], (double)bk);
             }
           }
@@ -212,6 +264,8 @@ __global__ void __launch_bounds__(512)
 scores_reduce_kernel(const int32_t* __restrict__ q_idx, const int32_t* __restrict__ q_cnt,
                      Shape s, int n_units, const double* __restrict__ E,
                      double2* __restrict__ stats, double* __restrict__ score) {
+  pdl_trigger();
+  pdl_wait();
   const int bg = blockIdx.x;
   const int b = bg / s.H_kv;
   const int nq = q_idx ? min(max(q_cnt[b], 0), s.L_q) : s.L_q;
@@ -237,7 +291,18 @@ scores_reduce_kernel(const int32_t* __restrict__ q_idx, const int32_t* __restric
   for (int u = threadIdx.x; u < n_units; u += blockDim.x) {
     const int t = u / kUT;
     double acc = 0.0;
-    for (int r = 0; r < R; ++r) acc += Eb[(size_t)r * pitch + u] * st[(size_t)r * n_tiles + t].x;
+    int r = 0;
+    for (; r + 8 <= R; r += 8) {  // 8 rows' loads in flight, then the sums in row order
+      double e[8], f[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        e[q] = Eb[(size_t)(r + q) * pitch + u];
+        f[q] = st[(size_t)(r + q) * n_tiles + t].x;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc += e[q] * f[q];
+    }
+    for (; r < R; ++r) acc += Eb[(size_t)r * pitch + u] * st[(size_t)r * n_tiles + t].x;
     score[(size_t)bg * n_units + u] = acc;
   }
 }
@@ -261,26 +326,25 @@ cudaError_t launch_scores(const Shape& s, const void* Q, const int32_t* q_idx,
       reinterpret_cast<double2*>(reinterpret_cast<char*>(ws) + scores_e_bytes(s, n_units));
   dim3 grid(score_tiles(n_units), s.batch * s.H_kv);
   const dim3 block(kWarps * 32);
-  if (s.dtype == 0) {
-    auto* q = reinterpret_cast<const __nv_bfloat16*>(Q);
-    if (s.d == 128)
-      scores_tile_kernel<__nv_bfloat16, 128><<<grid, block, 0, st>>>(q, q_idx, q_cnt, Kbar, s,
-                                                                     n_units, E, stats, err);
-    else
-      scores_tile_kernel<__nv_bfloat16, 64><<<grid, block, 0, st>>>(q, q_idx, q_cnt, Kbar, s,
-                                                                    n_units, E, stats, err);
-  } else {
-    auto* q = reinterpret_cast<const float*>(Q);
-    if (s.d == 128)
-      scores_tile_kernel<float, 128><<<grid, block, 0, st>>>(q, q_idx, q_cnt, Kbar, s, n_units,
-                                                             E, stats, err);
-    else
-      scores_tile_kernel<float, 64><<<grid, block, 0, st>>>(q, q_idx, q_cnt, Kbar, s, n_units, E,
-                                                            stats, err);
+  cudaError_t e;
+#define DL_TILE(T, D_)                                                                        \
+  {                                                                                          \
+    auto k = scores_tile_kernel<T, D_>;                                                      \
+    constexpr int smem = TileSmem<T, D_>::BYTES;                                                \
+    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=  \
+        cudaSuccess)                                                                         \
+      return e;                                                                              \
+    DL_LAUNCH(k, grid, block, smem, st, reinterpret_cast<const T*>(Q), q_idx, q_cnt, Kbar, s, n_units, \
+                                 E, stats, err);                                             \
   }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  scores_reduce_kernel<<<s.batch * s.H_kv, 512, 0, st>>>(q_idx, q_cnt, s, n_units, E, stats,
+  if (s.dtype == 0) {
+    if (s.d == 128) DL_TILE(__nv_bfloat16, 128) else DL_TILE(__nv_bfloat16, 64)
+  } else {
+    if (s.d == 128) DL_TILE(float, 128) else DL_TILE(float, 64)
+  }
+#undef DL_TILE
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  DL_LAUNCH(scores_reduce_kernel, s.batch * s.H_kv, 512, 0, st, q_idx, q_cnt, s, n_units, E, stats,
                                                          score);
   return cudaGetLastError();
 }

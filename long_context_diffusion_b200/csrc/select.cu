@@ -16,6 +16,7 @@
 // ballot/popc prefix count over the unit indices.
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace dl {
 
@@ -38,6 +39,8 @@ select_shfl_kernel(const double* __restrict__ score, int H_kv, int n_units, int 
                    int topK, const int32_t* __restrict__ sink_pos, int n_sinks,
                    int32_t* __restrict__ blk_idx, int32_t* __restrict__ blk_cnt, int max_sel,
                    unsigned* err) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ uint64_t s_key[kShflMax];
   __shared__ int s_idx[kShflMax];
   __shared__ uint8_t s_sink[kShflMax];
@@ -106,6 +109,8 @@ select_bitonic_kernel(const double* __restrict__ score, int H_kv, int n_units, i
                       int unit_size, int topK, const int32_t* __restrict__ sink_pos, int n_sinks,
                       int32_t* __restrict__ blk_idx, int32_t* __restrict__ blk_cnt, int max_sel,
                       unsigned* err) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ __align__(16) unsigned char smem[];
   uint64_t* s_key = reinterpret_cast<uint64_t*>(smem);
   int* s_idx = reinterpret_cast<int*>(s_key + n2);
@@ -180,6 +185,8 @@ __global__ void __launch_bounds__(kSelThreads)
 select_kernel(const double* __restrict__ score, int H_kv, int n_units, int unit_size, int topK,
               const int32_t* __restrict__ sink_pos, int n_sinks, int32_t* __restrict__ blk_idx,
               int32_t* __restrict__ blk_cnt, int max_sel, unsigned* err) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ unsigned char smem[];
   double* s_score = reinterpret_cast<double*>(smem);
   uint8_t* s_sink = reinterpret_cast<uint8_t*>(s_score + n_units);
@@ -236,7 +243,7 @@ cudaError_t launch_select(const double* score, int batch, int H_kv, int n_units,
   if (n_units <= kShflMax) {
     int n2 = 32;
     while (n2 < n_units) n2 <<= 1;
-    select_shfl_kernel<<<batch * H_kv, n2, 0, st>>>(score, H_kv, n_units, unit_size, topK,
+    DL_LAUNCH(select_shfl_kernel, batch * H_kv, n2, 0, st, score, H_kv, n_units, unit_size, topK,
                                                      sink_pos, n_sinks, blk_idx, blk_cnt, max_sel,
                                                      err);
     return cudaGetLastError();
@@ -251,7 +258,7 @@ cudaError_t launch_select(const double* score, int batch, int H_kv, int n_units,
       if (e != cudaSuccess) return e;
     }
     const int threads = n2 / 2 < 32 ? 32 : (n2 / 2 > kSelThreads ? kSelThreads : n2 / 2);
-    select_bitonic_kernel<<<batch * H_kv, threads, smem, st>>>(
+    DL_LAUNCH(select_bitonic_kernel, batch * H_kv, threads, smem, st, 
         score, H_kv, n_units, n2, unit_size, topK, sink_pos, n_sinks, blk_idx, blk_cnt, max_sel,
         err);
     return cudaGetLastError();
@@ -262,7 +269,7 @@ cudaError_t launch_select(const double* score, int batch, int H_kv, int n_units,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  select_kernel<<<batch * H_kv, kSelThreads, smem, st>>>(score, H_kv, n_units, unit_size, topK,
+  DL_LAUNCH(select_kernel, batch * H_kv, kSelThreads, smem, st, score, H_kv, n_units, unit_size, topK,
                                                          sink_pos, n_sinks, blk_idx, blk_cnt,
                                                          max_sel, err);
   return cudaGetLastError();

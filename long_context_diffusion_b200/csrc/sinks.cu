@@ -20,6 +20,7 @@
 //           position asc), written ascending.
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace dl {
 
@@ -122,6 +123,8 @@ sink_partial_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict_
                     const int32_t* __restrict__ q_cnt, const T* __restrict__ Kp,
                     const int32_t* __restrict__ page_table, const T* __restrict__ Kd,
                     SinkWs w, unsigned* err) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float sQ[kSinkRows * D];
   __shared__ float2 sRed[kSinkTile / 32][kSinkRows];
   const int tile = blockIdx.x, bh = blockIdx.y;
@@ -168,6 +171,8 @@ sink_partial_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict_
 }
 
 __global__ void sink_lse_kernel(Shape s, const int32_t* __restrict__ q_cnt, SinkWs w) {
+  pdl_trigger();
+  pdl_wait();
   const int bh = blockIdx.x, r = threadIdx.x;
   const int b = bh / s.H;
   const int nq = min(max(q_cnt[b], 0), s.L_q);
@@ -188,6 +193,8 @@ __global__ void __launch_bounds__(kSinkTile)
 sink_mass_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
                  const int32_t* __restrict__ q_cnt, const T* __restrict__ Kp,
                  const int32_t* __restrict__ page_table, SinkWs w, unsigned* err) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float sQ[kSinkRows * D];
   __shared__ float sL[kSinkRows];
   const int b = blockIdx.y;
@@ -223,6 +230,8 @@ sink_mass_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q
 
 __global__ void __launch_bounds__(1024)
 sink_topn_kernel(Shape s, int n_sinks, SinkWs w, int32_t* __restrict__ sink_pos) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float sv[32];
   __shared__ int si[32];
   __shared__ int chosen[64];
@@ -265,27 +274,29 @@ static cudaError_t run_sinks(const Shape& s, const void* Q, const int32_t* q_idx
   const T* q = reinterpret_cast<const T*>(Q);
   const T* kp = reinterpret_cast<const T*>(Kp);
   const T* kd = reinterpret_cast<const T*>(Kd);
-  sink_partial_kernel<T, D><<<dim3(sink_tiles(s), s.batch * s.H), kSinkTile, 0, st>>>(
+  DL_LAUNCH(sink_partial_kernel<T, D>, dim3(sink_tiles(s), s.batch * s.H), kSinkTile, 0, st, 
       s, q, q_idx, q_cnt, kp, page_table, kd, w, err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  sink_lse_kernel<<<s.batch * s.H, ((s.L_q + 31) / 32) * 32, 0, st>>>(s, q_cnt, w);
+  DL_LAUNCH(sink_lse_kernel, s.batch * s.H, ((s.L_q + 31) / 32) * 32, 0, st, s, q_cnt, w);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  sink_mass_kernel<T, D><<<dim3((s.L_ctx + kSinkTile - 1) / kSinkTile, s.batch), kSinkTile, 0,
-                           st>>>(s, q, q_idx, q_cnt, kp, page_table, w, err);
+  DL_LAUNCH(sink_mass_kernel<T, D>, dim3((s.L_ctx + kSinkTile - 1) / kSinkTile, s.batch), kSinkTile, 0,
+                           st, s, q, q_idx, q_cnt, kp, page_table, w, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  sink_topn_kernel<<<s.batch, 1024, 0, st>>>(s, n_sinks, w, sink_pos);
+  DL_LAUNCH(sink_topn_kernel, s.batch, 1024, 0, st, s, n_sinks, w, sink_pos);
   return cudaGetLastError();
 }
 
 bool attn_tc_supported(const AttnArgs& a);
+bool attn_tc_kt_supported(const AttnArgs& a);
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_sink_mass_tc(const Shape& s, const void* Q, const int32_t* q_idx,
                                 const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
                                 const float* lse, float* mass, unsigned* err, cudaStream_t st);
 
 // bf16 with at most 256 query rows per KV group: tensor cores (pass 1 = dense
-// attention with V = K for the row LSEs, pass 2 = sinks_tc.cu); otherwise
+// attention for the row LSEs -- LSE-only on the key-major kernel, otherwise
+// with V = K and the output discarded --, pass 2 = sinks_tc.cu); otherwise
 // the CUDA-core passes above.
 cudaError_t launch_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
                          const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
@@ -297,13 +308,15 @@ cudaError_t launch_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
   a.idx = nullptr; a.cnt = nullptr; a.max_idx = 0; a.Kd = Kd; a.Vd = Kd; a.O = tw.O;
   a.lse = tw.lse; a.ws = tw.attn; a.ws_bytes = attn_workspace(s); a.err = err;
   if (s.dtype == 0 && s.G * s.L_q <= 256 && attn_tc_supported(a)) {
+    // the key-major kernel can skip V and O: only the row LSEs are needed
+    if (attn_tc_kt_supported(a)) a.O = nullptr;
     cudaError_t e = launch_attn(a, st);
     if (e != cudaSuccess) return e;
     e = launch_sink_mass_tc(s, Q, q_idx, q_cnt, Kp, page_table, tw.lse, tw.mass, err, st);
     if (e != cudaSuccess) return e;
     SinkWs w = sink_ws(ws, s);
     w.mass = tw.mass;
-    sink_topn_kernel<<<s.batch, 1024, 0, st>>>(s, n_sinks, w, sink_pos);
+    DL_LAUNCH(sink_topn_kernel, s.batch, 1024, 0, st, s, n_sinks, w, sink_pos);
     return cudaGetLastError();
   }
   if (s.dtype == 0)

@@ -24,6 +24,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+#include "launch.cuh"
 
 namespace dl {
 
@@ -87,10 +88,17 @@ sink_mass_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const MassArgs a) 
   const int np = max(0, min(pp0 + a.pairs_per_cta, n_pairs_all) - pp0);
   const int n_tiles = np * s.H_kv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nq = min(max(a.q_cnt[b], 0), s.L_q);
-  const int Rg = nq * s.G;  // real rows per group
   const uint32_t tmem_cols = 2 * n_pad <= 32 ? 32 : 2 * n_pad <= 64 ? 64 : 2 * n_pad <= 128 ? 128
                              : 2 * n_pad <= 256 ? 256 : 512;
+  // tensor memory first; the successor may be scheduled only after that
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, tmem_cols);
+    tmem_relinquish();
+    pdl_trigger();
+  }
+  pdl_wait();
+  const int nq = min(max(a.q_cnt[b], 0), s.L_q);
+  const int Rg = nq * s.G;  // real rows per group
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < a.stages; ++i) {
@@ -107,10 +115,6 @@ sink_mass_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const MassArgs a) 
     fence_mbar_init();
   }
   for (int e = threadIdx.x; e < np * 128; e += blockDim.x) s_mass[e] = 0.0f;
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, tmem_cols);
-    tmem_relinquish();
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -314,12 +318,12 @@ cudaError_t launch_sink_mass_tc(const Shape& s, const void* Q, const int32_t* q_
     e = cudaFuncSetAttribute(sink_mass_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    sink_mass_tc_kernel<128><<<dim3(n_cta, s.batch), 256, smem, st>>>(mk, a);
+    DL_LAUNCH(sink_mass_tc_kernel<128>, dim3(n_cta, s.batch), 256, smem, st, mk, a);
   } else {
     e = cudaFuncSetAttribute(sink_mass_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    sink_mass_tc_kernel<64><<<dim3(n_cta, s.batch), 256, smem, st>>>(mk, a);
+    DL_LAUNCH(sink_mass_tc_kernel<64>, dim3(n_cta, s.batch), 256, smem, st, mk, a);
   }
   return cudaGetLastError();
 }

@@ -14,6 +14,7 @@
 // ascending position order.
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace dl {
 
@@ -26,6 +27,8 @@ token_select_kernel(Shape s, const T* __restrict__ Q, const T* __restrict__ Kp,
                     const int32_t* __restrict__ page_table, const int32_t* __restrict__ chunk_idx,
                     int n_sel, int stride, int content, int topT, int32_t* __restrict__ tok_pos,
                     int32_t* __restrict__ tok_cnt, unsigned* err) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float sQ[kTokRows * D];
   __shared__ float sRed[kTokRows][33];
   __shared__ float sStat[kTokRows];
@@ -148,22 +151,22 @@ cudaError_t launch_token_select(const Shape& s, const void* Q, const void* Kp,
     auto* q = reinterpret_cast<const __nv_bfloat16*>(Q);
     auto* k = reinterpret_cast<const __nv_bfloat16*>(Kp);
     if (s.d == 128)
-      token_select_kernel<__nv_bfloat16, 128><<<grid, kTokThreads, 0, st>>>(
+      DL_LAUNCH(token_select_kernel<__nv_bfloat16, 128>, grid, kTokThreads, 0, st, 
           s, q, k, page_table, chunk_idx, n_sel, chunk_stride, chunk_content, topT, tok_pos,
           tok_cnt, err);
     else
-      token_select_kernel<__nv_bfloat16, 64><<<grid, kTokThreads, 0, st>>>(
+      DL_LAUNCH(token_select_kernel<__nv_bfloat16, 64>, grid, kTokThreads, 0, st, 
           s, q, k, page_table, chunk_idx, n_sel, chunk_stride, chunk_content, topT, tok_pos,
           tok_cnt, err);
   } else {
     auto* q = reinterpret_cast<const float*>(Q);
     auto* k = reinterpret_cast<const float*>(Kp);
     if (s.d == 128)
-      token_select_kernel<float, 128><<<grid, kTokThreads, 0, st>>>(
+      DL_LAUNCH(token_select_kernel<float, 128>, grid, kTokThreads, 0, st, 
           s, q, k, page_table, chunk_idx, n_sel, chunk_stride, chunk_content, topT, tok_pos,
           tok_cnt, err);
     else
-      token_select_kernel<float, 64><<<grid, kTokThreads, 0, st>>>(
+      DL_LAUNCH(token_select_kernel<float, 64>, grid, kTokThreads, 0, st, 
           s, q, k, page_table, chunk_idx, n_sel, chunk_stride, chunk_content, topT, tok_pos,
           tok_cnt, err);
   }

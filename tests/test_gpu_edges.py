@@ -16,7 +16,7 @@ from tests.helpers import check_attention, desc_for, np_
 pytestmark = pytest.mark.gpu
 
 
-def _run(wl, cuda_device, sinks_given=None):
+def _run(wl, cuda_device, sinks_given=None, dense=False):
     inp = synth.make_step_inputs(wl, device=cuda_device)
     n_s = wl.sinks_given if sinks_given is None else sinks_given
     sinks = inp.sinks_planted[:, :n_s].contiguous() if n_s else None
@@ -24,19 +24,20 @@ def _run(wl, cuda_device, sinks_given=None):
     out = pipeline.layer_step(desc, inp.q_dec, inp.k_pool, inp.v_pool, inp.page_table,
                               inp.k_dec, inp.v_dec, topK=wl.topK, k=wl.k, w=wl.w,
                               conf_prev=inp.conf_prev, still_masked=inp.still_masked,
-                              sink_pos=sinks)
+                              sink_pos=sinks, dense=dense)
     assert dl.dl_get_status() == dl.DL_OK, dl._abi.lib.dl_last_error_message()
     ref = oracle.layer_step(inp.q_dec.cpu(), inp.k_pool.cpu(), inp.v_pool.cpu(),
                             inp.page_table.cpu(), inp.k_dec.cpu(), inp.v_dec.cpu(), wl.L_ctx,
                             wl.B, wl.topK, conf_prev=inp.conf_prev.cpu(),
                             still_masked=inp.still_masked.cpu(), k=wl.k, w=wl.w,
-                            sink_pos=None if sinks is None else sinks.cpu())
+                            sink_pos=None if sinks is None else sinks.cpu(), dense=dense)
     assert np.array_equal(np_(out.q_idx), ref.q_idx)
     assert np.array_equal(np_(out.q_cnt), ref.q_cnt)
-    assert np.array_equal(np_(out.Kbar), ref.Kbar)
-    assert np.allclose(np_(out.score), ref.score, rtol=1e-12, atol=1e-15)
-    assert np.array_equal(np_(out.blk_idx), ref.blk_idx)
-    assert np.array_equal(np_(out.blk_cnt), ref.blk_cnt)
+    if not dense:
+        assert np.array_equal(np_(out.Kbar), ref.Kbar)
+        assert np.allclose(np_(out.score), ref.score, rtol=1e-12, atol=1e-15)
+        assert np.array_equal(np_(out.blk_idx), ref.blk_idx)
+        assert np.array_equal(np_(out.blk_cnt), ref.blk_cnt)
     check_attention(out.O, out.lse, ref.O, ref.lse, wl.dtype == "fp32", wl.name)
     return inp, out, ref
 
@@ -57,6 +58,12 @@ CASES = {
                            scale_qkv=0.125),
     "fp32_lq64_d64": dict(dtype="fp32", H=4, H_kv=4, d=64, L_ctx=640, L_q=64, topK=2, batch=2,
                           scale_qkv=0.125),
+    # key-major tensor-core path (head dim 128, <= 32 rows per KV group):
+    # ragged NaN-padded last page, rows < 32, odd and even page counts
+    "km_ragged_nan_lq20": dict(H=8, H_kv=8, L_ctx=1000, L_q=20, topK=5, batch=2,
+                               nan_padding=True),
+    "km_gqa2_lq16_odd": dict(H=8, H_kv=4, L_ctx=2047, L_q=16, topK=6, batch=3,
+                             nan_padding=True),
 }
 
 
@@ -64,6 +71,13 @@ CASES = {
 def test_edge_case(case, cuda_device):
     wl = BASE.replace(name=case, wid=40 + sorted(CASES).index(case), **CASES[case])
     _run(wl, cuda_device)
+
+
+@pytest.mark.parametrize("L_ctx,L_q,H_kv", [(1500, 24, 8), (4096, 16, 4), (70, 9, 2)])
+def test_dense_layer_ragged(L_ctx, L_q, H_kv, cuda_device):
+    wl = BASE.replace(name=f"dense{L_ctx}", wid=63, H=8, H_kv=H_kv, L_ctx=L_ctx, L_q=L_q,
+                      batch=2, nan_padding=True)
+    _run(wl, cuda_device, dense=True)
 
 
 def test_no_sinks_given(cuda_device):
