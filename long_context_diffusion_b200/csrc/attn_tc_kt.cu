@@ -51,7 +51,8 @@ namespace kt {
 
 constexpr int D = 128;
 constexpr int NQ = 32;                     // query rows (MMA N)
-constexpr int ST = 2;                      // K / V ring stages (two pages each)
+constexpr int STK = 3;                     // K ring stages (two pages each)
+constexpr int STV = 2;                     // V ring stages
 constexpr int QB = 2;                      // Q buffers (alternating segments)
 constexpr int Q_BYTES = 2 * NQ * 128;      // [d-half][32 rows][128 B]
 constexpr int KS_BYTES = 2 * 128 * 128;    // [d-half][128 keys][128 B]
@@ -59,20 +60,21 @@ constexpr int PT_BYTES = 128 * 128;        // [128 keys][128 B] (64 B used)
 constexpr int MAX_STEPS = kTcMaxTiles / 2 + kMaxSegs;
 constexpr int Q_OFF = 0;
 constexpr int K_OFF = Q_OFF + QB * Q_BYTES;
-constexpr int V_OFF = K_OFF + ST * KS_BYTES;
-constexpr int PT_OFF = V_OFF + ST * KS_BYTES;
+constexpr int V_OFF = K_OFF + STK * KS_BYTES;
+constexpr int PT_OFF = V_OFF + STV * KS_BYTES;
 constexpr int RED_OFF = PT_OFF + 2 * PT_BYTES;   // float [4][32] maxima, [4][32] sums
 constexpr int FLAG_OFF = RED_OFF + 2 * 4 * NQ * 4;  // int [2][4] rescale votes
 constexpr int BAR_OFF = FLAG_OFF + 2 * 4 * 4;
-// full_k, empty_k, full_v, empty_v [ST]; q_full, q_free, s_full, p_ready,
-// pv_done, o_free, xbar [2]; mxbar, lbar
-constexpr int N_BARS = 4 * ST + 7 * 2 + 2;
+// full_k, empty_k [STK]; full_v, empty_v [STV]; q_full, q_free, s_full,
+// p_ready, pv_done, o_free, xbar [2]; mxbar, lbar
+constexpr int N_BARS = 2 * STK + 2 * STV + 7 * 2 + 2;
 constexpr int MISC_OFF = (BAR_OFF + N_BARS * 8 + 15) / 16 * 16;
 constexpr int STEP_OFF = MISC_OFF + 32;                  // int4 [MAX_STEPS]
 constexpr int SEG_OFF = STEP_OFF + MAX_STEPS * 16;       // int4 [kMaxSegs]
 constexpr int MARK_OFF = SEG_OFF + kMaxSegs * 16;        // int2 [kMaxSegs]
 constexpr int SEGHI_OFF = MARK_OFF + kMaxSegs * 8;       // int [kMaxSegs]
-constexpr int SMEM = SEGHI_OFF + kMaxSegs * 4 + 1024;    // + alignment slack
+constexpr int NCTX_OFF = SEGHI_OFF + kMaxSegs * 4;       // int [kMaxSegs]
+constexpr int SMEM = NCTX_OFF + kMaxSegs * 4 + 1024;     // + alignment slack
 constexpr int THREADS = 256;
 constexpr uint32_t TMEM_COLS = 128;  // S^T [2][32] at 0, O^T [2][32] at 64
 constexpr uint32_t S_COL = 0, O_COL = 64;
@@ -122,10 +124,10 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   float* s_sum = s_max + 4 * NQ;                            // [4][32]
   int* s_vote = reinterpret_cast<int*>(smem + FLAG_OFF);    // [2][4]
   uint64_t* full_k = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
-  uint64_t* empty_k = full_k + ST;
-  uint64_t* full_v = empty_k + ST;
-  uint64_t* empty_v = full_v + ST;
-  uint64_t* q_full = empty_v + ST;  // [2] Q of a segment landed
+  uint64_t* empty_k = full_k + STK;
+  uint64_t* full_v = empty_k + STK;
+  uint64_t* empty_v = full_v + STV;
+  uint64_t* q_full = empty_v + STV;  // [2] Q of a segment landed
   uint64_t* q_free = q_full + 2;    // [2] every S^T of a segment done
   uint64_t* s_full = q_free + 2;    // [2] S^T buffer written
   uint64_t* p_ready = s_full + 2;   // [2] P^T written (and O^T rescaled)
@@ -143,6 +145,7 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   int4* seg = reinterpret_cast<int4*>(smem + SEG_OFF);    // (bg, slot, first step, lo tile)
   int2* mark = reinterpret_cast<int2*>(smem + MARK_OFF);  // (bg, slot) of empty runs
   int* seg_hi = reinterpret_cast<int*>(smem + SEGHI_OFF);  // end tile (exclusive)
+  int* s_nctx = reinterpret_cast<int*>(smem + NCTX_OFF);   // context tiles of each (b, g) in range
 
   const Shape& s = a.s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -161,8 +164,12 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const long long u1 = (long long)(blockIdx.x + 1) * U / gridDim.x;
   Partials part = partials_of(a.ws, s, plan.nslot);
 
+  // the (b, g) pairs this CTA's slots touch, their tile counts in parallel
+  const int bg_lo = u1 > u0 ? (int)(u0 / plan.S) : 0;
+  const int nb = u1 > u0 ? (int)((u1 - 1) / plan.S) - bg_lo + 1 : 0;  // <= kMaxSegs (plan)
+  if (threadIdx.x < nb) s_nctx[threadIdx.x] = ctx_tile_count(a, bg_lo + threadIdx.x);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 4 * ST; ++i) mbar_init(&full_k[i], 1);
+    for (int i = 0; i < 2 * (STK + STV); ++i) mbar_init(&full_k[i], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_free[i], 1);
@@ -176,53 +183,52 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mbar_init(lbar, 4);
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  // the V ring starts zeroed: the keys of a missing second page are masked
+  // (p = 0), and 0 * (stale but finite) V = 0
+  for (int e = threadIdx.x; e < STV * KS_BYTES / 16; e += blockDim.x)
+    reinterpret_cast<uint4*>(sV)[e] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();  // before TMA writes the same bytes
+  __syncthreads();
+  if (threadIdx.x == 0) {
     int nseg = 0, nmark = 0, nstep = 0;
-    if (u1 > u0) {
-      for (int bg = (int)(u0 / plan.S); bg <= (int)((u1 - 1) / plan.S); ++bg) {
-        const long long base = (long long)bg * plan.S;
-        const int lo = (int)max(u0 - base, 0ll);
-        const int hi = (int)min(u1 - base, (long long)plan.S);
-        const int n_tiles = ctx_tile_count(a, bg) + n_dec;
-        const int thi = min(hi, n_tiles);
-        const int slot = (int)blockIdx.x - tc_owner(base, U, gridDim.x);
-        if (thi > lo) {
-          seg[nseg] = make_int4(bg, slot, nstep, lo);
-          seg_hi[nseg] = thi;
-          ++nseg;
-          nstep += (thi - lo + 1) / 2;
-        } else {
-          mark[nmark++] = make_int2(bg, slot);
-        }
+    for (int i = 0; i < nb; ++i) {
+      const int bg = bg_lo + i;
+      const long long base = (long long)bg * plan.S;
+      const int lo = (int)max(u0 - base, 0ll);
+      const int hi = (int)min(u1 - base, (long long)plan.S);
+      const int thi = min(hi, s_nctx[i] + n_dec);
+      const int slot = (int)blockIdx.x - tc_owner(base, U, gridDim.x);
+      if (thi > lo) {
+        seg[nseg] = make_int4(bg, slot, nstep, lo);
+        seg_hi[nseg] = thi;
+        ++nseg;
+        nstep += (thi - lo + 1) / 2;
+      } else {
+        mark[nmark++] = make_int2(bg, slot);
       }
     }
     *s_nstep = nstep;
     *s_nseg = nseg;
     *s_nmark = nmark;
   }
-  // the V ring starts zeroed: the keys of a missing second page are masked
-  // (p = 0), and 0 * (stale but finite) V = 0
-  for (int e = threadIdx.x; e < ST * KS_BYTES / 16; e += blockDim.x)
-    reinterpret_cast<uint4*>(sV)[e] = make_uint4(0u, 0u, 0u, 0u);
-  fence_proxy_async_smem();  // before TMA writes the same bytes
   __syncthreads();
   const int nst = *s_nstep, nseg = *s_nseg, nmark = *s_nmark;
   for (int e = threadIdx.x; e < nmark * R; e += blockDim.x) {
     const int2 mk = mark[e / R];
     part.ml[((size_t)mk.x * plan.nslot + mk.y) * R + e % R] = make_float2(-INFINITY, 0.0f);
   }
-  // step table: step t of segment k holds tiles lo + 2t and (if below the
-  // segment's end) lo + 2t + 1
-  for (int k = 0; k < nseg; ++k) {
+  // step table, every entry in parallel: step t of segment k holds tiles
+  // lo + 2(t - first) and (if below the segment's end) the next one
+  for (int t = threadIdx.x; t < nst; t += blockDim.x) {
+    int k = 0;
+    while (k + 1 < nseg && seg[k + 1].z <= t) ++k;
     const int bg = seg[k].x;
-    const int n_ctx = ctx_tile_count(a, bg);
-    const int lo = seg[k].w, hi = seg_hi[k];
-    const int n = (hi - lo + 1) / 2;
-    for (int t = threadIdx.x; t < n; t += blockDim.x) {
-      const int tile = lo + 2 * t;
-      const int2 p0 = tc_tile_info(a, bg, tile, n_ctx);
-      const int2 p1 = tile + 1 < hi ? tc_tile_info(a, bg, tile + 1, n_ctx) : make_int2(0, 0);
-      steps[seg[k].z + t] = make_int4(p0.x, p1.x, p0.y | (k << 16), p1.y);
-    }
+    const int n_ctx = s_nctx[bg - bg_lo];
+    const int tile = seg[k].w + 2 * (t - seg[k].z);
+    const int2 p0 = tc_tile_info(a, bg, tile, n_ctx);
+    const int2 p1 = tile + 1 < seg_hi[k] ? tc_tile_info(a, bg, tile + 1, n_ctx) : make_int2(0, 0);
+    steps[t] = make_int4(p0.x, p1.x, p0.y | (k << 16), p1.y);
   }
   tc_fence_before();
   __syncthreads();
@@ -239,6 +245,7 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint8_t* ring = is_k ? sK : sV;
     const CUtensorMap* map = is_k ? &tm_k : &tm_v;
     const CUtensorMap* map_dec = is_k ? &tm_kd : &tm_vd;
+    const int ST = is_k ? STK : STV;
     if (lane == 0 && nst > 0 && (is_k || !lse_only)) {
       prefetch_tmap(map);
       prefetch_tmap(map_dec);
@@ -309,8 +316,8 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           const int buf = j & 1;
           // the S^T buffer is free once the softmax of step j-2 has read it
           if (j >= 2 && !(ok = mbar_wait(&p_ready[buf], ((j - 2) >> 1) & 1, abort_flag))) break;
-          const int st = j % ST;
-          if (!(ok = mbar_wait(&full_k[st], (j / ST) & 1, abort_flag))) break;
+          const int st = j % STK;
+          if (!(ok = mbar_wait(&full_k[st], (j / STK) & 1, abort_flag))) break;
           tc_fence_after();
           const uint64_t ad0 = k_desc0 + (uint64_t)((st * KS_BYTES) >> 4);
           const uint64_t bd0 = q_desc0 + (uint64_t)((qb * Q_BYTES) >> 4);
@@ -334,8 +341,8 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           const int ob = k & 1;
           if (first && k >= 2 && !(ok = mbar_wait(&o_free[ob], ((k - 2) >> 1) & 1, abort_flag)))
             break;
-          const int st = j % ST;
-          if (!(ok = mbar_wait(&full_v[st], (j / ST) & 1, abort_flag))) break;
+          const int st = j % STV;
+          if (!(ok = mbar_wait(&full_v[st], (j / STV) & 1, abort_flag))) break;
           tc_fence_after();
           const uint64_t ad0 = v_desc0 + (uint64_t)((st * KS_BYTES) >> 4);
           const uint64_t bd0 = p_desc0 + (uint64_t)((buf * PT_BYTES) >> 4);
@@ -399,7 +406,7 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const bool first = first_of(j);
       const bool last = last_of(j);
       const int buf = j & 1;
-      const int st = j % ST;
+      const int st = j % STV;
       const int pinfo = (key < 64) ? (e.z & 0xFFFF) : e.w;
       const int pvalid = page_valid(pinfo);
       const bool kvalid = (key & 63) < pvalid;
@@ -483,7 +490,7 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (!kvalid && pvalid > 0) {
         // a loaded page's rows past its valid keys may hold anything (even
         // NaN): zero this key's V row once it has landed
-        ok = mbar_wait(&full_v[st], (j / ST) & 1, abort_flag);
+        ok = mbar_wait(&full_v[st], (j / STV) & 1, abort_flag);
         if (ok) {
           uint8_t* vr = sV + st * KS_BYTES + key * 128;
 #pragma unroll
@@ -548,7 +555,6 @@ cudaError_t launch_attn_tc_kt(const AttnArgs& a, int max_tiles, cudaStream_t st)
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kt::SMEM);
   if (e != cudaSuccess) return e;
   DL_LAUNCH(attn_tc_kt_kernel, L.grid, kt::THREADS, kt::SMEM, st, mq, mk, mv, mkd, mvd, a, L.plan);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return launch_combine(a, L.plan.nslot, st, L.plan.S, L.grid);
 }
 
