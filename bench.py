@@ -474,9 +474,11 @@ def run_ours(args):
 def count_launches(wl):
     """Kernels of this library launched per step (from the call sequence)."""
     n_sparse = wl.n_layers - wl.first_sparse_layer
-    pool, predict, attn, sinks, scores, select = 1, 1, 2, 4, 2, 1
+    pool, predict, attn, sinks = 1, 1, 2, 4
+    fused = wl.G * wl.L_q <= 32 and wl.n_blk <= 512  # dl_block_select: one kernel, else three
+    score_select = 1 if fused else 3
     return pool + predict + wl.first_sparse_layer * attn + sinks + n_sparse * (
-        scores + select + attn)
+        score_select + attn)
 
 
 def main():

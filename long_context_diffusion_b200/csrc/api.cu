@@ -247,6 +247,33 @@ dl_status dl_select(const double* score, int batch, int H_kv, int n_units, int u
                   "dl_select launch");
 }
 
+dl_status dl_block_select(const dl_attn_desc* desc, const void* Q_dec, const int32_t* q_idx,
+                          const int32_t* q_cnt, const float* Kbar, int n_units, int unit_size,
+                          int topK, const int32_t* sink_pos, int n_sinks, double* score,
+                          int32_t* blk_idx, int32_t* blk_cnt, int max_sel, void* ws,
+                          size_t ws_bytes, void* stream) {
+  dl::Shape s;
+  dl_status st = check_desc(desc, &s);
+  if (st != DL_OK) return st;
+  if (!Q_dec || !Kbar || !score || (q_idx && !q_cnt) || !blk_idx || !blk_cnt ||
+      (n_sinks > 0 && !sink_pos))
+    return fail(DL_ERR_INVALID_ARG, "dl_block_select: NULL pointer");
+  if (n_units < 1 || n_units > 16384)
+    return fail(DL_ERR_INVALID_ARG, "n_units=%d (need 1..16384)", n_units);
+  if (unit_size < 1 || topK < 0 || n_sinks < 0 || n_sinks > 1024)
+    return fail(DL_ERR_INVALID_ARG, "unit_size=%d topK=%d n_sinks=%d", unit_size, topK, n_sinks);
+  const int need = (topK < n_units ? topK : n_units) + n_sinks;
+  if (max_sel < need)
+    return fail(DL_ERR_INVALID_ARG, "max_sel=%d < min(topK, n_units) + n_sinks = %d", max_sel, need);
+  if ((st = need_ws(ws, ws_bytes, dl::scores_workspace(s, n_units))) != DL_OK) return st;
+  unsigned* err = nullptr;
+  if ((st = error_word(&err)) != DL_OK) return st;
+  return launched(dl::launch_block_select(s, Q_dec, q_idx, q_cnt, Kbar, n_units, score,
+                                          unit_size, topK, sink_pos, n_sinks, blk_idx, blk_cnt,
+                                          max_sel, ws, err, as_stream(stream)),
+                  "dl_block_select launch");
+}
+
 static dl_status attn_common(const dl_attn_desc* desc, const void* Q_dec, const void* K_pool,
                              const void* V_pool, const int32_t* page_table, int mode,
                              const int32_t* idx, const int32_t* cnt, int max_idx,

@@ -22,6 +22,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "launch.cuh"
+#include "score_common.cuh"
 
 namespace dl {
 
@@ -29,21 +30,6 @@ constexpr int kWarps = 8;              // warps per tile CTA
 constexpr int kNT = 2;                 // 8-unit MMA tiles per warp
 constexpr int kUT = kWarps * kNT * 8;  // 128 units per CTA
 constexpr int kRT = 32;                // query rows per pass (4 MMA row tiles)
-
-// D (8x8) += A (8x4, row-major) * B (4x8, column-major) in fp64.  Lane l
-// holds A[l/4][l%4], B[l%4][l/4] and D[l/4][2(l%4) .. 2(l%4)+1].
-__device__ __forceinline__ void dmma_m8n8k4(double (&d)[2], double a, double b) {
-  asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
-               : "+d"(d[0]), "+d"(d[1])
-               : "d"(a), "d"(b));
-}
-
-__device__ __forceinline__ float2 load_pair(const __nv_bfloat16* p) {
-  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
-}
-__device__ __forceinline__ float2 load_pair(const float* p) {
-  return *reinterpret_cast<const float2*>(p);
-}
 
 __host__ __device__ inline int score_tiles(int n_units) { return (n_units + kUT - 1) / kUT; }
 
@@ -71,14 +57,7 @@ struct TileSmem {
   static constexpr int BYTES = K_BYTES + Q_BYTES;
   static_assert(RAW_BYTES <= Q_BYTES && RAW_OFF % 16 == 0, "raw query rows inside the fp64 area");
 };
-__device__ __forceinline__ int key_chunk(int j, int chunk) { return chunk ^ ((j & 1) << 2); }
 
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src, bool ok) {
-  const uint32_t sp = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sp), "l"(src),
-               "r"(ok ? 16 : 0)
-               : "memory");
-}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kWarps * 32, 2)

@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "launch.cuh"
+#include "score_common.cuh"
 
 namespace dl {
 
@@ -24,13 +25,6 @@ constexpr int kSelThreads = 1024;
 constexpr int kShflMax = 1024;
 constexpr int kBitonicMax = 4096;
 
-// Ascending order of the result equals descending order of x (IEEE bits made
-// monotone, then inverted).
-__device__ __forceinline__ uint64_t desc_key(double x) {
-  const uint64_t b = static_cast<uint64_t>(__double_as_longlong(x));
-  const uint64_t mono = (b >> 63) ? ~b : (b | 0x8000000000000000ull);
-  return ~mono;
-}
 
 // blockDim.x = n2, a power of two in [32, 1024] with n2 >= n_units; thread
 // i holds the key at position i of the network.

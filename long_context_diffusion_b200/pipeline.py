@@ -48,8 +48,10 @@ class LayerOutputs:
 def layer_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec, v_dec, *,
                topK: int, conf_prev=None, still_masked=None, k: int = 4, w: int = 2,
                q_idx=None, q_cnt=None, sink_pos=None, detect_sinks: int = 0,
-               dense: bool = False, Kbar=None, ws=None, stream=None) -> LayerOutputs:
-    """One layer for a batch: (predict,) pool, score, (find sinks,) select,
+               dense: bool = False, Kbar=None, ws=None, stream=None,
+               fused_select: bool = True) -> LayerOutputs:
+    """One layer for a batch: (predict,) pool, (find sinks,) score and select
+    (one call, or dl_block_scores then dl_select when fused_select is False),
     attend -- or dense attention.  Mirrors the oracle's layer_step."""
     dev = q_dec.device
     B, L_q, d, H, H_kv = desc.batch, desc.L_q, desc.d, desc.H, desc.H_kv
@@ -70,7 +72,6 @@ def layer_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec, v
         Kbar = _empty((B, H_kv, n_blk, d), torch.float32, dev)
         A.dl_pool_keys(desc, k_pool, page_table, n_blk, desc.page, 0, desc.page, Kbar, stream)
     score = _empty((B, H_kv, n_blk), torch.float64, dev)
-    A.dl_block_scores(desc, q_dec, q_idx, q_cnt, Kbar, n_blk, score, ws, stream)
     if detect_sinks:
         sink_pos = _empty((B, detect_sinks), torch.int32, dev)
         A.dl_find_sinks(desc, q_dec, q_idx, q_cnt, k_pool, page_table, k_dec, detect_sinks,
@@ -79,7 +80,12 @@ def layer_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec, v
     max_sel = min(topK, n_blk) + n_s
     blk_idx = _empty((B, H_kv, max(max_sel, 1)), torch.int32, dev)
     blk_cnt = _empty((B, H_kv), torch.int32, dev)
-    A.dl_select(score, desc.page, topK, sink_pos, blk_idx, blk_cnt, stream)
+    if fused_select:
+        A.dl_block_select(desc, q_dec, q_idx, q_cnt, Kbar, n_blk, desc.page, topK, sink_pos,
+                          score, blk_idx, blk_cnt, ws, stream)
+    else:
+        A.dl_block_scores(desc, q_dec, q_idx, q_cnt, Kbar, n_blk, score, ws, stream)
+        A.dl_select(score, desc.page, topK, sink_pos, blk_idx, blk_cnt, stream)
     A.dl_sparse_attn(desc, q_dec, k_pool, v_pool, page_table, blk_idx, blk_cnt, k_dec, v_dec, O,
                      lse, ws, stream)
     return LayerOutputs(q_idx, q_cnt, Kbar, score, sink_pos, blk_idx, blk_cnt, O, lse)
@@ -178,10 +184,9 @@ class DenoiseStep:
             if l == self.first_sparse:
                 A.dl_find_sinks(d, q_dec[l], self.q_idx, self.q_cnt, k_pool[l], page_table,
                                 k_dec[l], self.n_sinks, self.sink_pos, self.ws, stream)
-            A.dl_block_scores(d, q_dec[l], self.q_idx, self.q_cnt, Kbar[l], self.n_blk,
-                              self.score, self.ws, stream)
-            A.dl_select(self.score, d.page, self.topK, self.sink_pos, self.blk_idx[l],
-                        self.blk_cnt[l], stream)
+            A.dl_block_select(d, q_dec[l], self.q_idx, self.q_cnt, Kbar[l], self.n_blk, d.page,
+                              self.topK, self.sink_pos, self.score, self.blk_idx[l],
+                              self.blk_cnt[l], self.ws, stream)
             ev = self._begin(attn_events, stream)
             A.dl_sparse_attn(d, q_dec[l], k_pool[l], v_pool[l], page_table, self.blk_idx[l],
                              self.blk_cnt[l], k_dec[l], v_dec[l], self.O[l], self.lse[l],

@@ -22,8 +22,8 @@ def _declared():
 def test_header_declares_the_path():
     names = _declared()
     for n in ("dl_predict_queries", "dl_pool_keys", "dl_block_scores", "dl_find_sinks",
-              "dl_select", "dl_sparse_attn", "dl_token_select", "dl_sparse_attn_gather",
-              "dl_workspace_size", "dl_get_status"):
+              "dl_select", "dl_block_select", "dl_sparse_attn", "dl_token_select",
+              "dl_sparse_attn_gather", "dl_workspace_size", "dl_get_status"):
         assert n in names
 
 
@@ -68,6 +68,14 @@ def test_null_and_range_arguments_rejected_before_launch():
     assert lib.dl_select(fake, 1, 1, 8, 64, 4, fake, 2, fake, fake, 5, None) == \
         dl.DL_ERR_INVALID_ARG
     assert "max_sel" in lib.dl_last_error_message().decode()
+    # fused scores + selection: the same checks before any launch
+    assert lib.dl_block_select(ctypes.byref(d), fake, None, None, None, 256, 64, 4, None, 0,
+                               fake, fake, fake, 4, fake, 1 << 40, None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_block_select(ctypes.byref(d), fake, None, None, fake, 256, 64, 4, fake, 2,
+                               fake, fake, fake, 5, fake, 1 << 40, None) == dl.DL_ERR_INVALID_ARG
+    assert "max_sel" in lib.dl_last_error_message().decode()
+    assert lib.dl_block_select(ctypes.byref(d), fake, None, None, fake, 256, 64, 4, None, 0,
+                               fake, fake, fake, 4, fake, 256, None) == dl.DL_ERR_WORKSPACE
     # misaligned attention pointers
     odd = ctypes.c_void_p(0x1008)
     st = lib.dl_sparse_attn(ctypes.byref(d), odd, fake, fake, fake, None, None, 0, fake, fake,

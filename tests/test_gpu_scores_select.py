@@ -99,3 +99,67 @@ def test_select_all_paths(n_units, topK, cuda_device):
             assert got_cnt[b, g] == len(ref)
             assert np.array_equal(got_idx[b, g, :len(ref)], ref)
             assert (got_idx[b, g, len(ref):] == -1).all()
+
+
+@pytest.mark.parametrize("n_units,H,H_kv,d,L_q,cnts,topK,dtype", [
+    (1, 4, 4, 128, 32, [32, 7], 4, "bf16"),           # one key
+    (129, 8, 8, 128, 32, [20, 32], 16, "bf16"),       # two chunks, ragged
+    (300, 4, 2, 64, 16, [16, 3], 40, "bf16"),         # G = 2, d 64, three chunks
+    (512, 8, 8, 128, 32, [0, 19], 128, "bf16"),       # four full chunks, a sequence with no rows
+    (200, 4, 4, 128, 32, [32, 5], 300, "fp32"),       # fp32 queries, topK beyond the candidates
+    (513, 4, 4, 128, 32, [20, 9], 64, "bf16"),        # separate kernels: more than 512 keys
+    (100, 8, 2, 128, 32, [20, 32], 10, "bf16"),       # separate kernels: 4 x 32 rows
+])
+def test_block_select_matches_oracle(n_units, H, H_kv, d, L_q, cnts, topK, dtype, cuda_device):
+    """dl_block_select (fused score + select) against the oracle, and against
+    dl_block_scores followed by dl_select."""
+    batch, n_sinks, unit = len(cnts), 3, 64
+    G = H // H_kv
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    sid = 9500 + n_units + 7 * G
+    q = (synth.normals(SEED, sid, 0, batch * H * L_q * d).reshape(batch, H, L_q, d) * 0.7).to(tdt)
+    kbar = (synth.normals(SEED, sid + 1, 0, batch * H_kv * n_units * d) * 0.5).to(
+        torch.float32).reshape(batch, H_kv, n_units, d)
+    q_idx = torch.full((batch, L_q), -1, dtype=torch.int32)
+    for b, c in enumerate(cnts):
+        keys = synth.uniforms(SEED, sid + 2 + b, 0, L_q)
+        q_idx[b, :c] = torch.sort(torch.argsort(keys)[:c]).values.to(torch.int32)
+    q_cnt = torch.tensor(cnts, dtype=torch.int32)
+    sp = synth.uniforms(SEED, sid + 9, 0, batch * n_sinks).reshape(batch, n_sinks)
+    sink_pos = (sp * n_units * unit).to(torch.int64).clamp(max=n_units * unit - 1)
+    sink_pos[0, 1] = sink_pos[0, 0]
+    sink_pos = sink_pos.to(torch.int32)
+    desc = _desc(batch, H, H_kv, d, L_q, n_units, dtype)
+    ws = torch.empty(max(dl.dl_workspace_size(desc), 256), dtype=torch.uint8, device=cuda_device)
+    max_sel = min(topK, n_units) + n_sinks
+    dev = lambda x: x.to(cuda_device)  # noqa: E731
+    outs = []
+    for fused in (True, False):
+        score = torch.full((batch, H_kv, n_units), float("nan"), dtype=torch.float64,
+                           device=cuda_device)
+        blk = torch.full((batch, H_kv, max_sel), -7, dtype=torch.int32, device=cuda_device)
+        cnt = torch.full((batch, H_kv), -7, dtype=torch.int32, device=cuda_device)
+        if fused:
+            dl.dl_block_select(desc, dev(q), dev(q_idx), dev(q_cnt), dev(kbar), n_units, unit,
+                               topK, dev(sink_pos), score, blk, cnt, ws)
+        else:
+            dl.dl_block_scores(desc, dev(q), dev(q_idx), dev(q_cnt), dev(kbar), n_units, score,
+                               ws)
+            dl.dl_select(score, unit, topK, dev(sink_pos), blk, cnt)
+        torch.cuda.synchronize()
+        assert dl.dl_get_status() == dl.DL_OK
+        outs.append((np_(score), np_(blk), np_(cnt)))
+    (s_f, b_f, c_f), (s_s, b_s, c_s) = outs
+    np.testing.assert_allclose(s_f, s_s, rtol=1e-13, atol=1e-16)
+    assert np.array_equal(b_f, b_s) and np.array_equal(c_f, c_s)
+    scale = oracle.scale_for(d)
+    for b, c in enumerate(cnts):
+        for g in range(H_kv):
+            rows = [q[b, g * G + j, int(q_idx[b, i])] for j in range(G) for i in range(c)]
+            Q_rows = torch.stack(rows) if rows else torch.zeros(0, d, dtype=tdt)
+            ref = oracle.block_scores(Q_rows, kbar[b, g], scale)
+            np.testing.assert_allclose(s_f[b, g], ref, rtol=1e-12, atol=1e-15)
+            sel = oracle.select_blocks(ref, sink_pos[b], unit, topK)
+            assert c_f[b, g] == len(sel)
+            assert np.array_equal(b_f[b, g, :len(sel)], sel)
+            assert (b_f[b, g, len(sel):] == -1).all()
