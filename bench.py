@@ -47,11 +47,11 @@ NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# DRAM traffic of the dominant kernel from one ncu capture (profiles/
-# attn_tc_kt_sparse_batch1.md: dram__bytes_read.sum + dram__bytes_write.sum of
-# the sparse layer at batch 1, 143.64 MB, scaled by 4 to the batch-4 launch).
+# DRAM traffic of the dominant kernel from one ncu capture at the benchmark's
+# size (profiles/attn_tc_kt_sparse_llada32k.md: dram__bytes_read.sum +
+# dram__bytes_write.sum of one sparse-layer launch, batch 4: 557.85 + 5.86 MB).
 # Reported only while the kernel's sources hash to the captured build.
-TRAFFIC_CAPTURE = {"sha": "261bf2e793aa28ca", "bytes_per_launch": 4 * 143.64e6,
+TRAFFIC_CAPTURE = {"sha": "fb06682a9ceea044", "bytes_per_launch": 557.849088e6 + 5.863424e6,
                    "sources": ["attn_tc_kt.cu", "tc_common.cuh", "sm100.cuh"]}
 
 

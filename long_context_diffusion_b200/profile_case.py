@@ -1,0 +1,87 @@
+"""One kernel of the denoising step, on one synthetic layer, for profiling.
+
+    python -m long_context_diffusion_b200.profile_case --case attn_sparse --reps 3
+    python -m long_context_diffusion_b200.profile_case --case block_select --reps 3
+
+Builds one sparse layer of the 32K workload (batch 4, 32 KV heads, 32K context:
+about 2.1 GB of K/V pages on the device), runs the steps before the profiled
+call once, then calls it `reps` times (the first is a warm-up) and prints its
+mean time from CUDA events.  Meant to sit under `ncu -k ... -s 1 -c 1`.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import torch
+
+import synth
+from . import _abi as A
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--case", choices=["attn_sparse", "attn_dense", "block_select", "pool"],
+                    required=True)
+    ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--batch", type=int, default=4)
+    args = ap.parse_args()
+    dev = torch.device("cuda", 0)
+    wl = synth.workload("llada32k_step", n_layers=3, batch=args.batch)
+    layer = wl.first_sparse_layer
+    pt = synth.page_permutation(wl).to(dev)
+    q = synth.make_q_dec(wl, layer, dev)
+    kd, vd = synth.make_kv_dec(wl, layer, dev)
+    kp, vp = synth.make_layer_kv(wl, layer, q, dev, pt.cpu())
+    confs, masks = zip(*(synth.confidence(wl, b) for b in range(wl.batch)))
+    conf, masked = torch.stack(confs).to(dev), torch.stack(masks).to(dev)
+    desc = A.make_desc(wl.batch, wl.H, wl.H_kv, wl.d, wl.L_ctx, wl.L_q, wl.B, wl.n_pages,
+                       wl.n_slots, A.DL_BF16)
+    ws = torch.empty(A.dl_workspace_size(desc), dtype=torch.uint8, device=dev)
+    q_idx = torch.empty((wl.batch, wl.L_q), dtype=torch.int32, device=dev)
+    q_cnt = torch.empty((wl.batch,), dtype=torch.int32, device=dev)
+    A.dl_predict_queries(conf, masked, wl.k, wl.w, q_idx, q_cnt)
+    Kbar = torch.empty((wl.batch, wl.H_kv, wl.n_blk, wl.d), dtype=torch.float32, device=dev)
+    A.dl_pool_keys(desc, kp, pt, wl.n_blk, wl.B, 0, wl.B, Kbar)
+    sinks = torch.empty((wl.batch, wl.detect_sinks), dtype=torch.int32, device=dev)
+    A.dl_find_sinks(desc, q, q_idx, q_cnt, kp, pt, kd, wl.detect_sinks, sinks, ws)
+    max_sel = min(wl.topK, wl.n_blk) + wl.detect_sinks
+    score = torch.empty((wl.batch, wl.H_kv, wl.n_blk), dtype=torch.float64, device=dev)
+    blk = torch.empty((wl.batch, wl.H_kv, max_sel), dtype=torch.int32, device=dev)
+    cnt = torch.empty((wl.batch, wl.H_kv), dtype=torch.int32, device=dev)
+    O = torch.empty((wl.batch, wl.L_q, wl.H, wl.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.batch, wl.H, wl.L_q), dtype=torch.float32, device=dev)
+
+    def block_select():
+        A.dl_block_select(desc, q, q_idx, q_cnt, Kbar, wl.n_blk, wl.B, wl.topK, sinks, score,
+                          blk, cnt, ws)
+
+    calls = {
+        "block_select": block_select,
+        "attn_sparse": lambda: A.dl_sparse_attn(desc, q, kp, vp, pt, blk, cnt, kd, vd, O, lse,
+                                                ws),
+        "attn_dense": lambda: A.dl_sparse_attn(desc, q, kp, vp, pt, None, None, kd, vd, O, lse,
+                                               ws),
+        "pool": lambda: A.dl_pool_keys(desc, kp, pt, wl.n_blk, wl.B, 0, wl.B, Kbar),
+    }
+    if args.case.startswith("attn"):
+        block_select()
+    fn = calls[args.case]
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3)
+    st = A.dl_get_status()
+    if st != A.DL_OK:
+        raise RuntimeError(f"device status {st}")
+    print(json.dumps({"case": args.case, "batch": wl.batch, "us_per_call": times,
+                      "mean_us_after_first": sum(times[1:]) / max(1, len(times) - 1)}))
+
+
+if __name__ == "__main__":
+    main()
