@@ -180,26 +180,42 @@ attn_combine_kernel(Shape s, int n_split, const void* ws, T* __restrict__ O,
     n_valid = (int)(c1 - c0 + 1);
     n_valid = n_valid < n_split ? n_valid : n_split;
   }
-  float M = -INFINITY;
-  for (int sp = 0; sp < n_valid; ++sp)
-    M = fmaxf(M, part.ml[((size_t)bg * n_split + sp) * R + r].x);
   constexpr int CPL = D / 32;
+  constexpr int SB = 4;  // slots per batch: their loads are all issued before any is used
   float o[CPL];
 #pragma unroll
   for (int c = 0; c < CPL; ++c) o[c] = 0.0f;
-  float L = 0.0f;
-  if (M != -INFINITY) {
-    for (int sp = 0; sp < n_valid; ++sp) {
-      const size_t row = ((size_t)bg * n_split + sp) * R + r;
-      const float2 ml = part.ml[row];
-      if (ml.x == -INFINITY) continue;
-      const float wgt = expf(ml.x - M);
-      L += ml.y * wgt;
-      if (O) {
+  float M = -INFINITY, L = 0.0f;
+  for (int s0 = 0; s0 < n_valid; s0 += SB) {
+    float2 ml[SB];
+    float ov[SB][CPL];
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) o[c] = fmaf(part.o[row * D + lane + 32 * c], wgt, o[c]);
-      }
+    for (int q = 0; q < SB; ++q) {
+      const size_t row = ((size_t)bg * n_split + s0 + q) * R + r;
+      const bool ok = s0 + q < n_valid;
+      ml[q] = ok ? part.ml[row] : make_float2(-INFINITY, 0.0f);
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) ov[q][c] = (ok && O) ? part.o[row * D + lane + 32 * c] : 0.0f;
     }
+    // merge this batch into the running (M, L, o), as the partials themselves
+    float Mb = M;
+#pragma unroll
+    for (int q = 0; q < SB; ++q) Mb = fmaxf(Mb, ml[q].x);
+    if (Mb == -INFINITY) continue;
+    const float a = M == -INFINITY ? 0.0f : expf(M - Mb);
+    L *= a;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) o[c] *= a;
+#pragma unroll
+    for (int q = 0; q < SB; ++q) {
+      // an empty run (m = -inf) wrote no output row: skip it, never 0 * garbage
+      if (ml[q].x == -INFINITY) continue;
+      const float wgt = expf(ml[q].x - Mb);
+      L += ml[q].y * wgt;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) o[c] = fmaf(ov[q][c], wgt, o[c]);
+    }
+    M = Mb;
   }
   if (O) {  // O == nullptr: the row LSEs only
     const float inv = L > 0.0f ? 1.0f / L : 0.0f;
