@@ -162,17 +162,22 @@ dl_status dl_select(const double* score, int batch, int H_kv, int n_units, int u
 
 /* (a3 + a5) Block scores and selection in one call: the results of
  * dl_block_scores followed by dl_select with the same arguments (score is
- * written too), computed by one kernel per (b, g) when G*L_q <= 32 and
+ * written too), computed by one kernel per (b, g) when G * max_q <= 32 and
  * n_units <= 512 (the scores then stay on chip between the two steps;
  * bf16 or fp32 queries, d 64 or 128), otherwise by the two separate kernels.
  * [F2 summary: the predicted queries rank the blocks; F1 abstract: the sinks
  * are always kept]
- * Arguments, layouts and requirements as for dl_block_scores and dl_select;
- * ws: workspace of dl_workspace_size (used only by the separate kernels). */
+ * max_q: an upper bound of q_cnt[b] that the caller guarantees (with the
+ *   prediction of dl_predict_queries: min(L_q, k * (2w + 1))); 0 = L_q.  The
+ *   fused kernel is compiled for that many rows; a sequence with more rows
+ *   is cut to the bound and reported as DL_ERR_BAD_INDEX by dl_get_status.
+ * Other arguments, layouts and requirements as for dl_block_scores and
+ * dl_select; ws: workspace of dl_workspace_size (used only by the separate
+ * kernels). */
 dl_status dl_block_select(const dl_attn_desc* desc, const void* Q_dec, const int32_t* q_idx,
                           const int32_t* q_cnt, const float* Kbar, int n_units, int unit_size,
                           int topK, const int32_t* sink_pos, int n_sinks, double* score,
-                          int32_t* blk_idx, int32_t* blk_cnt, int max_sel, void* ws,
+                          int32_t* blk_idx, int32_t* blk_cnt, int max_sel, int max_q, void* ws,
                           size_t ws_bytes, void* stream);
 
 /* (a6) Block-sparse bidirectional attention.  [F1 abstract; F2 summary]

@@ -53,8 +53,8 @@ _SIGS = {
     "dl_select": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _vp, _c_int,
                    _vp], _c_int),
     "dl_block_select": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _c_int, _c_int,
-                         _c_int, _vp, _c_int, _vp, _vp, _vp, _c_int, _vp, ctypes.c_size_t, _vp],
-                        _c_int),
+                         _c_int, _vp, _c_int, _vp, _vp, _vp, _c_int, _c_int, _vp,
+                         ctypes.c_size_t, _vp], _c_int),
     "dl_sparse_attn": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp,
                         _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp], _c_int),
     "dl_token_select": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _c_int, _c_int,
@@ -155,11 +155,11 @@ def dl_select(score, unit_size, topK, sink_pos, blk_idx, blk_cnt, stream=None):
 
 
 def dl_block_select(desc, Q_dec, q_idx, q_cnt, Kbar, n_units, unit_size, topK, sink_pos, score,
-                    blk_idx, blk_cnt, ws, stream=None):
+                    blk_idx, blk_cnt, ws, stream=None, max_q=0):
     n_sinks = 0 if sink_pos is None else sink_pos.shape[-1]
     _check(lib.dl_block_select(ctypes.byref(desc), _p(Q_dec), _p(q_idx), _p(q_cnt), _p(Kbar),
                                n_units, unit_size, topK, _p(sink_pos), n_sinks, _p(score),
-                               _p(blk_idx), _p(blk_cnt), blk_idx.shape[-1], _p(ws),
+                               _p(blk_idx), _p(blk_cnt), blk_idx.shape[-1], max_q, _p(ws),
                                ws.numel() * ws.element_size(), _s(stream)))
 
 

@@ -250,7 +250,7 @@ dl_status dl_select(const double* score, int batch, int H_kv, int n_units, int u
 dl_status dl_block_select(const dl_attn_desc* desc, const void* Q_dec, const int32_t* q_idx,
                           const int32_t* q_cnt, const float* Kbar, int n_units, int unit_size,
                           int topK, const int32_t* sink_pos, int n_sinks, double* score,
-                          int32_t* blk_idx, int32_t* blk_cnt, int max_sel, void* ws,
+                          int32_t* blk_idx, int32_t* blk_cnt, int max_sel, int max_q, void* ws,
                           size_t ws_bytes, void* stream) {
   dl::Shape s;
   dl_status st = check_desc(desc, &s);
@@ -265,12 +265,13 @@ dl_status dl_block_select(const dl_attn_desc* desc, const void* Q_dec, const int
   const int need = (topK < n_units ? topK : n_units) + n_sinks;
   if (max_sel < need)
     return fail(DL_ERR_INVALID_ARG, "max_sel=%d < min(topK, n_units) + n_sinks = %d", max_sel, need);
+  if (max_q < 0) return fail(DL_ERR_INVALID_ARG, "max_q=%d (need >= 0)", max_q);
   if ((st = need_ws(ws, ws_bytes, dl::scores_workspace(s, n_units))) != DL_OK) return st;
   unsigned* err = nullptr;
   if ((st = error_word(&err)) != DL_OK) return st;
   return launched(dl::launch_block_select(s, Q_dec, q_idx, q_cnt, Kbar, n_units, score,
                                           unit_size, topK, sink_pos, n_sinks, blk_idx, blk_cnt,
-                                          max_sel, ws, err, as_stream(stream)),
+                                          max_sel, max_q, ws, err, as_stream(stream)),
                   "dl_block_select launch");
 }
 

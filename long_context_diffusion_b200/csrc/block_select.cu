@@ -47,7 +47,7 @@ struct Smem {
 };
 }  // namespace bs
 
-template <typename T, int D>
+template <typename T, int D, int MT>
 __global__ void __launch_bounds__(bs::kThreads, 1)
 block_select_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
                     const int32_t* __restrict__ q_cnt, const float* __restrict__ Kbar, Shape s,
@@ -94,8 +94,12 @@ block_select_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
   load_chunk(0);
 
   // query rows: every predicted position of every query head of the group
-  const int nq = q_idx ? min(max(q_cnt[b], 0), s.L_q) : s.L_q;
-  const int R = nq * s.G;  // <= kMaxRows (the host routes larger groups elsewhere)
+  int nq = q_idx ? min(max(q_cnt[b], 0), s.L_q) : s.L_q;
+  if (nq * s.G > 8 * MT) {  // more rows than the caller's bound: reported, rows cut
+    if (tid == 0) flag_error(err, ERR_BAD_INDEX);
+    nq = 8 * MT / s.G;
+  }
+  const int R = nq * s.G;  // <= 8 * MT <= kMaxRows
   for (int c = tid; c < kMaxRows * CPR; c += kThreads) {
     const int r = c / CPR, ch = c % CPR;
     const T* src = Q;
@@ -133,8 +137,9 @@ block_select_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
   }
   __syncthreads();
 
-  // ---- logits: acc[c][m][i] = row 8m + gi, key c*128 + 8*warp + 2t + i
-  const int mt = (R + 7) / 8;
+  // ---- logits: acc[c][m][i] = row 8m + gi, key c*128 + 8*warp + 2t + i, for
+  // the MT row tiles of the launch (a compile-time count: a predicate on
+  // every MMA measured 30 % slower; tiles past R hold zero rows)
   double acc[kMaxChunks][kMaxRows / 8][2];
 #pragma unroll
   for (int c = 0; c < kMaxChunks; ++c)
@@ -151,22 +156,19 @@ block_select_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
 #pragma unroll 2
       for (int kg = 0; kg < KG; ++kg) {
         const float4 bv = *reinterpret_cast<const float4*>(sKc + key_chunk(gi, 4 * kg + t) * 4);
-        double a[kMaxRows / 8][4];
+        double a[MT][4];
 #pragma unroll
-        for (int m = 0; m < kMaxRows / 8; ++m) {
-          if (m < mt) {
-            const double* qa = sQ + (8 * m + gi) * L::QP + 16 * kg + 4 * t;
-            const double2 a01 = *reinterpret_cast<const double2*>(qa);
-            const double2 a23 = *reinterpret_cast<const double2*>(qa + 2);
-            a[m][0] = a01.x; a[m][1] = a01.y; a[m][2] = a23.x; a[m][3] = a23.y;
-          }
+        for (int m = 0; m < MT; ++m) {
+          const double* qa = sQ + (8 * m + gi) * L::QP + 16 * kg + 4 * t;
+          const double2 a01 = *reinterpret_cast<const double2*>(qa);
+          const double2 a23 = *reinterpret_cast<const double2*>(qa + 2);
+          a[m][0] = a01.x; a[m][1] = a01.y; a[m][2] = a23.x; a[m][3] = a23.y;
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const double bk = i == 0 ? bv.x : i == 1 ? bv.y : i == 2 ? bv.z : bv.w;
 #pragma unroll
-          for (int m = 0; m < kMaxRows / 8; ++m)
-            if (m < mt) dmma_m8n8k4(acc[c][m], a[m][i], bk);
+          for (int m = 0; m < MT; ++m) dmma_m8n8k4(acc[c][m], a[m][i], bk);
         }
       }
       __syncthreads();  // every warp is done with this buffer
@@ -209,7 +211,7 @@ block_select_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
     for (int c = 0; c < kMaxChunks; ++c)
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const double p = (m < mt && acc[c][m][i] != -INFINITY) ? exp(acc[c][m][i] - M) : 0.0;
+        const double p = (m < MT && acc[c][m][i] != -INFINITY) ? exp(acc[c][m][i] - M) : 0.0;
         acc[c][m][i] = p;
         z += p;
       }
@@ -294,23 +296,26 @@ block_select_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
   if (i == 0) blk_cnt[bg] = total < max_sel ? total : max_sel;
 }
 
-// Fused when the group's query rows fit four MMA row tiles and the keys one
-// thread each; otherwise block scores then selection, as separate kernels.
+// Fused when the group's query rows (G x the bound max_q on q_cnt, or x L_q)
+// fit four MMA row tiles and the keys one thread each; otherwise block scores
+// then selection, as separate kernels.
 cudaError_t launch_block_select(const Shape& s, const void* Q, const int32_t* q_idx,
                                 const int32_t* q_cnt, const float* Kbar, int n_units,
                                 double* score, int unit_size, int topK, const int32_t* sink_pos,
                                 int n_sinks, int32_t* blk_idx, int32_t* blk_cnt, int max_sel,
-                                void* ws, unsigned* err, cudaStream_t st) {
-  if (s.G * s.L_q > bs::kMaxRows || n_units > bs::kMaxUnits) {
+                                int max_q, void* ws, unsigned* err, cudaStream_t st) {
+  const int nq_max = (max_q > 0 && max_q < s.L_q && q_idx) ? max_q : s.L_q;
+  const int rows = s.G * nq_max;
+  if (rows > bs::kMaxRows || n_units > bs::kMaxUnits) {
     cudaError_t e = launch_scores(s, Q, q_idx, q_cnt, Kbar, n_units, score, ws, err, st);
     if (e != cudaSuccess) return e;
     return launch_select(score, s.batch, s.H_kv, n_units, unit_size, topK, sink_pos, n_sinks,
                          blk_idx, blk_cnt, max_sel, err, st);
   }
   cudaError_t e;
-#define DL_BLOCK_SELECT(T, D_)                                                                 \
+#define DL_BLOCK_SELECT_MT(T, D_, MT)                                                          \
   {                                                                                           \
-    auto k = block_select_kernel<T, D_>;                                                      \
+    auto k = block_select_kernel<T, D_, MT>;                                                  \
     constexpr int smem = bs::Smem<T, D_>::BYTES;                                              \
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=   \
         cudaSuccess)                                                                          \
@@ -319,12 +324,22 @@ cudaError_t launch_block_select(const Shape& s, const void* Q, const int32_t* q_
               q_cnt, Kbar, s, n_units, score, unit_size, topK, sink_pos, n_sinks, blk_idx,    \
               blk_cnt, max_sel, err);                                                         \
   }
+  // row tiles for the largest group the caller can produce (one kernel per count)
+#define DL_BLOCK_SELECT(T, D_)                                                                 \
+  switch ((rows + 7) / 8) {                                                                   \
+    case 0:                                                                                   \
+    case 1: DL_BLOCK_SELECT_MT(T, D_, 1) break;                                               \
+    case 2: DL_BLOCK_SELECT_MT(T, D_, 2) break;                                               \
+    case 3: DL_BLOCK_SELECT_MT(T, D_, 3) break;                                               \
+    default: DL_BLOCK_SELECT_MT(T, D_, 4) break;                                              \
+  }
   if (s.dtype == 0) {
     if (s.d == 128) DL_BLOCK_SELECT(__nv_bfloat16, 128) else DL_BLOCK_SELECT(__nv_bfloat16, 64)
   } else {
     if (s.d == 128) DL_BLOCK_SELECT(float, 128) else DL_BLOCK_SELECT(float, 64)
   }
 #undef DL_BLOCK_SELECT
+#undef DL_BLOCK_SELECT_MT
   return cudaGetLastError();
 }
 

@@ -70,7 +70,7 @@ cudaError_t launch_block_select(const Shape& s, const void* Q, const int32_t* q_
                                 const int32_t* q_cnt, const float* Kbar, int n_units,
                                 double* score, int unit_size, int topK, const int32_t* sink_pos,
                                 int n_sinks, int32_t* blk_idx, int32_t* blk_cnt, int max_sel,
-                                void* ws, unsigned* err, cudaStream_t st);
+                                int max_q, void* ws, unsigned* err, cudaStream_t st);
 
 cudaError_t launch_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
                          const int32_t* q_cnt, const void* Kp, const int32_t* page_table,

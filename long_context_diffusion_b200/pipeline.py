@@ -81,8 +81,10 @@ def layer_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec, v
     blk_idx = _empty((B, H_kv, max(max_sel, 1)), torch.int32, dev)
     blk_cnt = _empty((B, H_kv), torch.int32, dev)
     if fused_select:
+        # rows per sequence: the prediction gives at most k windows of 2w+1
+        max_q = min(L_q, k * (2 * w + 1)) if conf_prev is not None else 0
         A.dl_block_select(desc, q_dec, q_idx, q_cnt, Kbar, n_blk, desc.page, topK, sink_pos,
-                          score, blk_idx, blk_cnt, ws, stream)
+                          score, blk_idx, blk_cnt, ws, stream, max_q=max_q)
     else:
         A.dl_block_scores(desc, q_dec, q_idx, q_cnt, Kbar, n_blk, score, ws, stream)
         A.dl_select(score, desc.page, topK, sink_pos, blk_idx, blk_cnt, stream)
@@ -149,6 +151,7 @@ class DenoiseStep:
         B, L_q, d, H, H_kv = desc.batch, desc.L_q, desc.d, desc.H, desc.H_kv
         self.n_blk = -(-desc.L_ctx // desc.page)
         self.max_sel = min(topK, self.n_blk) + n_sinks
+        self.max_q = min(L_q, k * (2 * w + 1))  # predicted rows per sequence, at most
         self.device = device
         self.ws = workspace(desc, device)
         self.q_idx = _empty((B, L_q), torch.int32, device)
@@ -186,7 +189,7 @@ class DenoiseStep:
                                 k_dec[l], self.n_sinks, self.sink_pos, self.ws, stream)
             A.dl_block_select(d, q_dec[l], self.q_idx, self.q_cnt, Kbar[l], self.n_blk, d.page,
                               self.topK, self.sink_pos, self.score, self.blk_idx[l],
-                              self.blk_cnt[l], self.ws, stream)
+                              self.blk_cnt[l], self.ws, stream, max_q=self.max_q)
             ev = self._begin(attn_events, stream)
             A.dl_sparse_attn(d, q_dec[l], k_pool[l], v_pool[l], page_table, self.blk_idx[l],
                              self.blk_cnt[l], k_dec[l], v_dec[l], self.O[l], self.lse[l],

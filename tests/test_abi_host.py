@@ -70,12 +70,14 @@ def test_null_and_range_arguments_rejected_before_launch():
     assert "max_sel" in lib.dl_last_error_message().decode()
     # fused scores + selection: the same checks before any launch
     assert lib.dl_block_select(ctypes.byref(d), fake, None, None, None, 256, 64, 4, None, 0,
-                               fake, fake, fake, 4, fake, 1 << 40, None) == dl.DL_ERR_INVALID_ARG
+                               fake, fake, fake, 4, 0, fake, 1 << 40, None) == dl.DL_ERR_INVALID_ARG
     assert lib.dl_block_select(ctypes.byref(d), fake, None, None, fake, 256, 64, 4, fake, 2,
-                               fake, fake, fake, 5, fake, 1 << 40, None) == dl.DL_ERR_INVALID_ARG
+                               fake, fake, fake, 5, 0, fake, 1 << 40, None) == dl.DL_ERR_INVALID_ARG
     assert "max_sel" in lib.dl_last_error_message().decode()
     assert lib.dl_block_select(ctypes.byref(d), fake, None, None, fake, 256, 64, 4, None, 0,
-                               fake, fake, fake, 4, fake, 256, None) == dl.DL_ERR_WORKSPACE
+                               fake, fake, fake, 4, -1, fake, 1 << 40, None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_block_select(ctypes.byref(d), fake, None, None, fake, 256, 64, 4, None, 0,
+                               fake, fake, fake, 4, 0, fake, 256, None) == dl.DL_ERR_WORKSPACE
     # misaligned attention pointers
     odd = ctypes.c_void_p(0x1008)
     st = lib.dl_sparse_attn(ctypes.byref(d), odd, fake, fake, fake, None, None, 0, fake, fake,

@@ -110,9 +110,12 @@ def test_select_all_paths(n_units, topK, cuda_device):
     (513, 4, 4, 128, 32, [20, 9], 64, "bf16"),        # separate kernels: more than 512 keys
     (100, 8, 2, 128, 32, [20, 32], 10, "bf16"),       # separate kernels: 4 x 32 rows
 ])
-def test_block_select_matches_oracle(n_units, H, H_kv, d, L_q, cnts, topK, dtype, cuda_device):
+@pytest.mark.parametrize("tight", [False, True])
+def test_block_select_matches_oracle(n_units, H, H_kv, d, L_q, cnts, topK, dtype, tight,
+                                     cuda_device):
     """dl_block_select (fused score + select) against the oracle, and against
-    dl_block_scores followed by dl_select."""
+    dl_block_scores followed by dl_select; with max_q = L_q (0) and with the
+    tightest bound max(q_cnt) (fewer MMA row tiles)."""
     batch, n_sinks, unit = len(cnts), 3, 64
     G = H // H_kv
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
@@ -141,7 +144,8 @@ def test_block_select_matches_oracle(n_units, H, H_kv, d, L_q, cnts, topK, dtype
         cnt = torch.full((batch, H_kv), -7, dtype=torch.int32, device=cuda_device)
         if fused:
             dl.dl_block_select(desc, dev(q), dev(q_idx), dev(q_cnt), dev(kbar), n_units, unit,
-                               topK, dev(sink_pos), score, blk, cnt, ws)
+                               topK, dev(sink_pos), score, blk, cnt, ws,
+                               max_q=max(max(cnts), 1) if tight else 0)
         else:
             dl.dl_block_scores(desc, dev(q), dev(q_idx), dev(q_cnt), dev(kbar), n_units, score,
                                ws)
@@ -163,3 +167,26 @@ def test_block_select_matches_oracle(n_units, H, H_kv, d, L_q, cnts, topK, dtype
             assert c_f[b, g] == len(sel)
             assert np.array_equal(b_f[b, g, :len(sel)], sel)
             assert (b_f[b, g, len(sel):] == -1).all()
+
+
+def test_block_select_rows_past_the_bound_are_reported(cuda_device):
+    """A sequence with more predicted rows than max_q: reported through the
+    device error word (its rows are cut to the bound), nothing traps."""
+    batch, H, H_kv, d, L_q, n_units, unit = 2, 8, 8, 128, 32, 256, 64
+    q = (synth.normals(SEED, 9900, 0, batch * H * L_q * d).reshape(batch, H, L_q, d) * 0.7).to(
+        torch.bfloat16)
+    kbar = (synth.normals(SEED, 9901, 0, batch * H_kv * n_units * d) * 0.5).to(
+        torch.float32).reshape(batch, H_kv, n_units, d)
+    q_idx = torch.arange(L_q, dtype=torch.int32).repeat(batch, 1)
+    q_cnt = torch.tensor([12, 20], dtype=torch.int32)
+    desc = _desc(batch, H, H_kv, d, L_q, n_units, "bf16")
+    ws = torch.empty(max(dl.dl_workspace_size(desc), 256), dtype=torch.uint8, device=cuda_device)
+    score = torch.empty((batch, H_kv, n_units), dtype=torch.float64, device=cuda_device)
+    blk = torch.empty((batch, H_kv, 8), dtype=torch.int32, device=cuda_device)
+    cnt = torch.empty((batch, H_kv), dtype=torch.int32, device=cuda_device)
+    dl.dl_block_select(desc, q.to(cuda_device), q_idx.to(cuda_device), q_cnt.to(cuda_device),
+                       kbar.to(cuda_device), n_units, unit, 8, None, score, blk, cnt, ws,
+                       max_q=16)
+    assert dl.dl_get_status() == dl.DL_ERR_BAD_INDEX
+    assert torch.isfinite(score).all()
+    assert dl.dl_get_status() == dl.DL_OK
