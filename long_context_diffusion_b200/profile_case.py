@@ -52,9 +52,11 @@ def main():
     O = torch.empty((wl.batch, wl.L_q, wl.H, wl.d), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((wl.batch, wl.H, wl.L_q), dtype=torch.float32, device=dev)
 
+    max_q = min(wl.L_q, wl.k * (2 * wl.w + 1))  # the bound DenoiseStep passes
+
     def block_select():
         A.dl_block_select(desc, q, q_idx, q_cnt, Kbar, wl.n_blk, wl.B, wl.topK, sinks, score,
-                          blk, cnt, ws)
+                          blk, cnt, ws, max_q=max_q)
 
     calls = {
         "block_select": block_select,
