@@ -51,35 +51,43 @@ namespace kt {
 
 constexpr int D = 128;
 constexpr int NQ = 32;                     // query rows (MMA N)
-constexpr int STK = 3;                     // K ring stages (two pages each)
-constexpr int STV = 2;                     // V ring stages
 constexpr int QB = 2;                      // Q buffers (alternating segments)
 constexpr int Q_BYTES = 2 * NQ * 128;      // [d-half][32 rows][128 B]
 constexpr int KS_BYTES = 2 * 128 * 128;    // [d-half][128 keys][128 B]
 constexpr int PT_BYTES = 128 * 128;        // [128 keys][128 B] (64 B used)
 constexpr int MAX_STEPS = kTcMaxTiles / 2 + kMaxSegs;
-constexpr int Q_OFF = 0;
-constexpr int K_OFF = Q_OFF + QB * Q_BYTES;
-constexpr int V_OFF = K_OFF + STK * KS_BYTES;
-constexpr int PT_OFF = V_OFF + STV * KS_BYTES;
-constexpr int RED_OFF = PT_OFF + 2 * PT_BYTES;   // float [4][32] maxima, [4][32] sums
-constexpr int FLAG_OFF = RED_OFF + 2 * 4 * NQ * 4;  // int [2][4] rescale votes
-constexpr int BAR_OFF = FLAG_OFF + 2 * 4 * 4;
-// full_k, empty_k [STK]; full_v, empty_v [STV]; q_full, q_free, s_full,
-// p_ready, pv_done, o_free, xbar [2]; mxbar, lbar
-constexpr int N_BARS = 2 * STK + 2 * STV + 7 * 2 + 2;
-constexpr int MISC_OFF = (BAR_OFF + N_BARS * 8 + 15) / 16 * 16;
-constexpr int STEP_OFF = MISC_OFF + 32;                  // int4 [MAX_STEPS]
-constexpr int SEG_OFF = STEP_OFF + MAX_STEPS * 16;       // int4 [kMaxSegs]
-constexpr int MARK_OFF = SEG_OFF + kMaxSegs * 16;        // int2 [kMaxSegs]
-constexpr int SEGHI_OFF = MARK_OFF + kMaxSegs * 8;       // int [kMaxSegs]
-constexpr int NCTX_OFF = SEGHI_OFF + kMaxSegs * 4;       // int [kMaxSegs]
-constexpr int SMEM = NCTX_OFF + kMaxSegs * 4 + 1024;     // + alignment slack
 constexpr int THREADS = 256;
 constexpr uint32_t TMEM_COLS = 128;  // S^T [2][32] at 0, O^T [2][32] at 64
 constexpr uint32_t S_COL = 0, O_COL = 64;
-static_assert(SMEM <= 232448, "shared memory budget");
-static_assert(BAR_OFF % 16 == 0 && STEP_OFF % 16 == 0 && SEG_OFF % 16 == 0, "alignment");
+
+// Shared-memory layout.  Attention: a K ring of three two-page stages and a V
+// ring of two (a third V stage measured slower), two P^T tiles.  LSE-only
+// (the first pass of the sink search): no V, no P^T, so six K stages.
+template <bool LSE>
+struct Layout {
+  static constexpr int STK = LSE ? 6 : 3;
+  static constexpr int STV = LSE ? 0 : 2;
+  static constexpr int NPT = LSE ? 0 : 2;
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + QB * Q_BYTES;
+  static constexpr int V_OFF = K_OFF + STK * KS_BYTES;
+  static constexpr int PT_OFF = V_OFF + STV * KS_BYTES;
+  static constexpr int RED_OFF = PT_OFF + NPT * PT_BYTES;   // float [4][32] maxima, [4][32] sums
+  static constexpr int FLAG_OFF = RED_OFF + 2 * 4 * NQ * 4;  // int [2][4] rescale votes
+  static constexpr int BAR_OFF = FLAG_OFF + 2 * 4 * 4;
+  // full_k, empty_k [STK]; full_v, empty_v [STV]; q_full, q_free, s_full,
+  // p_ready, pv_done, o_free, xbar [2]; mxbar, lbar
+  static constexpr int N_BARS = 2 * STK + 2 * STV + 7 * 2 + 2;
+  static constexpr int MISC_OFF = (BAR_OFF + N_BARS * 8 + 15) / 16 * 16;
+  static constexpr int STEP_OFF = MISC_OFF + 32;                  // int4 [MAX_STEPS]
+  static constexpr int SEG_OFF = STEP_OFF + MAX_STEPS * 16;       // int4 [kMaxSegs]
+  static constexpr int MARK_OFF = SEG_OFF + kMaxSegs * 16;        // int2 [kMaxSegs]
+  static constexpr int SEGHI_OFF = MARK_OFF + kMaxSegs * 8;       // int [kMaxSegs]
+  static constexpr int NCTX_OFF = SEGHI_OFF + kMaxSegs * 4;       // int [kMaxSegs]
+  static constexpr int SMEM = NCTX_OFF + kMaxSegs * 4 + 1024;     // + alignment slack
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(BAR_OFF % 16 == 0 && STEP_OFF % 16 == 0 && SEG_OFF % 16 == 0, "alignment");
+};
 
 // After the call, lane L holds op over the 32 lanes of v[L] (v is clobbered):
 // a butterfly in which each level keeps half of the entries and trades the
@@ -108,12 +116,20 @@ __device__ __forceinline__ bool page_dec(int info) { return (info >> 15) & 1; }
 
 }  // namespace kt
 
+template <bool LSE>
 __global__ void __launch_bounds__(kt::THREADS, 1)
 attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v,
                   const __grid_constant__ CUtensorMap tm_kd,
                   const __grid_constant__ CUtensorMap tm_vd, const AttnArgs a, const TcPlan plan) {
   using namespace kt;
+  using Lk = Layout<LSE>;
+  constexpr int STK = Lk::STK, STV = Lk::STV;
+  constexpr int STVd = STV > 0 ? STV : 1;  // divisor in the (LSE-unreachable) V paths
+  constexpr int Q_OFF = Lk::Q_OFF, K_OFF = Lk::K_OFF, V_OFF = Lk::V_OFF, PT_OFF = Lk::PT_OFF;
+  constexpr int RED_OFF = Lk::RED_OFF, FLAG_OFF = Lk::FLAG_OFF, BAR_OFF = Lk::BAR_OFF;
+  constexpr int MISC_OFF = Lk::MISC_OFF, STEP_OFF = Lk::STEP_OFF, SEG_OFF = Lk::SEG_OFF;
+  constexpr int MARK_OFF = Lk::MARK_OFF, SEGHI_OFF = Lk::SEGHI_OFF, NCTX_OFF = Lk::NCTX_OFF;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sQ = smem + Q_OFF;
@@ -149,7 +165,7 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   const Shape& s = a.s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool lse_only = a.O == nullptr;  // row LSEs only: no V, no P V, no O
+  constexpr bool lse_only = LSE;  // row LSEs only: no V, no P V, no O
   // tensor memory first; the successor may be scheduled only after that
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -245,7 +261,7 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint8_t* ring = is_k ? sK : sV;
     const CUtensorMap* map = is_k ? &tm_k : &tm_v;
     const CUtensorMap* map_dec = is_k ? &tm_kd : &tm_vd;
-    const int ST = is_k ? STK : STV;
+    const int ST = is_k ? STK : STVd;
     if (lane == 0 && nst > 0 && (is_k || !lse_only)) {
       prefetch_tmap(map);
       prefetch_tmap(map_dec);
@@ -341,8 +357,8 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           const int ob = k & 1;
           if (first && k >= 2 && !(ok = mbar_wait(&o_free[ob], ((k - 2) >> 1) & 1, abort_flag)))
             break;
-          const int st = j % STV;
-          if (!(ok = mbar_wait(&full_v[st], (j / STV) & 1, abort_flag))) break;
+          const int st = j % STVd;
+          if (!(ok = mbar_wait(&full_v[st], (j / STVd) & 1, abort_flag))) break;
           tc_fence_after();
           const uint64_t ad0 = v_desc0 + (uint64_t)((st * KS_BYTES) >> 4);
           const uint64_t bd0 = p_desc0 + (uint64_t)((buf * PT_BYTES) >> 4);
@@ -406,7 +422,7 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const bool first = first_of(j);
       const bool last = last_of(j);
       const int buf = j & 1;
-      const int st = j % STV;
+      const int st = j % STVd;
       const int pinfo = (key < 64) ? (e.z & 0xFFFF) : e.w;
       const int pvalid = page_valid(pinfo);
       const bool kvalid = (key & 63) < pvalid;
@@ -490,7 +506,7 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (!kvalid && pvalid > 0) {
         // a loaded page's rows past its valid keys may hold anything (even
         // NaN): zero this key's V row once it has landed
-        ok = mbar_wait(&full_v[st], (j / STV) & 1, abort_flag);
+        ok = mbar_wait(&full_v[st], (j / STVd) & 1, abort_flag);
         if (ok) {
           uint8_t* vr = sV + st * KS_BYTES + key * 128;
 #pragma unroll
@@ -551,10 +567,22 @@ cudaError_t launch_attn_tc_kt(const AttnArgs& a, int max_tiles, cudaStream_t st)
     return cudaErrorInvalidValue;
   const TcLaunch L = tc_plan((int)n_bg, max_tiles, tc_sm_count());
   if (L.plan.nslot > kMaxSplits) return cudaErrorInvalidValue;  // workspace bound
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kt_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kt::SMEM);
-  if (e != cudaSuccess) return e;
-  DL_LAUNCH(attn_tc_kt_kernel, L.grid, kt::THREADS, kt::SMEM, st, mq, mk, mv, mkd, mvd, a, L.plan);
+  cudaError_t e;
+  if (a.O == nullptr) {  // the row LSEs only
+    constexpr int smem = kt::Layout<true>::SMEM;
+    if ((e = cudaFuncSetAttribute(attn_tc_kt_kernel<true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+      return e;
+    DL_LAUNCH(attn_tc_kt_kernel<true>, L.grid, kt::THREADS, smem, st, mq, mk, mv, mkd, mvd, a,
+              L.plan);
+  } else {
+    constexpr int smem = kt::Layout<false>::SMEM;
+    if ((e = cudaFuncSetAttribute(attn_tc_kt_kernel<false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+      return e;
+    DL_LAUNCH(attn_tc_kt_kernel<false>, L.grid, kt::THREADS, smem, st, mq, mk, mv, mkd, mvd, a,
+              L.plan);
+  }
   return launch_combine(a, L.plan.nslot, st, L.plan.S, L.grid);
 }
 

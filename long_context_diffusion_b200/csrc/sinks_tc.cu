@@ -5,9 +5,10 @@
 // head h and predicted row i of exp(scale q_hi . k_t - LSE_hi), where LSE_hi
 // is the row's log-sum-exp over the whole context plus the decode block.
 //
-// Pass 1 (the LSEs) is the tensor-core attention kernel in dense mode with V
-// taken equal to K (the V tile is the K tile just fetched, so it comes from
-// L2), which returns the natural-log LSE of every decode row.
+// Pass 1 (the LSEs) is the tensor-core attention kernel in dense mode, in
+// its LSE-only form where it has one (when the key-major kernel takes the
+// shape: no V, no P V, no O), otherwise with V taken equal to K; it returns
+// the natural-log LSE of every decode row.
 //
 // Pass 2 (this file) computes S^T = K Q^T with the keys as the MMA's M
 // dimension: 128 keys (two pages) on the 128 TMEM lanes and the predicted
@@ -30,7 +31,7 @@ namespace dl {
 
 using namespace sm100;
 
-constexpr int kMassMaxStages = 4;
+constexpr int kMassMaxStages = 6;
 constexpr int kMassMaxPairs = 64;  // page pairs per CTA
 
 struct MassArgs {
@@ -43,7 +44,7 @@ struct MassArgs {
   float* mass;            // [b][L_ctx]
   int n_pad;              // N of the MMA: G*L_q rounded up to 32
   int pairs_per_cta;
-  int stages;             // K tiles in flight (2..4, as shared memory allows)
+  int stages;             // K tiles in flight (2..6, as shared memory allows)
   unsigned* err;
 };
 
