@@ -1,5 +1,5 @@
 // sm_100a building blocks written as inline PTX: mbarriers with bounded
-// waits, TMA tile loads (no multicast), tcgen05 MMA / TMEM access, and the
+// waits, TMA tile loads into this CTA only, tcgen05 MMA / TMEM access, and the
 // shared-memory and instruction descriptors of tcgen05.mma kind::f16.
 //
 // Descriptor layouts (tcgen05 "matrix descriptor" and "instruction
