@@ -49,9 +49,9 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 
 # DRAM traffic of the dominant kernel from one ncu capture at the benchmark's
 # size (profiles/attn_tc_kt_sparse_llada32k.md: dram__bytes_read.sum +
-# dram__bytes_write.sum of one sparse-layer launch, batch 4: 557.85 + 5.86 MB).
+# dram__bytes_write.sum of one sparse-layer launch, batch 4: 557.93 + 8.33 MB).
 # Reported only while the kernel's sources hash to the captured build.
-TRAFFIC_CAPTURE = {"sha": "fb06682a9ceea044", "bytes_per_launch": 557.849088e6 + 5.863424e6,
+TRAFFIC_CAPTURE = {"sha": "c35242f1710dd185", "bytes_per_launch": 557.928192e6 + 8.3264e6,
                    "sources": ["attn_tc_kt.cu", "tc_common.cuh", "sm100.cuh"]}
 
 
