@@ -17,9 +17,10 @@
 // no cross-thread reduction.  One CTA owns a run of page pairs of one
 // sequence and loops over the KV groups (outer) and its page pairs (inner),
 // accumulating each key's mass in shared memory in group order, then writes
-// it.  Roles: warp 0 = TMA producer, warp 1 = MMA issuer, warp 2 = gathers
-// the predicted Q rows (and their LSEs) of the next group, warps 4-7 =
-// epilogue.  Every wait is bounded.
+// it.  Roles: warp 0 = TMA producer, warp 1 = MMA issuer, warps 2-3 = gather
+// the predicted Q rows (and their LSEs) of the next group, every lane with
+// up to eight 16-byte loads in flight, warps 4-7 = epilogue.  Every wait is
+// bounded.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -55,7 +56,7 @@ struct MassCfg {
   __host__ __device__ static size_t q_bytes(int n_pad) { return (size_t)HALVES * n_pad * 128; }
   static size_t smem(int n_pad, int pairs, int stages) {
     return 1024 + 2 * q_bytes(n_pad) + (size_t)stages * KT_BYTES + 2 * 256 * 4 +
-           (size_t)pairs * 128 * 4 + 64 * 8 + 64;
+           (size_t)pairs * 128 * 4 + 64 * 8 + 64 + 256 * 4;
   }
 };
 
@@ -81,6 +82,7 @@ sink_mass_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const MassArgs a) 
   uint64_t* s_free = s_full + 2;                    // [2]  (128 epilogue)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_free + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_qidx = reinterpret_cast<int*>(bars + 64) + 16;  // [L_q <= 256] predicted rows
 
   const int b = blockIdx.y;
   const int n_ctx_pages = (s.L_ctx + 63) / 64;
@@ -107,7 +109,7 @@ sink_mass_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const MassArgs a) 
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&q_full[i], 32);
+      mbar_init(&q_full[i], 64);
       mbar_init(&q_empty[i], 1 + 128);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
@@ -116,6 +118,7 @@ sink_mass_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const MassArgs a) 
     fence_mbar_init();
   }
   for (int e = threadIdx.x; e < np * 128; e += blockDim.x) s_mass[e] = 0.0f;
+  for (int i = threadIdx.x; i < nq; i += blockDim.x) s_qidx[i] = a.q_idx[(size_t)b * s.L_q + i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -185,10 +188,13 @@ sink_mass_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const MassArgs a) 
       if (*abort_flag)
         for (uint32_t k = 0; k < (1u << 16); ++k) __nanosleep(1000);
     }
-  } else if (n_tiles > 0 && warp == 2) {
+  } else if (n_tiles > 0 && (warp == 2 || warp == 3)) {
     // ------------------------------------------------------------ Q gather
+    constexpr int per_row = C::HALVES * 8;  // 16-byte chunks
+    constexpr int IN_FLIGHT = 8;
     const float log2e = 1.4426950408889634f;
-    const int per_row = C::HALVES * 8;  // 16-byte chunks
+    const int gt = threadIdx.x - 64;  // 0..63
+    const int total = n_pad * per_row;
     for (int g = 0; g < s.H_kv; ++g) {
       const int qb = g & 1;
       if (g >= 2) {
@@ -196,26 +202,38 @@ sink_mass_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const MassArgs a) 
         if (!__all_sync(0xffffffffu, w)) break;
       }
       uint8_t* dst = sQ + qb * QB;
-      for (int e = lane; e < n_pad * per_row; e += 32) {
-        const int n = e / per_row, rem = e % per_row;
-        const int h_half = rem >> 3, ch = rem & 7;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (n < Rg) {
-          const int h = g * s.G + n / nq;
-          const int i = a.q_idx[(size_t)b * s.L_q + (n % nq)];
-          if (i >= 0 && i < s.L_q) {
-            const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.Q) +
-                                       (((size_t)b * s.H + h) * s.L_q + i) * D + rem * 8;
-            v = __ldg(reinterpret_cast<const uint4*>(src));
+      for (int e0 = 0; e0 < total; e0 += 64 * IN_FLIGHT) {
+        uint4 v[IN_FLIGHT];
+#pragma unroll
+        for (int u = 0; u < IN_FLIGHT; ++u) {  // every load issued before any store
+          const int e = e0 + u * 64 + gt;
+          const int n = e / per_row, rem = e % per_row;
+          v[u] = make_uint4(0u, 0u, 0u, 0u);
+          if (e < total && n < Rg) {
+            const int h = g * s.G + n / nq;
+            const int i = s_qidx[n % nq];
+            if (i >= 0 && i < s.L_q) {
+              const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.Q) +
+                                         (((size_t)b * s.H + h) * s.L_q + i) * D + rem * 8;
+              v[u] = __ldg(reinterpret_cast<const uint4*>(src));
+            }
           }
         }
-        *reinterpret_cast<uint4*>(dst + h_half * n_pad * 128 + n * 128 + ((ch ^ (n & 7)) << 4)) = v;
+#pragma unroll
+        for (int u = 0; u < IN_FLIGHT; ++u) {
+          const int e = e0 + u * 64 + gt;
+          if (e >= total) continue;
+          const int n = e / per_row, rem = e % per_row;
+          const int h_half = rem >> 3, ch = rem & 7;
+          *reinterpret_cast<uint4*>(dst + h_half * n_pad * 128 + n * 128 + ((ch ^ (n & 7)) << 4)) =
+              v[u];
+        }
       }
-      for (int n = lane; n < n_pad; n += 32) {
+      for (int n = gt; n < n_pad; n += 64) {
         float l2 = INFINITY;  // padded rows contribute exp2(-inf) = 0
         if (n < Rg) {
           const int h = g * s.G + n / nq;
-          const int i = a.q_idx[(size_t)b * s.L_q + (n % nq)];
+          const int i = s_qidx[n % nq];
           if (i >= 0 && i < s.L_q) l2 = a.lse[((size_t)b * s.H + h) * s.L_q + i] * log2e;
         }
         s_lse2[qb * 256 + n] = l2;

@@ -2,6 +2,7 @@
 
     python -m long_context_diffusion_b200.profile_case --case attn_sparse --reps 3
     python -m long_context_diffusion_b200.profile_case --case block_select --reps 3
+    python -m long_context_diffusion_b200.profile_case --case sinks --reps 3
 
 Builds one sparse layer of the 32K workload (batch 4, 32 KV heads, 32K context:
 about 2.1 GB of K/V pages on the device), runs the steps before the profiled
@@ -21,7 +22,7 @@ from . import _abi as A
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["attn_sparse", "attn_dense", "block_select", "pool"],
+    ap.add_argument("--case", choices=["attn_sparse", "attn_dense", "block_select", "pool", "sinks"],
                     required=True)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--batch", type=int, default=4)
@@ -65,6 +66,8 @@ def main():
         "attn_dense": lambda: A.dl_sparse_attn(desc, q, kp, vp, pt, None, None, kd, vd, O, lse,
                                                ws),
         "pool": lambda: A.dl_pool_keys(desc, kp, pt, wl.n_blk, wl.B, 0, wl.B, Kbar),
+        "sinks": lambda: A.dl_find_sinks(desc, q, q_idx, q_cnt, kp, pt, kd, wl.detect_sinks,
+                                         sinks, ws),
     }
     if args.case.startswith("attn"):
         block_select()
