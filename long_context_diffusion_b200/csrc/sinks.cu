@@ -228,8 +228,10 @@ sink_mass_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q
   if (in_range) w.mass[(size_t)b * s.L_ctx + t] = mass;
 }
 
+// Top-n columns by mass (ties to the lower position), ascending.  Any n:
+// n rounds of a block argmax over a scan of the masses.
 __global__ void __launch_bounds__(1024)
-sink_topn_kernel(Shape s, int n_sinks, SinkWs w, int32_t* __restrict__ sink_pos) {
+sink_topn_scan_kernel(Shape s, int n_sinks, SinkWs w, int32_t* __restrict__ sink_pos) {
   pdl_trigger();
   pdl_wait();
   __shared__ float sv[32];
@@ -265,6 +267,116 @@ sink_topn_kernel(Shape s, int n_sinks, SinkWs w, int32_t* __restrict__ sink_pos)
   }
 }
 
+// n <= KL: one pass in which every thread keeps the KL largest masses of its
+// own positions (descending; a thread meets its positions in increasing order,
+// so equal masses keep the lower position first), then n rounds of a block
+// argmax over the threads' leading entries, the winner dropping its lead.
+// Every global top-n column is among its thread's top n, so the result is
+// that of the scan.
+template <int KL>
+__global__ void __launch_bounds__(512)
+sink_topn_kernel(Shape s, int n_sinks, const float* __restrict__ mass_all,
+                 int32_t* __restrict__ sink_pos) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float sv[32];
+  __shared__ int si[32];
+  __shared__ int chosen[KL];
+  constexpr int U = 8;  // loads in flight per thread
+  const int b = blockIdx.x;
+  const float* mass = mass_all + (size_t)b * s.L_ctx;
+  float lv[KL];
+  int li[KL];
+#pragma unroll
+  for (int k = 0; k < KL; ++k) {
+    lv[k] = -INFINITY;
+    li[k] = 0x7fffffff;
+  }
+  auto push = [&](float m, int t) {
+    if (!(m > lv[KL - 1])) return;
+    lv[KL - 1] = m;
+    li[KL - 1] = t;
+#pragma unroll
+    for (int k = KL - 1; k > 0; --k) {
+      if (lv[k] > lv[k - 1]) {
+        const float tv = lv[k]; lv[k] = lv[k - 1]; lv[k - 1] = tv;
+        const int ti = li[k]; li[k] = li[k - 1]; li[k - 1] = ti;
+      }
+    }
+  };
+  const int L = s.L_ctx;
+  if ((L & 3) == 0 && (reinterpret_cast<uintptr_t>(mass) & 15) == 0) {
+    const float4* m4 = reinterpret_cast<const float4*>(mass);
+    const int n4 = L >> 2;
+    for (int base = threadIdx.x; base < n4; base += U * blockDim.x) {
+      float4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = base + u * blockDim.x;
+        v[u] = i < n4 ? __ldg(m4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = base + u * blockDim.x;
+        if (i < n4) {
+          push(v[u].x, 4 * i);
+          push(v[u].y, 4 * i + 1);
+          push(v[u].z, 4 * i + 2);
+          push(v[u].w, 4 * i + 3);
+        }
+      }
+    }
+  } else {
+    for (int base = threadIdx.x; base < L; base += U * blockDim.x) {
+      float v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = base + u * blockDim.x;
+        v[u] = i < L ? __ldg(mass + i) : 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (base + u * (int)blockDim.x < L) push(v[u], base + u * blockDim.x);
+    }
+  }
+  for (int r = 0; r < n_sinks; ++r) {
+    float bv;
+    int bi;
+    block_argmax(lv[0], li[0], sv, si, bv, bi);
+    const bool found = bv != -INFINITY && bi < L;
+    if (found && li[0] == bi) {  // positions are unique: this thread led
+#pragma unroll
+      for (int k = 0; k < KL - 1; ++k) {
+        lv[k] = lv[k + 1];
+        li[k] = li[k + 1];
+      }
+      lv[KL - 1] = -INFINITY;
+      li[KL - 1] = 0x7fffffff;
+    }
+    if (threadIdx.x == 0) chosen[r] = found ? bi : -1;
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < n_sinks; ++i) {  // insertion sort, ascending
+      const int x = chosen[i];
+      int j = i - 1;
+      while (j >= 0 && chosen[j] > x) { chosen[j + 1] = chosen[j]; --j; }
+      chosen[j + 1] = x;
+    }
+    for (int i = 0; i < n_sinks; ++i) sink_pos[(size_t)b * n_sinks + i] = chosen[i];
+  }
+}
+
+static cudaError_t launch_sink_topn(const Shape& s, int n_sinks, const SinkWs& w,
+                                    int32_t* sink_pos, cudaStream_t st) {
+  if (n_sinks <= 8) {
+    DL_LAUNCH(sink_topn_kernel<8>, s.batch, 512, 0, st, s, n_sinks, (const float*)w.mass,
+              sink_pos);
+  } else {
+    DL_LAUNCH(sink_topn_scan_kernel, s.batch, 1024, 0, st, s, n_sinks, w, sink_pos);
+  }
+  return cudaGetLastError();
+}
+
 template <typename T, int D>
 static cudaError_t run_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
                              const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
@@ -283,8 +395,7 @@ static cudaError_t run_sinks(const Shape& s, const void* Q, const int32_t* q_idx
   DL_LAUNCH(sink_mass_kernel<T, D>, dim3((s.L_ctx + kSinkTile - 1) / kSinkTile, s.batch), kSinkTile, 0,
                            st, s, q, q_idx, q_cnt, kp, page_table, w, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  DL_LAUNCH(sink_topn_kernel, s.batch, 1024, 0, st, s, n_sinks, w, sink_pos);
-  return cudaGetLastError();
+  return launch_sink_topn(s, n_sinks, w, sink_pos, st);
 }
 
 bool attn_tc_supported(const AttnArgs& a);
@@ -316,8 +427,7 @@ cudaError_t launch_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
     if (e != cudaSuccess) return e;
     SinkWs w = sink_ws(ws, s);
     w.mass = tw.mass;
-    DL_LAUNCH(sink_topn_kernel, s.batch, 1024, 0, st, s, n_sinks, w, sink_pos);
-    return cudaGetLastError();
+    return launch_sink_topn(s, n_sinks, w, sink_pos, st);
   }
   if (s.dtype == 0)
     return s.d == 128 ? run_sinks<__nv_bfloat16, 128>(s, Q, q_idx, q_cnt, Kp, page_table, Kd,

@@ -11,7 +11,7 @@ import oracle
 import synth
 from long_context_diffusion_b200 import pipeline
 from oracle import steps as S
-from tests.helpers import check_attention, desc_for, np_
+from tests.helpers import check_attention, cut_margin, desc_for, np_
 
 pytestmark = pytest.mark.gpu
 
@@ -77,6 +77,39 @@ def test_find_sinks_recovers_planted(name, cuda_device):
             # query) dominates; averaged over a GQA group of 7 it does not, so
             # there only the match with the oracle is required
             assert top.tolist() == np_(inp.sinks_planted)[b].tolist()
+
+
+@pytest.mark.parametrize("name,n", [("tiny", 1), ("tiny", 12), ("llada8k", 1), ("llada8k", 8),
+                                    ("llada8k", 12)])
+def test_find_sinks_top_n(name, n, cuda_device):
+    """n sinks through both top-n kernels (one pass for n <= 8, rounds of a
+    scan beyond): ascending, distinct, equal to the oracle's where its cut has
+    a margin above the fp32 mass error, else within that error of the cut."""
+    wl = synth.workload(name)
+    inp = synth.make_step_inputs(wl, device=cuda_device)
+    desc = desc_for(wl)
+    q_idx = torch.empty((wl.batch, wl.L_q), dtype=torch.int32, device=cuda_device)
+    q_cnt = torch.empty((wl.batch,), dtype=torch.int32, device=cuda_device)
+    dl.dl_predict_queries(inp.conf_prev, inp.still_masked, wl.k, wl.w, q_idx, q_cnt)
+    ws = pipeline.workspace(desc, cuda_device)
+    sinks = torch.empty((wl.batch, n), dtype=torch.int32, device=cuda_device)
+    dl.dl_find_sinks(desc, inp.q_dec, q_idx, q_cnt, inp.k_pool, inp.page_table, inp.k_dec, n,
+                     sinks, ws)
+    assert dl.dl_get_status() == dl.DL_OK
+    qi, qc = np_(q_idx), np_(q_cnt)
+    for b in range(wl.batch):
+        Kc = np.stack([S.gather_context(np_(inp.k_pool), np_(inp.page_table)[b], g,
+                                        np.arange(wl.L_ctx), wl.B) for g in range(wl.H_kv)])
+        top, mass = S.find_sinks(np_(inp.q_dec)[b], Kc, np_(inp.k_dec)[b], qi[b, : qc[b]], n,
+                                 S.scale_for(wl.d))
+        got = np_(sinks)[b]
+        assert got.tolist() == sorted(set(got.tolist())) and len(got) == n
+        assert got.min() >= 0 and got.max() < wl.L_ctx
+        tol = 1e-5 * mass.max()
+        if cut_margin(mass, top) > tol:
+            assert got.tolist() == top.tolist()
+        else:
+            assert (mass[got] >= np.sort(mass)[-n] - tol).all()
 
 
 def test_chunked_prefix_workload(cuda_device):
