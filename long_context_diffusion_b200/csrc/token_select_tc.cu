@@ -1,0 +1,530 @@
+// (a7) Intra-chunk token selection on the sm_100a tensor cores (bf16, d 128).
+//
+// Prefilling-dLLM abstract: the prefix is split into chunks cached once; the
+// top-K chunks are kept with intra-chunk token sparsity, and the BOS token
+// prepended to each chunk acts as an attention anchor.  For one selected
+// chunk of one KV group, every decode query row r of the group gives
+// p_rt = softmax over the chunk's content tokens t of scale q_r . k_t, the
+// token's mass is tau_t = sum_r p_rt, and the top-T tokens by (mass
+// descending, position ascending) are kept with the chunk's BOS.
+//
+// One CTA per (b, g, selected chunk).  The chunk starts on a page boundary,
+// so its first 1024 positions (the BOS and content tokens 1..1023) are eight
+// tiles of two 64-key pages; a content token at position 1024 (a chunk of
+// 1024 content tokens) is scored on the CUDA cores.  Keys are the MMA's M
+// side: S^T [128 keys x N rows] = K_tile . Q^T for each tile, all eight tiles
+// resident in TMEM at once (8 x N <= 512 columns).  Then, with thread =
+// TMEM lane = key of a tile (8 warps, four tiles each): pass 1 takes each
+// row's maximum; pass 2 the exponentials 2^(x - max) (written back over S^T)
+// and each row's sum; pass 3 each key's mass, the sum over rows of its
+// exponentials divided by the row sums.  The top-T cut is a radix select on
+// the masses' bit patterns (non-negative floats order as integers) with the
+// tied entries at the cut taken in position order; the kept tokens are
+// written in ascending position order.
+//
+// Roles while streaming: warp 0 one thread: TMA of the K tiles (a ring of
+// four); warp 1 one thread: the MMAs; warps 2-3: gather the query rows into
+// shared memory; warps 4-5: the score of the token past the tiles.  Every
+// wait is bounded.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+#include "launch.cuh"
+
+namespace dl {
+
+using namespace sm100;
+
+namespace ts {
+
+constexpr int D = 128;
+constexpr int MAX_TILES = 8;              // 8 tiles x 128 keys = 1024 positions
+constexpr int STAGES = 4;
+constexpr int KT_BYTES = 2 * 128 * 128;   // [d-half][128 keys][128 B]
+constexpr int THREADS = 256;
+constexpr int MAXC = 1024;                // content tokens per chunk
+
+template <int N>
+struct Layout {
+  static constexpr int Q_BYTES = 2 * N * 128;           // [d-half][N rows][128 B]
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + Q_BYTES;
+  static constexpr int RED_OFF = K_OFF + STAGES * KT_BYTES;  // float [8 warps][N]
+  static constexpr int ROW_OFF = RED_OFF + 8 * N * 4;       // float [4][N]: M, 1/Z, x_left, e_left
+  static constexpr int TAU_OFF = ROW_OFF + 4 * N * 4;       // uint32 [MAXC] mass keys
+  static constexpr int HIST_OFF = TAU_OFF + MAXC * 4;       // int [256]
+  static constexpr int SCAN_OFF = HIST_OFF + 256 * 4;       // int [40]
+  static constexpr int PV_OFF = SCAN_OFF + 40 * 4;          // int [2 * MAX_TILES + 1] page valid
+  static constexpr int BAR_OFF = (PV_OFF + (2 * MAX_TILES + 1) * 4 + 15) / 16 * 16;
+  // full, empty [STAGES]; q_full; s_done
+  static constexpr int N_BARS = 2 * STAGES + 2;
+  static constexpr int MISC_OFF = BAR_OFF + N_BARS * 8;      // tmem slot, abort flag
+  static constexpr int SMEM = MISC_OFF + 16 + 1024;          // + alignment slack
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+// Lane L ends with op over the 32 lanes of v[L] (v is clobbered): a butterfly
+// in which each level keeps half of the entries and trades the other half.
+template <bool MAX>
+__device__ __forceinline__ float xreduce32(float* v, int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool up = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float send = up ? v[i] : v[i + w];
+      const float keep = up ? v[i + w] : v[i];
+      const float got = __shfl_xor_sync(0xffffffffu, send, w);
+      v[i] = MAX ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  return v[0];
+}
+
+// Exclusive prefix sum of v over the block (256 threads); *total = the sum.
+__device__ __forceinline__ int block_exclusive_sum(int v, int* s_scan, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  __syncthreads();
+  if (lane == 31) s_scan[warp] = inc;
+  __syncthreads();
+  int before = 0, all = 0;
+  for (int w = 0; w < THREADS / 32; ++w) {
+    const int t = s_scan[w];
+    before += w < warp ? t : 0;
+    all += t;
+  }
+  *total = all;
+  return before + inc - v;
+}
+
+}  // namespace ts
+
+template <int N>
+__global__ void __launch_bounds__(ts::THREADS, 1)
+token_select_tc_kernel(const __grid_constant__ CUtensorMap tm_k, Shape s,
+                       const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ Kp,
+                       const int32_t* __restrict__ page_table,
+                       const int32_t* __restrict__ chunk_idx, int n_sel, int stride, int content,
+                       int topT, int32_t* __restrict__ tok_pos, int32_t* __restrict__ tok_cnt,
+                       unsigned* err) {
+  using namespace ts;
+  using L = Layout<N>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sQ = smem + L::Q_OFF;
+  uint8_t* sK = smem + L::K_OFF;
+  float* s_red = reinterpret_cast<float*>(smem + L::RED_OFF);   // [8][N]
+  float* s_M = reinterpret_cast<float*>(smem + L::ROW_OFF);     // [N] row maxima (log2 units)
+  float* s_iZ = s_M + N;                                        // [N] 1 / row sums
+  float* s_xl = s_iZ + N;                                       // [N] score of the last token
+  float* s_el = s_xl + N;                                       // [N] its exponential
+  uint32_t* s_key = reinterpret_cast<uint32_t*>(smem + L::TAU_OFF);  // [content] mass keys
+  int* s_hist = reinterpret_cast<int*>(smem + L::HIST_OFF);
+  int* s_scan = reinterpret_cast<int*>(smem + L::SCAN_OFF);
+  int* s_pv = reinterpret_cast<int*>(smem + L::PV_OFF);         // [17] page slot valid
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* empty = full + STAGES;
+  uint64_t* q_full = empty + STAGES;
+  uint64_t* s_done = q_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  pdl_trigger();
+  pdl_wait();
+  const int sel = blockIdx.x, bg = blockIdx.y;
+  const int b = bg / s.H_kv, g = bg % s.H_kv;
+  const int per = topT + 1;
+  int32_t* out = tok_pos + ((size_t)bg * n_sel + sel) * per;
+  const int c = chunk_idx[(size_t)bg * n_sel + sel];
+  const long long base = (long long)c * stride;
+  const bool chunk_ok = c >= 0 && base + content < (long long)s.L_ctx;
+  const int R = s.G * s.L_q;
+  const int last_o = min(content, MAXC - 1);          // last position offset in the tiles
+  const int n_t = chunk_ok ? last_o / 128 + 1 : 0;    // MMA tiles
+  const bool has_left = chunk_ok && content >= MAXC;  // the token at offset 1024
+  const int page0 = (int)(base / 64);
+  const float c2 = (float)(s.scale * 1.4426950408889634);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(q_full, 64);
+    mbar_init(s_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x <= 2 * MAX_TILES) s_pv[threadIdx.x] = 0;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (n_t > 0 && warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_k);
+      for (int t = 0; t < n_t; ++t) {
+        const int st = t % STAGES;
+        if (t >= STAGES && !mbar_wait(&empty[st], ((t / STAGES) - 1) & 1, abort_flag)) break;
+        int y[2], nload = 0;
+        for (int p = 0; p < 2; ++p) {
+          const int lp = 2 * t + p;  // page of the chunk
+          y[p] = -1;
+          if (lp * 64 <= last_o) {
+            const int slot = page_table[(size_t)b * s.n_pages + page0 + lp];
+            if (slot >= 0 && slot < s.n_slots) {
+              y[p] = (slot * s.H_kv + g) * 64;
+              s_pv[lp] = 1;
+              ++nload;
+            } else {
+              flag_error(err, ERR_BAD_INDEX);
+            }
+          }
+        }
+        if (nload == 0) {
+          mbar_arrive(&full[st]);
+          continue;
+        }
+        mbar_arrive_expect_tx(&full[st], nload * 16384);
+        uint8_t* dst = sK + st * KT_BYTES;
+        for (int p = 0; p < 2; ++p) {
+          if (y[p] < 0) continue;
+          for (int h = 0; h < 2; ++h) tma_load_2d(dst + h * 16384 + p * 8192, &tm_k, h * 64, y[p], &full[st]);
+        }
+      }
+      if (*abort_flag) {  // do not leave with copies in flight
+        for (int t = max(0, n_t - STAGES); t < n_t; ++t)
+          for (uint32_t i = 0; i < (1u << 20) && !mbar_try_wait(&full[t % STAGES], (t / STAGES) & 1); ++i) {
+          }
+      }
+    }
+  } else if (n_t > 0 && warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, N, false);
+      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK);
+      bool ok = mbar_wait(q_full, 0, abort_flag);
+      for (int t = 0; ok && t < n_t; ++t) {
+        const int st = t % STAGES;
+        if (!(ok = mbar_wait(&full[st], (t / STAGES) & 1, abort_flag))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const int h = k >> 2, kk = k & 3;
+          const uint64_t ad = sdesc_sw128(k_base + st * KT_BYTES + h * 16384 + kk * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(q_base + h * N * 128 + kk * 32, 16, 1024);
+          mma_f16_ss(tmem + t * N, ad, bd, idesc, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&empty[st]);
+      }
+      if (ok) mma_commit(s_done);
+      if (*abort_flag)  // give issued MMAs time to finish before TMEM is freed
+        for (uint32_t k = 0; k < (1u << 16); ++k) __nanosleep(1000);
+    }
+  } else if (n_t > 0 && (warp == 2 || warp == 3)) {
+    // ------------------------------------------------------------ Q gather
+    constexpr int per_row = 16;  // 16-byte chunks of a 128-element row
+    constexpr int IN_FLIGHT = 8;
+    const int gt = threadIdx.x - 64;
+    constexpr int total = N * per_row;
+    for (int e0 = 0; e0 < total; e0 += 64 * IN_FLIGHT) {
+      uint4 v[IN_FLIGHT];
+#pragma unroll
+      for (int u = 0; u < IN_FLIGHT; ++u) {
+        const int e = e0 + u * 64 + gt;
+        const int n = e / per_row, rem = e % per_row;
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (e < total && n < R) {
+          const int h = g * s.G + n / s.L_q, i = n % s.L_q;
+          v[u] = __ldg(reinterpret_cast<const uint4*>(Q + (((size_t)b * s.H + h) * s.L_q + i) * D +
+                                                      rem * 8));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < IN_FLIGHT; ++u) {
+        const int e = e0 + u * 64 + gt;
+        if (e >= total) continue;
+        const int n = e / per_row, rem = e % per_row;
+        const int h_half = rem >> 3, ch = rem & 7;
+        *reinterpret_cast<uint4*>(sQ + h_half * N * 128 + n * 128 + ((ch ^ (n & 7)) << 4)) = v[u];
+      }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(q_full);
+  } else if (warp == 4 || warp == 5) {
+    // ------------------------------------------------------------ last token
+    const int r = threadIdx.x - 128;
+    float x = -INFINITY;
+    if (has_left) {
+      const long long pos = base + MAXC;
+      const int slot = page_table[(size_t)b * s.n_pages + pos / 64];
+      const bool slot_ok = slot >= 0 && slot < s.n_slots;
+      if (r == 0) {
+        s_pv[2 * MAX_TILES] = slot_ok ? 1 : 0;
+        if (!slot_ok) flag_error(err, ERR_BAD_INDEX);
+      }
+      if (slot_ok && r < R && r < N) {
+        const int h = g * s.G + r / s.L_q, i = r % s.L_q;
+        const __nv_bfloat16* qr = Q + (((size_t)b * s.H + h) * s.L_q + i) * D;
+        const __nv_bfloat16* kr = Kp + (((size_t)slot * s.H_kv + g) * 64 + pos % 64) * D;
+        float acc = 0.0f;
+        for (int x0 = 0; x0 < D; x0 += 8) {
+          float qv[8], kv[8];
+          Vec16<__nv_bfloat16>::load(qr + x0, qv);
+          Vec16<__nv_bfloat16>::load(kr + x0, kv);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc = fmaf(qv[k], kv[k], acc);
+        }
+        x = acc * c2;
+      }
+    }
+    if (r < N) s_xl[r] = x;
+  }
+  // ---------------------------------------------------------------- epilogue
+  // every warp: TMEM lanes of its quadrant, four of the tiles
+  if (n_t > 0 && threadIdx.x == 128) {
+    if (!mbar_wait(s_done, 0, abort_flag)) *abort_flag = 1;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const bool run = n_t > 0 && !*abort_flag;
+  const int quad = warp & 3;
+  const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+  auto key_ok = [&](int o) {  // offset o from the chunk start holds a usable content token
+    return o >= 1 && o <= last_o && s_pv[o >> 6] != 0;
+  };
+  if (run) {
+    // pass 1: row maxima
+    float m[N];
+#pragma unroll
+    for (int r = 0; r < N; ++r) m[r] = -INFINITY;
+    for (int j = warp >> 2; j < n_t; j += 2) {
+      const int o = j * 128 + quad * 32 + lane;
+      const bool kv = key_ok(o);
+      uint32_t v[N];
+      tmem_ld<N>(tmem + lane_base + j * N, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int r = 0; r < N; ++r)
+        m[r] = fmaxf(m[r], (kv && r < R) ? __uint_as_float(v[r]) * c2 : -INFINITY);
+    }
+#pragma unroll
+    for (int r0 = 0; r0 < N; r0 += 32) s_red[warp * N + r0 + lane] = xreduce32<true>(m + r0, lane);
+  }
+  __syncthreads();
+  if (run && threadIdx.x < N) {
+    const int r = threadIdx.x;
+    float mx = s_xl[r];
+    for (int w = 0; w < 8; ++w) mx = fmaxf(mx, s_red[w * N + r]);
+    s_M[r] = mx;
+  }
+  __syncthreads();
+  if (run) {
+    // pass 2: exponentials (written back over S^T) and row sums
+    float z[N];
+#pragma unroll
+    for (int r = 0; r < N; ++r) z[r] = 0.0f;
+    for (int j = warp >> 2; j < n_t; j += 2) {
+      const int o = j * 128 + quad * 32 + lane;
+      const bool kv = key_ok(o);
+      uint32_t v[N];
+      tmem_ld<N>(tmem + lane_base + j * N, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int r = 0; r < N; ++r) {
+        const float mr = s_M[r];
+        const float e = (kv && r < R && mr != -INFINITY)
+                            ? ex2_approx(__uint_as_float(v[r]) * c2 - mr) : 0.0f;
+        z[r] += e;
+        v[r] = __float_as_uint(e);
+      }
+      tmem_st<N>(tmem + lane_base + j * N, v);
+    }
+    tmem_st_wait();
+#pragma unroll
+    for (int r0 = 0; r0 < N; r0 += 32) s_red[warp * N + r0 + lane] = xreduce32<false>(z + r0, lane);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (run && threadIdx.x < N) {
+    const int r = threadIdx.x;
+    const float mr = s_M[r];
+    const float el = (s_xl[r] != -INFINITY && mr != -INFINITY) ? ex2_approx(s_xl[r] - mr) : 0.0f;
+    float zt = el;
+    for (int w = 0; w < 8; ++w) zt += s_red[w * N + r];
+    s_el[r] = el;
+    s_iZ[r] = zt > 0.0f ? 1.0f / zt : 0.0f;
+  }
+  __syncthreads();
+  // pass 3: masses, as order-preserving keys (0 = unusable token)
+  if (run) {
+    for (int j = warp >> 2; j < n_t; j += 2) {
+      const int o = j * 128 + quad * 32 + lane;
+      uint32_t v[N];
+      tmem_ld<N>(tmem + lane_base + j * N, v);
+      tmem_ld_wait();
+      float tau = 0.0f;
+#pragma unroll
+      for (int r = 0; r < N; ++r) tau = fmaf(__uint_as_float(v[r]), s_iZ[r], tau);
+      if (o >= 1 && o <= last_o) s_key[o - 1] = key_ok(o) ? __float_as_uint(tau) + 1u : 0u;
+    }
+    if (has_left && threadIdx.x == 0) {
+      float tau = 0.0f;
+      for (int r = 0; r < N; ++r) tau = fmaf(s_el[r], s_iZ[r], tau);
+      s_key[MAXC - 1] = s_pv[2 * MAX_TILES] ? __float_as_uint(tau) + 1u : 0u;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) flag_error(err, ERR_TIMEOUT);
+  if (!chunk_ok || !run) {
+    if (threadIdx.x == 0 && !chunk_ok) flag_error(err, ERR_BAD_INDEX);
+    for (int e = threadIdx.x; e < per; e += blockDim.x) out[e] = -1;
+    if (threadIdx.x == 0 && sel == 0) tok_cnt[bg] = n_sel * per;
+  } else {
+    // top-T by (key desc, position asc): radix select of the T-th largest key
+    const int n = content;
+    const int T = min(topT, n);
+    uint32_t prefix = 0u, mask = 0u;
+    int k_rem = T;
+    for (int pass = 0; pass < 4 && T > 0; ++pass) {
+      const int shift = 24 - 8 * pass;
+      s_hist[threadIdx.x] = 0;  // 256 bins, 256 threads
+      __syncthreads();
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const uint32_t v = s_key[i];
+        if ((v & mask) == prefix) atomicAdd(&s_hist[(v >> shift) & 255u], 1);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        int cnt[8], tot = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          cnt[q] = s_hist[lane * 8 + q];
+          tot += cnt[q];
+        }
+        int above = tot;  // elements in this lane's bins and every higher lane's
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int x = __shfl_down_sync(0xffffffffu, above, o);
+          if (lane + o < 32) above += x;
+        }
+        int run_cnt = above - tot;  // elements in higher lanes' bins
+        for (int q = 7; q >= 0; --q) {
+          if (run_cnt < k_rem && run_cnt + cnt[q] >= k_rem) {
+            s_scan[32] = lane * 8 + q;
+            s_scan[33] = run_cnt;
+          }
+          run_cnt += cnt[q];
+        }
+      }
+      __syncthreads();
+      prefix |= static_cast<uint32_t>(s_scan[32]) << shift;
+      mask |= 255u << shift;
+      k_rem -= s_scan[33];
+      __syncthreads();
+    }
+    // keep: above the cut, or at it among the first k_rem in position order
+    constexpr int PER_T = MAXC / THREADS;  // positions per thread, contiguous
+    const int i0 = threadIdx.x * PER_T;
+    int n_eq = 0;
+#pragma unroll
+    for (int q = 0; q < PER_T; ++q) {
+      const int i = i0 + q;
+      n_eq += (T > 0 && i < n && s_key[i] == prefix) ? 1 : 0;
+    }
+    int tot_eq = 0;
+    int eq_before = block_exclusive_sum(n_eq, s_scan, &tot_eq);
+    bool keep[PER_T];
+    int n_keep = 0;
+#pragma unroll
+    for (int q = 0; q < PER_T; ++q) {
+      const int i = i0 + q;
+      bool k = false;
+      if (T > 0 && i < n) {
+        const uint32_t v = s_key[i];
+        if (v > prefix) {
+          k = true;
+        } else if (v == prefix) {
+          k = eq_before < k_rem;
+          ++eq_before;
+        }
+      }
+      keep[q] = k;
+      n_keep += k ? 1 : 0;
+    }
+    int total = 0;
+    const int p0 = block_exclusive_sum(n_keep, s_scan, &total);
+    int p = p0;
+#pragma unroll
+    for (int q = 0; q < PER_T; ++q)
+      if (keep[q]) out[1 + p++] = (int)(base + 1 + i0 + q);
+    if (threadIdx.x == 0) {
+      out[0] = (int)base;
+      if (sel == 0) tok_cnt[bg] = n_sel * per;
+    }
+    for (int e = 1 + total + threadIdx.x; e < per; e += blockDim.x) out[e] = -1;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+bool tc_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows);
+
+// Whether the tensor-core kernel takes this call: bf16, head dim 128, 64-token
+// pages, chunks starting on a page boundary, at most 64 query rows per group.
+bool token_select_tc_supported(const Shape& s, int chunk_stride, int chunk_content) {
+  return s.dtype == 0 && s.d == 128 && s.page == 64 && chunk_stride % 64 == 0 &&
+         chunk_content <= ts::MAXC && s.G * s.L_q <= 64 &&
+         (uint64_t)s.n_slots * s.H_kv * 64 < (1ull << 31);
+}
+
+cudaError_t launch_token_select_tc(const Shape& s, const void* Q, const void* Kp,
+                                   const int32_t* page_table, const int32_t* chunk_idx, int n_sel,
+                                   int chunk_stride, int chunk_content, int topT, int32_t* tok_pos,
+                                   int32_t* tok_cnt, unsigned* err, cudaStream_t st) {
+  CUtensorMap mk;
+  if (!tc_map_2d(&mk, Kp, ts::D, (uint64_t)s.n_slots * s.H_kv * 64, 64)) return cudaErrorInvalidValue;
+  dim3 grid(n_sel, s.batch * s.H_kv);
+  auto* q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  auto* k = reinterpret_cast<const __nv_bfloat16*>(Kp);
+  cudaError_t e;
+  if (s.G * s.L_q <= 32) {
+    constexpr int smem = ts::Layout<32>::SMEM;
+    if ((e = cudaFuncSetAttribute(token_select_tc_kernel<32>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+      return e;
+    DL_LAUNCH(token_select_tc_kernel<32>, grid, ts::THREADS, smem, st, mk, s, q, k, page_table,
+              chunk_idx, n_sel, chunk_stride, chunk_content, topT, tok_pos, tok_cnt, err);
+  } else {
+    constexpr int smem = ts::Layout<64>::SMEM;
+    if ((e = cudaFuncSetAttribute(token_select_tc_kernel<64>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+      return e;
+    DL_LAUNCH(token_select_tc_kernel<64>, grid, ts::THREADS, smem, st, mk, s, q, k, page_table,
+              chunk_idx, n_sel, chunk_stride, chunk_content, topT, tok_pos, tok_cnt, err);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace dl

@@ -3,11 +3,19 @@
     python -m long_context_diffusion_b200.profile_case --case attn_sparse --reps 3
     python -m long_context_diffusion_b200.profile_case --case block_select --reps 3
     python -m long_context_diffusion_b200.profile_case --case sinks --reps 3
+    python -m long_context_diffusion_b200.profile_case --case chunk_step --reps 20
 
 Builds one sparse layer of the 32K workload (batch 4, 32 KV heads, 32K context:
 about 2.1 GB of K/V pages on the device), runs the steps before the profiled
 call once, then calls it `reps` times (the first is a warm-up) and prints its
 mean time from CUDA events.  Meant to sit under `ncu -k ... -s 1 -c 1`.
+
+`chunk_step` instead times the chunked-prefix step (32 chunks of a BOS and
+1024 content tokens in permuted 64-token pages, 64 decode queries, top-8
+chunks, top-256 tokens per chunk): chunk scores, chunk selection, token
+selection and the gathered attention, with the chunk keys built beforehand
+(they belong to the cache refresh), and reports the step's algorithmic bytes
+per second.
 """
 from __future__ import annotations
 
@@ -22,12 +30,14 @@ from . import _abi as A
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["attn_sparse", "attn_dense", "block_select", "pool", "sinks"],
+    ap.add_argument("--case", choices=["attn_sparse", "attn_dense", "block_select", "pool", "sinks", "chunk_step"],
                     required=True)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--batch", type=int, default=4)
     args = ap.parse_args()
     dev = torch.device("cuda", 0)
+    if args.case == "chunk_step":
+        return chunk_step(args.reps, dev)
     wl = synth.workload("llada32k_step", n_layers=3, batch=args.batch)
     layer = wl.first_sparse_layer
     pt = synth.page_permutation(wl).to(dev)
@@ -86,6 +96,62 @@ def main():
         raise RuntimeError(f"device status {st}")
     print(json.dumps({"case": args.case, "batch": wl.batch, "us_per_call": times,
                       "mean_us_after_first": sum(times[1:]) / max(1, len(times) - 1)}))
+
+
+def chunk_step(reps: int, dev):
+    from . import pipeline
+    wl = synth.workload("chunked32k")
+    inp = synth.make_step_inputs(wl, device=dev)
+    desc = A.make_desc(wl.batch, wl.H, wl.H_kv, wl.d, wl.L_ctx, wl.L_q, wl.B, wl.n_pages,
+                       wl.n_slots, A.DL_BF16)
+    ws = torch.empty(A.dl_workspace_size(desc), dtype=torch.uint8, device=dev)
+    Kbar = torch.empty((wl.batch, wl.H_kv, wl.n_chunks, wl.d), dtype=torch.float32, device=dev)
+    A.dl_pool_keys(desc, inp.k_pool, inp.page_table, wl.n_chunks, wl.chunk_stride, 1,
+                   wl.chunk_content, Kbar)
+
+    def fn():
+        return pipeline.chunked_step(desc, inp.q_dec, inp.k_pool, inp.v_pool, inp.page_table,
+                                     inp.k_dec, inp.v_dec, n_chunks=wl.n_chunks,
+                                     stride=wl.chunk_stride, content=wl.chunk_content,
+                                     topK_chunks=wl.topK_chunks, topT=wl.topT_tokens,
+                                     Kbar=Kbar, ws=ws)
+    out = fn()
+    torch.cuda.synchronize()
+    # algorithmic bytes per step: pooled chunk keys, Q, the content K rows of
+    # the selected chunks (token scores), K and V of the gathered tokens and of
+    # the decode block, O and LSE written
+    esz = 2
+    kc = int(out.chunk_cnt.sum().item())
+    n_tok = int(out.tok_cnt.sum().item())
+    nbytes = (Kbar.numel() * 4 + inp.q_dec.numel() * esz + kc * wl.chunk_content * wl.d * esz +
+              n_tok * wl.d * esz * 2 + inp.k_dec.numel() * esz * 2 + out.O.numel() * esz +
+              out.lse.numel() * 4)
+    # one graph replay per timed step, so that host launch overhead is not timed
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fn()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # larger than L2
+    times = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3)
+    st = A.dl_get_status()
+    if st != A.DL_OK:
+        raise RuntimeError(f"device status {st}")
+    mean = sum(times[1:]) / max(1, len(times) - 1)
+    print(json.dumps({"case": "chunk_step", "workload": "chunked32k", "us_per_call": times,
+                      "mean_us_after_first": mean, "bytes_per_step": nbytes,
+                      "achieved_GBps": nbytes / (mean * 1e-6) / 1e9}))
 
 
 if __name__ == "__main__":

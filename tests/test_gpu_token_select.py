@@ -1,0 +1,87 @@
+"""GPU parity of intra-chunk token selection (the chunked-prefix path) called
+directly through the C ABI: chunks of 1024 content tokens (eight key tiles
+and the token past them), ragged chunks, one and two query heads per KV
+group, 16 to 64 query rows, T from 0 to the whole chunk, and a chunk stride
+off the page grid (the CUDA-core kernel).  Every page-aligned case also runs
+through the CUDA-core kernel.  Kept tokens must equal the oracle's wherever
+its cut has a margin above the fp32 error of the masses, and be within that
+error of the cut otherwise."""
+
+import numpy as np
+import pytest
+import torch
+
+import long_context_diffusion_b200 as dl
+import oracle
+import synth
+from oracle import steps as S
+from tests.helpers import cut_margin, np_
+
+pytestmark = pytest.mark.gpu
+
+SEED = 20261202
+
+
+@pytest.mark.parametrize("content,stride,H,H_kv,L_q,topT,n_sel", [
+    (1024, 1088, 4, 4, 64, 256, 2),   # the benchmark's chunk shape: 64 rows
+    (1000, 1024, 4, 2, 16, 100, 2),   # G = 2, 32 rows, ragged last tile
+    (200, 256, 2, 2, 20, 0, 1),       # T = 0: the BOS only
+    (200, 256, 2, 2, 20, 200, 3),     # T = the whole chunk
+    (64, 128, 3, 3, 48, 1, 2),        # one tile, 48 rows
+    (300, 301, 2, 2, 32, 37, 2),      # stride off the page grid
+])
+@pytest.mark.parametrize("simt", [False, True])
+def test_token_select_matches_oracle(content, stride, H, H_kv, L_q, topT, n_sel, simt,
+                                     cuda_device, monkeypatch):
+    if simt:
+        monkeypatch.setenv("DL_TOKEN_SIMT", "1")
+    batch, d, page, n_chunks = 2, 128, 64, 3
+    G = H // H_kv
+    L_ctx = n_chunks * stride
+    n_pages = -(-L_ctx // page)
+    n_slots = batch * n_pages
+    sid = 12000 + content + 7 * L_q + topT
+    q = (synth.normals(SEED, sid, 0, batch * H * L_q * d).reshape(batch, H, L_q, d)).to(
+        torch.bfloat16)
+    kp = (synth.normals(SEED, sid + 1, 0, n_slots * H_kv * page * d).reshape(
+        n_slots, H_kv, page, d)).to(torch.bfloat16)
+    perm = torch.argsort(synth.uniforms(SEED, sid + 2, 0, n_slots)).to(torch.int32)
+    page_table = perm.reshape(batch, n_pages)
+    sel_keys = synth.uniforms(SEED, sid + 3, 0, batch * H_kv * n_chunks).reshape(
+        batch * H_kv, n_chunks)
+    chunk_idx = torch.sort(torch.argsort(sel_keys, dim=1)[:, :n_sel], dim=1).values.to(
+        torch.int32).reshape(batch, H_kv, n_sel)
+    desc = dl.make_desc(batch=batch, H=H, H_kv=H_kv, d=d, L_ctx=L_ctx, L_q=L_q, page=page,
+                        n_pages=n_pages, n_slots=n_slots, dtype=dl.DL_BF16)
+    ws = torch.empty(max(dl.dl_workspace_size(desc), 256), dtype=torch.uint8, device=cuda_device)
+    per = topT + 1
+    tok_pos = torch.full((batch, H_kv, n_sel * per), -7, dtype=torch.int32, device=cuda_device)
+    tok_cnt = torch.full((batch, H_kv), -7, dtype=torch.int32, device=cuda_device)
+    dl.dl_token_select(desc, q.to(cuda_device), kp.to(cuda_device), page_table.to(cuda_device),
+                       chunk_idx.to(cuda_device), stride, content, topT, tok_pos, tok_cnt, ws)
+    torch.cuda.synchronize()
+    assert dl.dl_get_status() == dl.DL_OK
+    got, cnt = np_(tok_pos), np_(tok_cnt)
+    assert (cnt == n_sel * per).all()
+    scale = oracle.scale_for(d)
+    Q, K = S.f64(q), S.f64(kp)
+    pt = np.asarray(page_table, dtype=np.int64)
+    for b in range(batch):
+        for g in range(H_kv):
+            rows = Q[b, g * G:(g + 1) * G].reshape(-1, d)
+            for j in range(n_sel):
+                c = int(chunk_idx[b, g, j])
+                base = c * stride
+                keys = S.gather_context(K, pt[b], g, base + 1 + np.arange(content), page)
+                off, tau = S.token_select(rows, keys, topT, scale)
+                out = got[b, g, j * per:(j + 1) * per]
+                assert out[0] == base, (b, g, j)
+                kept = out[1:]
+                assert (kept[len(off):] == -1).all() if topT else True
+                mine = kept[: len(off)] - base - 1
+                assert np.all(np.diff(mine) > 0), (b, g, j)
+                tol = 1e-5 * tau.max()
+                if cut_margin(tau, off) > tol:
+                    assert mine.tolist() == off.tolist(), (b, g, j)
+                else:
+                    assert (tau[mine] >= np.sort(tau)[-topT] - tol).all(), (b, g, j)
