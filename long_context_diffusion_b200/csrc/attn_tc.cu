@@ -31,6 +31,15 @@
 //                        max grows by more than 2^8) and sum, writes P (bf16)
 //                        to shared memory in the MMA's K-major swizzled
 //                        layout, and at the end writes its partial (O, m, l).
+// Gathered tokens (the chunked prefix: arbitrary cached positions): a tile is
+// 64 consecutive entries of the (b, g)'s position list, and the whole
+// producer warp copies its rows with 16-byte cp.async into the same swizzled
+// layout (each lane resolves two rows' positions through the page table);
+// a tile is released to the MMAs (wait for the copies, proxy fence, arrive)
+// once ST - 1 newer gathered tiles are in flight, before the producer waits
+// for its ring slot again, and before the next segment's Q is loaded.  Rows
+// past a tile's valid keys are zero-filled by the copies.  Decode tiles keep
+// their TMA path.
 // The G*L_q query rows of a KV group are padded to M-tiles of 128 rows (the
 // path is HBM-bound: padding costs tensor time, not bytes).  Partials of the
 // splits of one (b, g) are merged by the combine kernel of attn_simt.cu.
@@ -38,9 +47,11 @@
 // Every wait is bounded: a role that gives up raises the shared abort flag
 // and the device error word (ERR_TIMEOUT) and leaves its loop; the CTA then
 // frees its TMEM and returns.
+#include <cstdlib>
 #include <mutex>
 
 #include "sm100.cuh"
+#include "score_common.cuh"
 #include "tc_common.cuh"
 #include "launch.cuh"
 
@@ -191,7 +202,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int n_ctx = ctx_tile_count(a, bg);
     const int lo = seg_lo[k];
     for (int t = threadIdx.x; t < seg[k].w; t += blockDim.x) {
-      const int2 ti = tc_tile_info(a, bg, lo + t, n_ctx);
+      int2 ti;
+      if (a.mode == kGather && lo + t < n_ctx) {  // rows are resolved by the producer
+        const int c = min(max(a.cnt[bg], 0), a.max_idx);
+        ti = make_int2(0, min(64, c - (lo + t) * 64));
+      } else {
+        ti = tc_tile_info(a, bg, lo + t, n_ctx);
+      }
       t_info[seg[k].z + t] = make_int2(ti.x, ti.y | (k << 16));
     }
   }
@@ -212,7 +229,120 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint8_t* ring = is_k ? sK : sV;
     const CUtensorMap* map = is_k ? &tm_k : &tm_v;
     const CUtensorMap* map_dec = is_k ? &tm_kd : &tm_vd;
-    if (lane == 0 && nt > 0) {
+    if (a.mode == kGather && nt > 0) {
+      // ---- gathered rows: the whole warp copies, tiles released in order
+      if (lane == 0) prefetch_tmap(map_dec);
+      const __nv_bfloat16* pool =
+          reinterpret_cast<const __nv_bfloat16*>(is_k ? a.Kp : a.Vp);
+      int pend[ST] = {};  // gathered tiles whose copies may be in flight, oldest first
+      int n_pend = 0;
+      // the oldest pending tile: its copies have landed (all but the newest
+      // n_pend - 1 groups), then the fence that orders them before the MMAs
+      auto release_oldest = [&]() {
+        switch (n_pend - 1) {
+          case 0: cp_async_wait<0>(); break;
+          case 1: cp_async_wait<1>(); break;
+          case 2: cp_async_wait<2>(); break;
+          case 3: cp_async_wait<3>(); break;
+          case 4: cp_async_wait<4>(); break;
+          case 5: cp_async_wait<5>(); break;
+          default: cp_async_wait<0>(); break;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[pend[0] % ST]);
+        for (int q = 1; q < n_pend; ++q) pend[q - 1] = pend[q];
+        --n_pend;
+      };
+      auto load_q = [&](int k) -> bool {
+        const int qb = QB == 2 ? (k & 1) : 0;
+        bool w = true;
+        if (k >= QB) {  // the buffer's previous segment must be done with it
+          while (n_pend > 0) release_oldest();
+          const int prev = k - QB;
+          if (lane == 0)
+            w = mbar_wait(&q_free[qb], (QB == 2 ? (prev >> 1) : prev) & 1, abort_flag);
+          w = __shfl_sync(0xffffffffu, w, 0);
+        }
+        if (w && lane == 0) {
+          const int bg = seg[k].x;
+          const int b = bg / s.H_kv, g = bg % s.H_kv;
+          const int q_row0 = (b * s.H + g * s.G) * s.L_q;
+          mbar_arrive_expect_tx(&q_full[qb], C::Q_TILE);
+          for (int m = 0; m < NM; ++m)
+            for (int h = 0; h < C::HALVES; ++h)
+              for (int c = 0; c < REP; ++c)
+                tma_load_2d(sQ + qb * C::Q_TILE + (m * C::HALVES + h) * 16384 + c * C::RB * 128,
+                            &tm_q, h * 64, q_row0 + m * 128, &q_full[qb]);
+        }
+        return w;
+      };
+      if (is_k && lane == 0) prefetch_tmap(&tm_q);
+      int next_q = 0;
+      bool ok = true;
+      for (int i = 0; ok && i < nt; ++i) {
+        const int k = tile_seg(i);
+        while (is_k && ok && next_q < nseg && next_q <= k) {
+          ok = load_q(next_q);
+          ++next_q;
+        }
+        if (!ok) break;
+        const int st = i % ST;
+        // tile i - ST (same ring slot; decode tiles hold slots too) must be
+        // released before waiting for its slot
+        while (n_pend > 0 && pend[0] <= i - ST) release_oldest();
+        if (i >= ST) {
+          bool w = true;
+          if (lane == 0) w = mbar_wait(&empty[st], ((i / ST) - 1) & 1, abort_flag);
+          if (!(ok = __shfl_sync(0xffffffffu, w, 0))) break;
+        }
+        uint8_t* dst = ring + st * C::KT_BYTES;
+        const int valid = tile_valid(i);
+        if (valid > 0 && !tile_dec(i)) {
+          const int bg = seg[k].x;
+          const int b = bg / s.H_kv, g = bg % s.H_kv;
+          const int tile = seg_lo[k] + (i - seg[k].z);  // tile of the (b, g)'s list
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            const int r = lane + 32 * rr;
+            const __nv_bfloat16* src = pool;
+            bool okr = false;
+            if (r < valid) {
+              const int pos = a.idx[(size_t)bg * a.max_idx + tile * 64 + r];
+              const int slot = pos >= 0 && pos < s.L_ctx
+                                   ? a.page_table[(size_t)b * s.n_pages + pos / 64] : -1;
+              if (slot >= 0 && slot < s.n_slots) {
+                src = pool + (((size_t)slot * s.H_kv + g) * 64 + pos % 64) * D;
+                okr = true;
+              } else {
+                flag_error(a.err, ERR_BAD_INDEX);  // the key is left zero
+              }
+            }
+#pragma unroll
+            for (int c = 0; c < C::HALVES * 8; ++c)
+              cp_async16(dst + (c >> 3) * 8192 + r * 128 + (((c & 7) ^ (r & 7)) << 4),
+                         src + c * 8, okr);
+          }
+          cp_async_commit();
+          pend[n_pend++] = i;
+          if (n_pend >= ST) release_oldest();
+        } else if (valid > 0) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[st], C::KT_BYTES);
+            for (int h = 0; h < C::HALVES; ++h)
+              tma_load_3d(dst + h * 8192, map_dec, h * 64, t_info[i].x, seg[k].x, &full[st]);
+          }
+        } else if (lane == 0) {
+          mbar_arrive(&full[st]);
+        }
+      }
+      while (n_pend > 0) release_oldest();  // every copy has landed before leaving
+      if (*abort_flag && lane == 0) {  // nor with a decode tile's TMA in flight
+        for (int i = max(0, nt - ST); i < nt; ++i)
+          for (uint32_t t = 0; t < (1u << 20) && !mbar_try_wait(&full[i % ST], (i / ST) & 1); ++t) {
+          }
+      }
+    } else if (lane == 0 && nt > 0) {
       prefetch_tmap(map);
       prefetch_tmap(map_dec);
       auto load_q = [&](int k) -> bool {
@@ -454,9 +584,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
         }
       }
-      if (m == 0 && valid < 64) {
+      if (m == 0 && valid < 64 && (a.mode != kGather || tile_dec(i))) {
         // rows past the valid keys may hold anything (even NaN): zero V there
-        // once it has landed
+        // once it has landed (gathered tiles are zero-filled by their copies)
         ok = __all_sync(0xffffffffu, mbar_wait(&full_v[i % ST], (i / ST) & 1, abort_flag));
         if (!ok) break;
         uint8_t* sVt = sV + (i % ST) * C::KT_BYTES;
@@ -631,7 +761,7 @@ static cudaError_t run_tc(const AttnArgs& a, int max_tiles, cudaStream_t st) {
 // at most two M-tiles of query rows, pool addressable by 32-bit TMA rows).
 bool attn_tc_supported(const AttnArgs& a) {
   const Shape& s = a.s;
-  return s.dtype == 0 && a.mode != kGather && s.G * s.L_q <= 256 &&
+  return s.dtype == 0 && (a.mode != kGather || !getenv("DL_GATHER_SIMT")) && s.G * s.L_q <= 256 &&
          (uint64_t)s.n_slots * s.H_kv * 64 < (1ull << 31) &&
          (uint64_t)s.batch * s.H * s.L_q < (1ull << 31);
 }
