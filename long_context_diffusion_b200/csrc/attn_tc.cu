@@ -88,8 +88,10 @@ struct TcCfg {
   static constexpr int SEG_OFF = TILE_OFF + kTcMaxTiles * 8;       // int4 [kMaxSegs]
   static constexpr int SEGLO_OFF = SEG_OFF + kMaxSegs * 16;        // int [kMaxSegs]
   static constexpr int MARK_OFF = SEGLO_OFF + kMaxSegs * 4;        // int2 [kMaxSegs]
+  static constexpr int ROWS_OFF = MARK_OFF + kMaxSegs * 8;         // int [ROWS_CAP]
+  static constexpr int ROWS_CAP = 64 * 64;  // gathered rows resolved up front (64 tiles)
   static_assert(BAR_OFF % 16 == 0 && TILE_OFF % 16 == 0 && SEG_OFF % 16 == 0, "alignment");
-  static constexpr int SMEM = MARK_OFF + kMaxSegs * 8 + 1024;      // + alignment slack
+  static constexpr int SMEM = ROWS_OFF + ROWS_CAP * 4 + 1024;      // + alignment slack
   static constexpr int THREADS = 128 + SOFTMAX_THREADS;
   static constexpr uint32_t TMEM_NEED = OB * NM * D + 2 * NM * 64;
   static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
@@ -135,6 +137,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   int4* seg = reinterpret_cast<int4*>(smem + C::SEG_OFF);      // (bg, slot, first, n)
   int* seg_lo = reinterpret_cast<int*>(smem + C::SEGLO_OFF);   // first tile index in (b, g)
   int2* mark = reinterpret_cast<int2*>(smem + C::MARK_OFF);    // (bg, slot) of empty runs
+  int* s_rows = reinterpret_cast<int*>(smem + C::ROWS_OFF);    // pool row of each gathered key
   int* s_nmark = s_nt + 2;
 
   const Shape& s = a.s;
@@ -219,6 +222,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   auto tile_seg = [&](int i) { return t_info[i].y >> 16; };
   auto tile_valid = [&](int i) { return t_info[i].y & 0x7F; };
   auto tile_dec = [&](int i) { return (t_info[i].y >> 15) & 1; };
+  // gathered keys: each row's pool row (through its position and the page
+  // table), resolved by every thread at once so that the producers only copy
+  const bool rows_staged = a.mode == kGather && nt * 64 <= C::ROWS_CAP;
+  if (rows_staged) {
+    for (int e = threadIdx.x; e < nt * 64; e += blockDim.x) {
+      const int i = e >> 6, r = e & 63;
+      int row = -1;
+      if (!tile_dec(i) && r < tile_valid(i)) {
+        const int k = tile_seg(i);
+        const int bg = seg[k].x;
+        const int b = bg / s.H_kv, g = bg % s.H_kv;
+        const int pos = a.idx[(size_t)bg * a.max_idx + (seg_lo[k] + i - seg[k].z) * 64 + r];
+        const int slot =
+            pos >= 0 && pos < s.L_ctx ? a.page_table[(size_t)b * s.n_pages + pos / 64] : -1;
+        if (slot >= 0 && slot < s.n_slots)
+          row = (slot * s.H_kv + g) * 64 + pos % 64;
+        else
+          flag_error(a.err, ERR_BAD_INDEX);  // the key is left zero
+      }
+      s_rows[e] = row;
+    }
+    __syncthreads();
+  }
 
   if (warp == 0 || warp == 2) {
     // ------------------------------------------------------------ producers
@@ -307,7 +333,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int r = lane + 32 * rr;
             const __nv_bfloat16* src = pool;
             bool okr = false;
-            if (r < valid) {
+            if (rows_staged) {
+              const int row = s_rows[i * 64 + r];
+              okr = row >= 0;
+              if (okr) src = pool + (size_t)row * D;
+            } else if (r < valid) {
               const int pos = a.idx[(size_t)bg * a.max_idx + tile * 64 + r];
               const int slot = pos >= 0 && pos < s.L_ctx
                                    ? a.page_table[(size_t)b * s.n_pages + pos / 64] : -1;

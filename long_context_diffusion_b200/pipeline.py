@@ -119,11 +119,12 @@ def chunked_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec,
         Kbar = _empty((B, H_kv, n_chunks, d), torch.float32, dev)
         A.dl_pool_keys(desc, k_pool, page_table, n_chunks, stride, 1, content, Kbar, stream)
     score = _empty((B, H_kv, n_chunks), torch.float64, dev)
-    A.dl_block_scores(desc, q_dec, None, None, Kbar, n_chunks, score, ws, stream)
     kc = min(topK_chunks, n_chunks)
     chunk_idx = _empty((B, H_kv, kc), torch.int32, dev)
     chunk_cnt = _empty((B, H_kv), torch.int32, dev)
-    A.dl_select(score, stride, kc, None, chunk_idx, chunk_cnt, stream)
+    # chunk scores from every decode row, then the top chunks: one call
+    A.dl_block_select(desc, q_dec, None, None, Kbar, n_chunks, stride, kc, None, score, chunk_idx,
+                      chunk_cnt, ws, stream)
     tok_pos = _empty((B, H_kv, kc * (topT + 1)), torch.int32, dev)
     tok_cnt = _empty((B, H_kv), torch.int32, dev)
     A.dl_token_select(desc, q_dec, k_pool, page_table, chunk_idx, stride, content, topT, tok_pos,

@@ -109,6 +109,9 @@ def test_select_all_paths(n_units, topK, cuda_device):
     (200, 4, 4, 128, 32, [32, 5], 300, "fp32"),       # fp32 queries, topK beyond the candidates
     (513, 4, 4, 128, 32, [20, 9], 64, "bf16"),        # separate kernels: more than 512 keys
     (100, 8, 2, 128, 32, [20, 32], 10, "bf16"),       # separate kernels: 4 x 32 rows
+    (32, 8, 8, 128, 64, [64, 13], 8, "bf16"),         # separate kernels: few units, 64 rows
+    (128, 8, 4, 64, 40, [40, 1], 20, "fp32"),         # 128 units, 80 rows, d 64, fp32
+    (7, 4, 2, 128, 48, [48, 0], 3, "bf16"),           # 96 rows over 7 units, a sequence with none
 ])
 @pytest.mark.parametrize("tight", [False, True])
 def test_block_select_matches_oracle(n_units, H, H_kv, d, L_q, cnts, topK, dtype, tight,
