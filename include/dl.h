@@ -217,7 +217,9 @@ dl_status dl_token_select(const dl_attn_desc* desc, const void* Q_dec, const voi
  * block.  [P1 abstract: a kernel that parallelises decoding over the
  * non-contiguously cached chunk KV]
  * As dl_sparse_attn with S = logical positions tok_pos[b][g][0..tok_cnt)
- * (each < n_pages*page) plus the L_q decode keys.
+ * (each < n_pages*page) plus the L_q decode keys.  A position out of range,
+ * or one whose page-table slot is, is reported through dl_get_status
+ * (DL_ERR_BAD_INDEX) and that (b, g)'s output is then unspecified.
  *   tok_pos int32 [batch][H_kv][max_tok], tok_cnt int32 [batch][H_kv] */
 dl_status dl_sparse_attn_gather(const dl_attn_desc* desc, const void* Q_dec, const void* K_pool,
                                 const void* V_pool, const int32_t* page_table,
