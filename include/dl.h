@@ -121,6 +121,25 @@ dl_status dl_pool_keys(const dl_attn_desc* desc, const void* K_pool, const int32
                        int n_units, int unit_stride, int unit_offset, int unit_len,
                        float* Kbar, void* stream);
 
+/* Cache refresh with the block pooling fused into the write.  [F2 summary:
+ * the context is held in a KV cache; blocks are scored by their mean key]
+ * A finished decode block's n_new tokens of every sequence b join the cached
+ * context at logical positions start[b] .. start[b] + n_new - 1: they are
+ * written into the pools through the page table, and the pooled key of every
+ * block those positions touch is recomputed as dl_pool_keys (page, 0, page)
+ * would (mean over the block's positions < L_ctx, in fp64, rounded once to
+ * fp32; the block's other rows are read back from the pool).  Other blocks
+ * of Kbar are left as they are.  The descriptor describes the context after
+ * the write: start[b] + n_new <= L_ctx, else the sequence is skipped and
+ * DL_ERR_BAD_INDEX reported; so is a touched page whose slot is out of range.
+ *   K_new, V_new  [batch][H_kv][n_new][d] (bf16/fp32, 16-byte aligned)
+ *   start         int32 [batch] (device)
+ *   K_pool, V_pool, page_table  see layouts (written / read)
+ *   Kbar          fp32 [batch][H_kv][n_blk][d]  (touched blocks written) */
+dl_status dl_cache_write(const dl_attn_desc* desc, const void* K_new, const void* V_new,
+                         int n_new, const int32_t* start, const int32_t* page_table,
+                         void* K_pool, void* V_pool, float* Kbar, void* stream);
+
 /* (a3) Block scores with a fused block-level softmax.  [F2 summary]
  * For KV head g, rows r = (h in g's query heads, i in predicted positions):
  *   score[b][g][j] = sum_r softmax_j( scale * q_{h,i} . Kbar[b][g][j] )

@@ -46,6 +46,8 @@ _SIGS = {
     "dl_predict_queries": ([_vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
     "dl_pool_keys": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _c_int, _c_int, _c_int, _c_int,
                       _vp, _vp], _c_int),
+    "dl_cache_write": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp,
+                        _vp], _c_int),
     "dl_block_scores": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _c_int, _vp, _vp,
                          ctypes.c_size_t, _vp], _c_int),
     "dl_find_sinks": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp,
@@ -132,6 +134,12 @@ def dl_pool_keys(desc, K_pool, page_table, n_units, unit_stride, unit_offset, un
                  stream=None):
     _check(lib.dl_pool_keys(ctypes.byref(desc), _p(K_pool), _p(page_table), n_units, unit_stride,
                             unit_offset, unit_len, _p(Kbar), _s(stream)))
+
+
+def dl_cache_write(desc, K_new, V_new, start, page_table, K_pool, V_pool, Kbar, stream=None):
+    _check(lib.dl_cache_write(ctypes.byref(desc), _p(K_new), _p(V_new), K_new.shape[-2],
+                              _p(start), _p(page_table), _p(K_pool), _p(V_pool), _p(Kbar),
+                              _s(stream)))
 
 
 def dl_block_scores(desc, Q_dec, q_idx, q_cnt, Kbar, n_units, score, ws, stream=None):

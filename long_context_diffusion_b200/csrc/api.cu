@@ -187,6 +187,25 @@ dl_status dl_pool_keys(const dl_attn_desc* desc, const void* K_pool, const int32
                   "dl_pool_keys launch");
 }
 
+dl_status dl_cache_write(const dl_attn_desc* desc, const void* K_new, const void* V_new,
+                         int n_new, const int32_t* start, const int32_t* page_table,
+                         void* K_pool, void* V_pool, float* Kbar, void* stream) {
+  dl::Shape s;
+  dl_status st = check_desc(desc, &s);
+  if (st != DL_OK) return st;
+  if (!K_new || !V_new || !start || !page_table || !K_pool || !V_pool || !Kbar)
+    return fail(DL_ERR_INVALID_ARG, "dl_cache_write: NULL pointer");
+  if (!aligned16(K_new) || !aligned16(V_new) || !aligned16(K_pool) || !aligned16(V_pool))
+    return fail(DL_ERR_INVALID_ARG, "dl_cache_write: K/V buffers must be 16-byte aligned");
+  if (n_new < 1 || n_new > s.L_ctx)
+    return fail(DL_ERR_INVALID_ARG, "n_new=%d (need 1..L_ctx=%d)", n_new, s.L_ctx);
+  unsigned* err = nullptr;
+  if ((st = error_word(&err)) != DL_OK) return st;
+  return launched(dl::launch_cache_write(s, K_new, V_new, n_new, start, page_table, K_pool,
+                                         V_pool, Kbar, err, as_stream(stream)),
+                  "dl_cache_write launch");
+}
+
 dl_status dl_block_scores(const dl_attn_desc* desc, const void* Q_dec, const int32_t* q_idx,
                           const int32_t* q_cnt, const float* Kbar, int n_units, double* score,
                           void* ws, size_t ws_bytes, void* stream) {

@@ -79,6 +79,9 @@ cudaError_t launch_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
 
+cudaError_t launch_cache_write(const Shape& s, const void* K_new, const void* V_new, int n_new,
+                               const int32_t* start, const int32_t* page_table, void* Kp,
+                               void* Vp, float* Kbar, unsigned* err, cudaStream_t st);
 cudaError_t launch_token_select(const Shape& s, const void* Q, const void* Kp,
                                 const int32_t* page_table, const int32_t* chunk_idx, int n_sel,
                                 int chunk_stride, int chunk_content, int topT, int32_t* tok_pos,

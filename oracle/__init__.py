@@ -49,6 +49,6 @@ from .steps import (  # noqa: F401
     scale_for, predict_queries, pool_mean, pooled_keys, block_scores,
     select_blocks, find_sinks, attention_rows, sparse_attention,
     gather_context, chunk_pooled_keys, chunk_scores, token_select,
-    chunk_attention, dense_attention, topk_lower_index,
+    chunk_attention, dense_attention, topk_lower_index, cache_write,
 )
 from .step import layer_step, chunked_step, StepResult, ChunkResult  # noqa: F401

@@ -12,7 +12,7 @@ __all__ = [
     "scale_for", "topk_lower_index", "predict_queries", "pool_mean", "pooled_keys",
     "block_scores", "select_blocks", "find_sinks", "attention_rows",
     "gather_context", "sparse_attention", "dense_attention", "chunk_pooled_keys",
-    "chunk_scores", "token_select", "chunk_attention",
+    "chunk_scores", "token_select", "chunk_attention", "cache_write",
 ]
 
 
@@ -265,3 +265,33 @@ def chunk_attention(Q, K_pool, V_pool, page_row, positions_per_g, B: int, K_dec,
         for h in range(g * G, (g + 1) * G):
             O[:, h], lse[h] = attention_rows(Qf[h], keys, vals, scale)
     return O, lse
+
+
+# --------------------------------------------------------------------------
+# cache refresh: a finished decode block written into the paged cache, with
+# the pooled keys of the blocks it touches
+# --------------------------------------------------------------------------
+def cache_write(K_pool, V_pool, page_row, K_new, V_new, start: int, L_ctx: int, B: int):
+    """The decode block's tokens join the cached context (Focus-dLLM summary:
+    the context is held in a KV cache; its pooled block keys are what the
+    block scores read).  K_new, V_new: [H_kv][n_new][d] at logical positions
+    start .. start + n_new - 1, written through the page table (slot
+    page_row[t // B], row t % B); then every block j those positions touch
+    gets the pooled key of pooled_keys (mean of its positions < L_ctx, read
+    back through the page table, rounded once to fp32).  Returns the updated
+    pools (copies) and {j: Kbar_j [H_kv][d]}."""
+    Kp = np.array(f64(K_pool), copy=True)
+    Vp = np.array(f64(V_pool), copy=True)
+    Kn, Vn = f64(K_new), f64(V_new)
+    row = np.asarray(page_row, dtype=np.int64)
+    n_new = Kn.shape[1]
+    for t in range(n_new):
+        pos = start + t
+        Kp[row[pos // B], :, pos % B] = Kn[:, t]
+        Vp[row[pos // B], :, pos % B] = Vn[:, t]
+    kbar = {}
+    for j in range(start // B, (start + n_new - 1) // B + 1):
+        pos = np.arange(j * B, min((j + 1) * B, L_ctx))
+        kbar[j] = np.stack([pool_mean(gather_context(Kp, row, g, pos, B))
+                            for g in range(Kp.shape[1])]).astype(np.float32).astype(np.float64)
+    return Kp, Vp, kbar

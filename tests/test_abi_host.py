@@ -23,7 +23,7 @@ def test_header_declares_the_path():
     names = _declared()
     for n in ("dl_predict_queries", "dl_pool_keys", "dl_block_scores", "dl_find_sinks",
               "dl_select", "dl_block_select", "dl_sparse_attn", "dl_token_select",
-              "dl_sparse_attn_gather", "dl_workspace_size", "dl_get_status"):
+              "dl_sparse_attn_gather", "dl_cache_write", "dl_workspace_size", "dl_get_status"):
         assert n in names
 
 
@@ -91,3 +91,20 @@ def test_null_and_range_arguments_rejected_before_launch():
     st = lib.dl_token_select(ctypes.byref(d), fake, fake, fake, fake, 8, 1088, 2048, 256, fake,
                              fake, None, 0, None)
     assert st == dl.DL_ERR_INVALID_ARG
+
+
+
+def test_cache_write_arguments_rejected_before_launch():
+    lib = _abi.lib
+    d = _desc()
+    fake = ctypes.c_void_p(0x1000)
+    args = [fake, fake, 32, fake, fake, fake, fake, fake, None]
+    assert lib.dl_cache_write(ctypes.byref(d), *args[:1], None, *args[2:]) == dl.DL_ERR_INVALID_ARG
+    for n_new in (0, 16385):  # 1 .. L_ctx
+        a = list(args)
+        a[2] = n_new
+        assert lib.dl_cache_write(ctypes.byref(d), *a) == dl.DL_ERR_INVALID_ARG
+    a = list(args)
+    a[0] = ctypes.c_void_p(0x1008)  # K_new off the 16-byte grid
+    assert lib.dl_cache_write(ctypes.byref(d), *a) == dl.DL_ERR_INVALID_ARG
+    assert "aligned" in lib.dl_last_error_message().decode()

@@ -400,3 +400,48 @@ def test_layer_step_tiny_invariants():
                                inp.v_dec, wl.L_ctx, wl.B, 0, q_idx=r.q_idx, q_cnt=r.q_cnt,
                                dense=True)
     assert np.allclose(rd.O, rdense.O, rtol=0, atol=1e-13)
+
+
+# ------------------------------------------------------------ cache refresh
+def _paged(n_pages, H_kv, B, d, seed):
+    r = np.random.default_rng(seed)
+    pool = r.standard_normal((n_pages, H_kv, B, d)).astype(np.float32).astype(np.float64)
+    row = r.permutation(n_pages)
+    return pool, row
+
+
+def test_cache_write_of_cached_tokens_changes_nothing():
+    B, d, H_kv, L_ctx = 8, 4, 2, 45
+    Kp, row = _paged(6, H_kv, B, d, 1)
+    Vp, _ = _paged(6, H_kv, B, d, 2)
+    start, n = 13, 20
+    pos = np.arange(start, start + n)
+    Kn = np.stack([S.gather_context(Kp, row, g, pos, B) for g in range(H_kv)])
+    Vn = np.stack([S.gather_context(Vp, row, g, pos, B) for g in range(H_kv)])
+    K2, V2, kbar = oracle.cache_write(Kp, Vp, row, Kn, Vn, start, L_ctx, B)
+    assert np.array_equal(K2, Kp) and np.array_equal(V2, Vp)
+    assert sorted(kbar) == [1, 2, 3, 4]
+    for g in range(H_kv):
+        ref = S.pooled_keys(S.gather_context(Kp, row, g, np.arange(L_ctx), B), L_ctx, B)
+        for j, v in kbar.items():
+            assert np.array_equal(v[g], ref[j])
+
+
+def test_cache_write_closed_forms_and_untouched_rows():
+    B, d, H_kv, L_ctx = 8, 3, 1, 30   # blocks 0..3, the last holds 6 positions
+    Kp = np.full((4, H_kv, B, d), 2.0)
+    Vp = np.full((4, H_kv, B, d), -1.0)
+    row = np.array([2, 0, 3, 1])
+    start, n = 5, 20                  # positions 5..24: block 0 partly, 1 and 2 fully, 3 partly
+    Kn = np.full((H_kv, n, d), 6.0)
+    Vn = np.full((H_kv, n, d), 7.0)
+    K2, V2, kbar = oracle.cache_write(Kp, Vp, row, Kn, Vn, start, L_ctx, B)
+    assert sorted(kbar) == [0, 1, 2, 3]
+    assert np.allclose(kbar[0], (5 * 2.0 + 3 * 6.0) / 8)   # 5 old rows, 3 new
+    assert np.allclose(kbar[1], 6.0) and np.allclose(kbar[2], 6.0)
+    assert np.allclose(kbar[3], (1 * 6.0 + 5 * 2.0) / 6)  # position 24: 1 new of 6 valid
+    for t in range(32):
+        k = K2[row[t // B], 0, t % B]
+        v = V2[row[t // B], 0, t % B]
+        new = start <= t < start + n
+        assert np.all(k == (6.0 if new else 2.0)) and np.all(v == (7.0 if new else -1.0))
