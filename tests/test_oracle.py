@@ -403,7 +403,7 @@ def test_layer_step_tiny_invariants():
 
 
 # ------------------------------------------------------------ cache refresh
-def _paged(n_pages, H_kv, B, d, seed):
+def _random_pool(n_pages, H_kv, B, d, seed):
     r = np.random.default_rng(seed)
     pool = r.standard_normal((n_pages, H_kv, B, d)).astype(np.float32).astype(np.float64)
     row = r.permutation(n_pages)
@@ -412,8 +412,8 @@ def _paged(n_pages, H_kv, B, d, seed):
 
 def test_cache_write_of_cached_tokens_changes_nothing():
     B, d, H_kv, L_ctx = 8, 4, 2, 45
-    Kp, row = _paged(6, H_kv, B, d, 1)
-    Vp, _ = _paged(6, H_kv, B, d, 2)
+    Kp, row = _random_pool(6, H_kv, B, d, 1)
+    Vp, _ = _random_pool(6, H_kv, B, d, 2)
     start, n = 13, 20
     pos = np.arange(start, start + n)
     Kn = np.stack([S.gather_context(Kp, row, g, pos, B) for g in range(H_kv)])
