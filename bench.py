@@ -9,12 +9,19 @@ reuse; sparse layers keep the top-128 of 512 blocks plus the sink blocks.
 Synthetic bf16 inputs drawn by the seeded generator (`synth`), resident in
 HBM (68.7 GB of KV cache) before the timed region.
 
-A step = one refresh of one layer's pooled keys (the KV-cache refresh of a
-32-step block, amortised one layer per step) + query prediction + 32 layers
+A step = the cache refresh of one layer (a finished 32-token decode block
+joins the cached context of one layer: written into the pools with its
+block's pooled key recomputed, dl_cache_write; the 32 layers of a 32-step
+block amortised one layer per step) + query prediction + 32 layers
 (pooled-key scores, sinks at layer 2, selection, attention).  K steps are
 captured in one CUDA graph and timed with CUDA events on the launch stream;
-each attention call is bracketed by graph event nodes to time the dominant
-kernel over the same region.
+each attention call and each cache write is bracketed by graph event nodes to
+time them over the same region.
+
+The same line carries sub-records for the other workloads (single-layer
+steps at 8K and 16K, the chunked 32K prefix, the tiny fp32 layer), each timed
+as a CUDA-graph replay with the L2 flushed before it, and the whole-layer
+pooled-key rebuild that a cache whose context K/V are recomputed needs.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -38,7 +45,6 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 import synth  # noqa: E402
-from long_context_diffusion_b200 import runtime  # noqa: E402
 
 METRIC = "sparse-attn denoise steps/s and KV-tokens/s at 32K; % of HBM/tensor roofline"
 WORKLOAD = "llada32k_step"
@@ -48,9 +54,9 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 
 
 # DRAM traffic of the dominant kernel from one ncu capture at the benchmark's
-# size (profiles/attn_tc_kt_sparse_llada32k.md: dram__bytes_read.sum +
-# dram__bytes_write.sum of one sparse-layer launch, batch 4: 557.93 + 8.33 MB).
-# Reported only while the kernel's sources hash to the captured build.
+# size (dram__bytes_read.sum + dram__bytes_write.sum of one sparse-layer
+# launch, batch 4: 557.93 + 8.33 MB).  Reported only while the kernel's
+# sources hash to the captured build.
 TRAFFIC_CAPTURE = {"sha": "c35242f1710dd185", "bytes_per_launch": 557.928192e6 + 8.3264e6,
                    "sources": ["attn_tc_kt.cu", "tc_common.cuh", "sm100.cuh"]}
 
@@ -167,6 +173,110 @@ def attn_flops(wl, n_ctx_tokens_per_bg):
     return 4.0 * wl.d * keys * wl.G * wl.L_q
 
 
+def cache_write_bytes(wl, start, n_new):
+    """Algorithmic HBM bytes of one dl_cache_write over all (b, g): the new K
+    and V rows read and written, the touched blocks' other rows read back,
+    and their pooled keys written."""
+    e = 2
+    j0, j1 = start // wl.B, (start + n_new - 1) // wl.B
+    rows = sum(min(wl.B, wl.L_ctx - j * wl.B) for j in range(j0, j1 + 1))
+    per_bg = n_new * wl.d * e * 4 + (rows - n_new) * wl.d * e + (j1 - j0 + 1) * wl.d * 4
+    return wl.batch * wl.H_kv * per_bg
+
+
+def _graph_time_us(fn, device, reps, flush_l2=True):
+    """Median device time of one CUDA-graph replay of fn (captured on a side
+    stream), the L2 flushed (a 256 MiB write) before each replay."""
+    side = torch.cuda.Stream(device)
+    side.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(side):
+        out = fn(side)
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        out = fn(side)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    times = []
+    for r in range(reps + 3):
+        with torch.cuda.stream(side):
+            if flush_l2:
+                flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(side)
+            g.replay()
+            e1.record(side)
+        torch.cuda.synchronize(device)
+        if r >= 3:
+            times.append(e0.elapsed_time(e1) * 1e3)
+    del g
+    return float(statistics.median(times)), out
+
+
+def workload_record(name, device, pk, reps=30):
+    """One step of a single-layer or chunked workload: median graph-replay
+    time, algorithmic bytes, and the fraction of the measured and nominal
+    HBM rooflines."""
+    import long_context_diffusion_b200 as dl
+    from long_context_diffusion_b200 import pipeline
+    wl = synth.workload(name)
+    inp = synth.make_step_inputs(wl, device=device)
+    e = 4 if wl.dtype == "fp32" else 2
+    desc = dl.make_desc(wl.batch, wl.H, wl.H_kv, wl.d, wl.L_ctx, wl.L_q, wl.B, wl.n_pages,
+                        wl.n_slots, dl.DL_FP32 if wl.dtype == "fp32" else dl.DL_BF16)
+    ws = pipeline.workspace(desc, device)
+    n_units = wl.n_chunks if wl.chunked else wl.n_blk
+    Kbar = torch.empty((wl.batch, wl.H_kv, n_units, wl.d), dtype=torch.float32, device=device)
+    if wl.chunked:  # chunk keys belong to the cache build, not to the step
+        dl.dl_pool_keys(desc, inp.k_pool, inp.page_table, wl.n_chunks, wl.chunk_stride, 1,
+                        wl.chunk_content, Kbar)
+
+        def fn(st):
+            return pipeline.chunked_step(desc, inp.q_dec, inp.k_pool, inp.v_pool, inp.page_table,
+                                         inp.k_dec, inp.v_dec, n_chunks=wl.n_chunks,
+                                         stride=wl.chunk_stride, content=wl.chunk_content,
+                                         topK_chunks=wl.topK_chunks, topT=wl.topT_tokens,
+                                         Kbar=Kbar, ws=ws, stream=st)
+    else:
+        dl.dl_pool_keys(desc, inp.k_pool, inp.page_table, wl.n_blk, wl.B, 0, wl.B, Kbar)
+        sinks = inp.sinks_planted[:, :wl.sinks_given].contiguous() if wl.sinks_given else None
+
+        def fn(st):
+            return pipeline.layer_step(desc, inp.q_dec, inp.k_pool, inp.v_pool, inp.page_table,
+                                       inp.k_dec, inp.v_dec, topK=wl.topK,
+                                       conf_prev=inp.conf_prev, still_masked=inp.still_masked,
+                                       k=wl.k, w=wl.w, sink_pos=sinks, Kbar=Kbar, ws=ws,
+                                       stream=st)
+    us, out = _graph_time_us(fn, device, reps)
+    if dl.dl_get_status() != dl.DL_OK:
+        raise RuntimeError(f"device status after the {name} step")
+    q_b = inp.q_dec.numel() * e
+    dec_b = inp.k_dec.numel() * e * 2
+    o_b = out.O.numel() * e + out.lse.numel() * 4
+    if wl.chunked:
+        kc = int(out.chunk_cnt.sum().item())
+        n_tok = int(out.tok_cnt.sum().item())
+        ctx_tokens = n_tok / (wl.batch * wl.H_kv)
+        nbytes = (Kbar.numel() * 4 + q_b + kc * wl.chunk_content * wl.d * e +
+                  n_tok * wl.d * e * 2 + dec_b + o_b)
+    else:
+        cnt = out.blk_cnt.view(-1).cpu().tolist()
+        idx = out.blk_idx.view(len(cnt), -1).cpu()
+        toks = 0
+        for r, c in enumerate(cnt):
+            last = int((idx[r, :c] == wl.n_blk - 1).sum().item())
+            toks += int(c) * wl.B - last * (wl.n_blk * wl.B - wl.L_ctx)
+        ctx_tokens = toks / (wl.batch * wl.H_kv)
+        nbytes = (Kbar.numel() * 4 + q_b + wl.batch * wl.H_kv * wl.n_blk * 8 +
+                  toks * wl.d * e * 2 + dec_b + o_b)
+    t = us * 1e-6
+    return {"workload": name, "us_per_step": us, "steps_per_s": 1.0 / t,
+            "kv_tokens_per_s": wl.batch * (ctx_tokens + wl.L_q) / t,
+            "bytes": int(nbytes), "achieved_GBps": nbytes / t / 1e9,
+            "frac_of_measured": nbytes / t / 1e9 / pk["hbm_gbs"],
+            "frac_of_nominal_8tbs": nbytes / t / 1e9 / NOMINAL_HBM_GBS,
+            "timing": f"median of {reps} CUDA-graph replays, L2 flushed before each"}
+
+
 # ---------------------------------------------------------------- oracle arm
 def oracle_sample(wl, seconds_budget=8.0):
     """Times the fp64 oracle on a bounded sample of the step and scales it to
@@ -237,8 +347,9 @@ def oracle_sample(wl, seconds_budget=8.0):
 
 
 def run_reference(args):
-    rank, world, _ = runtime.env_rank()
-    if rank != 0:
+    # The oracle arm never touches the GPU library: the package (which loads
+    # libdlsparse.so on import) is not imported here.
+    if int(os.environ.get("RANK", "0")) != 0:
         return 0
     wl = synth.workload(WORKLOAD)
     times = []
@@ -272,6 +383,7 @@ def config_of(wl):
 
 # ---------------------------------------------------------------- our arm
 def run_ours(args):
+    from long_context_diffusion_b200 import runtime
     rank, world, local, device = runtime.init()
     import long_context_diffusion_b200 as dl
     from long_context_diffusion_b200 import pipeline
@@ -293,8 +405,18 @@ def run_ours(args):
                        [x["vp"] for x in layers], pt, [x["kd"] for x in layers],
                        [x["vd"] for x in layers], Kbar)
 
-    def one_step(i, events=None):
-        step.refresh_pooled_keys(i % L, layers[i % L]["kp"], pt, Kbar[i % L], stream)
+    # the finished decode block joins the context as its last L_q positions
+    start = torch.full((wl.batch,), wl.L_ctx - wl.L_q, dtype=torch.int32, device=device)
+    cw_events = []
+
+    def commit(i, kd, vd, events=None):
+        ev = step._begin(events, stream)
+        step.commit_block(kd, vd, start, layers[i % L]["kp"], layers[i % L]["vp"], pt,
+                          Kbar[i % L], stream)
+        step._end(events, ev, i % L, stream)
+
+    def one_step(i, events=None, cw=None):
+        commit(i, layers[i % L]["kd"], layers[i % L]["vd"], cw)
         step.run(*args_of(), stream=stream, attn_events=events)
 
     with torch.cuda.stream(stream):
@@ -314,7 +436,7 @@ def run_ours(args):
     g_timed = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_timed, stream=stream):
         for i in range(K):
-            one_step(i, events)
+            one_step(i, events, cw_events)
     for _ in range(W):
         g_warm.replay()
     torch.cuda.synchronize(device)
@@ -378,7 +500,7 @@ def run_ours(args):
 
     # step-level roofline: algorithmic bytes of every kernel of one step
     e2b = 2
-    pool_b = wl.batch * wl.H_kv * wl.L_ctx * wl.d * e2b + wl.batch * wl.H_kv * n_blk * wl.d * 4
+    cw_b = cache_write_bytes(wl, wl.L_ctx - wl.L_q, wl.L_q)
     kbar_b = wl.batch * wl.H_kv * n_blk * wl.d * 4
     q_b = wl.batch * wl.H * wl.L_q * wl.d * e2b
     # sink search: K counted once (the kernels stream it twice: the row LSEs
@@ -386,7 +508,7 @@ def run_ours(args):
     sink_b = wl.batch * wl.H_kv * (wl.L_ctx + wl.L_q) * wl.d * e2b + q_b
     n_sparse = L - wl.first_sparse_layer
     score_b = n_sparse * (kbar_b + q_b + wl.batch * wl.H_kv * n_blk * 8)
-    step_bytes = pool_b + sink_b + score_b + sum(attn_b)
+    step_bytes = cw_b + sink_b + score_b + sum(attn_b)
     step_flops = sum(attn_f)
     t_roof_meas = max(step_bytes / (pk["hbm_gbs"] * 1e9), step_flops / (pk["bf16_tflops"] * 1e12))
     t_roof_nom = max(step_bytes / (NOMINAL_HBM_GBS * 1e9),
@@ -447,7 +569,7 @@ def run_ours(args):
                 if i + 1 < K:
                     upload(i + 1)
                 stream.wait_event(in_ready[j])
-                step.refresh_pooled_keys(i % L, layers[i % L]["kp"], pt, Kbar[i % L], stream)
+                commit(i, dev_in[j][(i % L, "kd")], dev_in[j][(i % L, "vd")])
                 step.run(*args_set(j), stream=stream)
                 in_free[j] = torch.cuda.Event()
                 in_free[j].record(stream)
@@ -511,6 +633,33 @@ def run_ours(args):
         "gpu_launches": launches_per_step * K,
         "gen_seconds": t_gen,
     }
+    # cache refresh on the timed path: one decode block joining one layer
+    cw_us = [s_.elapsed_time(e_) * 1e3 for _, s_, e_ in cw_events]
+    cw_b = cache_write_bytes(wl, wl.L_ctx - wl.L_q, wl.L_q)
+    cw_mean = sum(cw_us) / max(1, len(cw_us))
+    line["cache_write"] = {
+        "call": "dl_cache_write", "n_new": wl.L_q, "start": wl.L_ctx - wl.L_q,
+        "avg_us": cw_mean, "launches": len(cw_us), "bytes_per_call": cw_b,
+        "achieved_GBps": cw_b / (cw_mean * 1e-6) / 1e9 if cw_mean > 0 else None}
+    # whole-layer pooled-key rebuild (a cache whose context K/V are recomputed)
+    with torch.cuda.stream(stream):
+        ts = []
+        for r in range(6):
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            step.refresh_pooled_keys(r % L, layers[r % L]["kp"], pt, Kbar[r % L], stream)
+            b_.record(stream)
+            ts.append((a_, b_))
+    torch.cuda.synchronize(device)
+    pool_us = [a_.elapsed_time(b_) * 1e3 for a_, b_ in ts[1:]]
+    pool_b = wl.batch * wl.H_kv * (wl.L_ctx * wl.d * 2 + wl.n_blk * wl.d * 4)
+    pm = sum(pool_us) / len(pool_us)
+    line["full_layer_pool"] = {"call": "dl_pool_keys", "avg_us": pm, "bytes": pool_b,
+                               "achieved_GBps": pool_b / (pm * 1e-6) / 1e9,
+                               "step_ms_if_amortised_per_step": ms_step + (pm - cw_mean) / 1e3}
+    if not args.no_configs:
+        line["workloads"] = {n: workload_record(n, device, pk)
+                             for n in ("tiny", "llada8k", "dream16k", "chunked32k")}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         v, cores, sample, _ = oracle_sample(synth.workload(WORKLOAD))
         line["cpu_baseline"] = {"value": v, "unit": "steps/s", "cores": cores, "kind": "oracle",
@@ -542,6 +691,8 @@ def main():
     ap.add_argument("--batch", type=int, default=4)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the sub-records of the other workloads")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours" and args.layers == 32:
         args.warmup = 3

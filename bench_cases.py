@@ -1,9 +1,9 @@
 """One kernel of the denoising step, on one synthetic layer, for profiling.
 
-    python -m long_context_diffusion_b200.profile_case --case attn_sparse --reps 3
-    python -m long_context_diffusion_b200.profile_case --case block_select --reps 3
-    python -m long_context_diffusion_b200.profile_case --case sinks --reps 3
-    python -m long_context_diffusion_b200.profile_case --case chunk_step --reps 20
+    python bench_cases.py --case attn_sparse --reps 3
+    python bench_cases.py --case block_select --reps 3
+    python bench_cases.py --case sinks --reps 3
+    python bench_cases.py --case chunk_step --reps 20
 
 Builds one sparse layer of the 32K workload (batch 4, 32 KV heads, 32K context:
 about 2.1 GB of K/V pages on the device), runs the steps before the profiled
@@ -21,11 +21,15 @@ from __future__ import annotations
 
 import argparse
 import json
+import os
+import sys
 
-import torch
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 
-import synth
-from . import _abi as A
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+from long_context_diffusion_b200 import _abi as A  # noqa: E402
 
 
 def main():
@@ -99,7 +103,7 @@ def main():
 
 
 def chunk_step(reps: int, dev):
-    from . import pipeline
+    from long_context_diffusion_b200 import pipeline
     wl = synth.workload("chunked32k")
     inp = synth.make_step_inputs(wl, device=dev)
     desc = A.make_desc(wl.batch, wl.H, wl.H_kv, wl.d, wl.L_ctx, wl.L_q, wl.B, wl.n_pages,

@@ -76,6 +76,21 @@ typedef struct {
   int dtype;    /* dl_dtype of Q_dec, K/V pools, K_dec/V_dec and O         */
 } dl_attn_desc;
 
+/* Kernel-choice switches.  They exist for the tests, which run every kernel
+ * of a step against the oracle: each switch sends a call to another kernel
+ * that computes the same result.  The default, 0, is the product path.
+ *   DL_FLAG_TOKEN_SIMT   dl_token_select on its CUDA-core kernel
+ *   DL_FLAG_GATHER_SIMT  dl_sparse_attn_gather on its CUDA-core kernel
+ *   DL_FLAG_PDL          every kernel launched with programmatic dependent
+ *                        launch (measured no faster inside a CUDA graph)
+ *   DL_FLAG_SCORE_FP64   dl_block_select always on the fp64 scoring kernel
+ *                        (skips the certified integer tensor-core scoring)
+ * Process-wide; read by each later call at launch time.  No environment
+ * variable changes the kernel choice.  Returns the previous flags. */
+enum { DL_FLAG_TOKEN_SIMT = 1u, DL_FLAG_GATHER_SIMT = 2u, DL_FLAG_PDL = 4u,
+       DL_FLAG_SCORE_FP64 = 8u };
+unsigned dl_set_kernel_flags(unsigned flags);
+
 /* Library version (major*10000 + minor*100 + patch). */
 int dl_version(void);
 
@@ -112,7 +127,9 @@ dl_status dl_predict_queries(const float* conf_prev, const uint8_t* still_masked
  * relevant KV; pooling reading: one mean key per block]
  * Unit u of sequence b covers logical tokens
  *   [u*unit_stride + unit_offset, u*unit_stride + unit_offset + unit_len)
- * clipped to [0, L_ctx).  Kbar[b][g][u] = (exact sum of those K rows) / n,
+ * clipped to [0, L_ctx).  Kbar[b][g][u] = (sum of those K rows) / n, the
+ * sum taken in fp64 (exact for bf16 keys; for fp32 keys exact while the
+ * summed values' exponents lie within 29 - log2(n) binades of each other),
  * rounded once to fp32 (units with no valid token get 0).  Key blocks use
  * (stride, offset, len) = (page, 0, page); Prefilling-dLLM chunks [P1] with a
  * BOS anchor first use (chunk_stride, 1, chunk_content).
@@ -128,10 +145,17 @@ dl_status dl_pool_keys(const dl_attn_desc* desc, const void* K_pool, const int32
  * written into the pools through the page table, and the pooled key of every
  * block those positions touch is recomputed as dl_pool_keys (page, 0, page)
  * would (mean over the block's positions < L_ctx, in fp64, rounded once to
- * fp32; the block's other rows are read back from the pool).  Other blocks
- * of Kbar are left as they are.  The descriptor describes the context after
- * the write: start[b] + n_new <= L_ctx, else the sequence is skipped and
- * DL_ERR_BAD_INDEX reported; so is a touched page whose slot is out of range.
+ * fp32; the block's other rows are read back from the pool).  For bf16 the
+ * result equals dl_pool_keys' bit for bit; for fp32 keys the fp64 sums of
+ * the two calls are taken in different orders and the pooled key can differ
+ * by one fp32 ulp.  Other blocks of Kbar are left as they are.  The
+ * descriptor describes the context after the write: start[b] + n_new <=
+ * L_ctx, else that sequence is skipped entirely and DL_ERR_BAD_INDEX is
+ * reported.  Blocks are checked one by one: a touched block whose page slot
+ * is out of range is skipped (its pool rows and its Kbar entry are not
+ * written) and DL_ERR_BAD_INDEX is reported, while the sequence's other
+ * touched blocks are still written, so that sequence's cache is then
+ * partly updated.
  *   K_new, V_new  [batch][H_kv][n_new][d] (bf16/fp32, 16-byte aligned)
  *   start         int32 [batch] (device)
  *   K_pool, V_pool, page_table  see layouts (written / read)

@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_PKG, "lib", "libdlsparse.so")
 DL_OK, DL_ERR_INVALID_ARG, DL_ERR_UNSUPPORTED, DL_ERR_WORKSPACE = 0, 1, 2, 3
 DL_ERR_CUDA, DL_ERR_BAD_INDEX, DL_ERR_TIMEOUT = 4, 5, 6
 DL_BF16, DL_FP32 = 0, 1
+DL_FLAG_TOKEN_SIMT, DL_FLAG_GATHER_SIMT, DL_FLAG_PDL, DL_FLAG_SCORE_FP64 = 1, 2, 4, 8
 STATUS_NAMES = {0: "DL_OK", 1: "DL_ERR_INVALID_ARG", 2: "DL_ERR_UNSUPPORTED",
                 3: "DL_ERR_WORKSPACE", 4: "DL_ERR_CUDA", 5: "DL_ERR_BAD_INDEX",
                 6: "DL_ERR_TIMEOUT"}
@@ -40,6 +41,7 @@ class dl_attn_desc(ctypes.Structure):
 _c_int, _vp, _i32p = ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p
 _SIGS = {
     "dl_version": ([], ctypes.c_int),
+    "dl_set_kernel_flags": ([ctypes.c_uint], ctypes.c_uint),
     "dl_last_error_message": ([], ctypes.c_char_p),
     "dl_get_status": ([_vp], _c_int),
     "dl_workspace_size": ([ctypes.POINTER(dl_attn_desc), ctypes.POINTER(ctypes.c_size_t)], _c_int),
@@ -111,6 +113,12 @@ def make_desc(batch, H, H_kv, d, L_ctx, L_q, page, n_pages, n_slots, dtype) -> d
 
 def dl_version() -> int:
     return lib.dl_version()
+
+
+def dl_set_kernel_flags(flags: int) -> int:
+    """Kernel-choice switches for the tests (DL_FLAG_*); returns the previous
+    flags."""
+    return int(lib.dl_set_kernel_flags(int(flags)))
 
 
 def dl_get_status(stream=None) -> int:

@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/dl.h"
@@ -106,6 +107,8 @@ dl_status launched(cudaError_t e, const char* what) {
 
 int n_blk_of(const dl::Shape& s) { return (s.L_ctx + s.page - 1) / s.page; }
 
+std::atomic<unsigned> g_kernel_flags{0u};
+
 }  // namespace
 
 // Validation and error-word access for entry points defined in other files.
@@ -114,11 +117,14 @@ dl_status api_check_desc(const dl_attn_desc* d, Shape* s) { return check_desc(d,
 dl_status api_error_word(unsigned** out) { return error_word(out); }
 dl_status api_fail(dl_status st, const char* msg) { return fail(st, "%s", msg); }
 dl_status api_ok() { return ok(); }
+unsigned kernel_flags() { return g_kernel_flags.load(std::memory_order_relaxed); }
 }  // namespace dl
 
 extern "C" {
 
-int dl_version(void) { return 100; }
+int dl_version(void) { return 200; }
+
+unsigned dl_set_kernel_flags(unsigned flags) { return g_kernel_flags.exchange(flags); }
 
 const char* dl_last_error_message(void) { return g_msg; }
 

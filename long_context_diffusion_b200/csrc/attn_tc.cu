@@ -791,7 +791,7 @@ static cudaError_t run_tc(const AttnArgs& a, int max_tiles, cudaStream_t st) {
 // at most two M-tiles of query rows, pool addressable by 32-bit TMA rows).
 bool attn_tc_supported(const AttnArgs& a) {
   const Shape& s = a.s;
-  return s.dtype == 0 && (a.mode != kGather || !getenv("DL_GATHER_SIMT")) && s.G * s.L_q <= 256 &&
+  return s.dtype == 0 && (a.mode != kGather || !(kernel_flags() & DL_FLAG_GATHER_SIMT)) && s.G * s.L_q <= 256 &&
          (uint64_t)s.n_slots * s.H_kv * 64 < (1ull << 31) &&
          (uint64_t)s.batch * s.H * s.L_q < (1ull << 31);
 }

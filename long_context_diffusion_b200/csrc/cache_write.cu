@@ -10,10 +10,12 @@
 // CTA (k, b, g): the k-th block touched by sequence b's positions
 // start[b] .. start[b] + n_new - 1, KV head g.  Thread (row group, 16-byte
 // column chunk): its rows of the block, new ones copied from K_new/V_new into
-// the pools, old ones read from the K pool, summed in fp64 (exact for bf16,
-// so the order does not matter); the row groups' sums are added in shared
-// memory and the mean over the block's positions below L_ctx is rounded once
-// to fp32.
+// the pools, old ones read from the K pool, summed in fp64; the row groups'
+// sums are added in shared memory and the mean over the block's positions
+// below L_ctx is rounded once to fp32.  For bf16 keys the fp64 sum is exact,
+// so the result equals dl_pool_keys bit for bit whatever the order; for fp32
+// keys the fp64 sum is exact only while the 64 values' exponents are close,
+// and the pooled key can then differ from dl_pool_keys' by one fp32 ulp.
 #include "common.cuh"
 #include "internal.h"
 #include "launch.cuh"
@@ -39,7 +41,7 @@ cache_write_kernel(Shape s, const T* __restrict__ K_new, const T* __restrict__ V
   const int b = bg / s.H_kv, g = bg % s.H_kv;
   const int tid = threadIdx.x, c = tid % TPR, rg = tid / TPR;
   const int st = start[b];
-  if (st < 0 || st + n_new > s.L_ctx) {
+  if (st < 0 || (long long)st + n_new > s.L_ctx) {  // 64-bit: start comes from device memory
     if (blockIdx.x == 0 && tid == 0) flag_error(err, ERR_BAD_INDEX);
     return;
   }

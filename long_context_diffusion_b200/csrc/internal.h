@@ -92,6 +92,7 @@ dl_status api_check_desc(const dl_attn_desc* d, Shape* s);
 dl_status api_error_word(unsigned** out);
 dl_status api_fail(dl_status st, const char* msg);
 dl_status api_ok();
+unsigned kernel_flags();  // dl_set_kernel_flags (DL_FLAG_*)
 
 __host__ __device__ inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 

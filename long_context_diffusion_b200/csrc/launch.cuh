@@ -13,30 +13,27 @@
 // so an early successor never takes resources this grid still needs; kernels
 // that allocate tensor memory trigger only after their allocation.
 // Measured inside a CUDA graph of the denoising step, PDL gave no gain (the
-// graph's launch gaps are already small), so it is opt-in: DL_PDL=1 in the
-// environment turns it on; otherwise kernels launch plainly and pdl_wait()
-// returns at once.
+// graph's launch gaps are already small), so it is opt-in: the DL_FLAG_PDL
+// kernel flag (dl_set_kernel_flags) turns it on; otherwise kernels launch
+// plainly and pdl_wait() returns at once.
 #pragma once
 
 #include <cuda_runtime.h>
 
-#include <cstdlib>
 #include <utility>
 
+#include "../../include/dl.h"
+
 namespace dl {
+
+unsigned kernel_flags();  // api.cu
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-inline bool pdl_enabled() {
-  static const bool on = [] {
-    const char* v = std::getenv("DL_PDL");
-    return v && v[0] && v[0] != '0';
-  }();
-  return on;
-}
+inline bool pdl_enabled() { return (kernel_flags() & DL_FLAG_PDL) != 0; }
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,

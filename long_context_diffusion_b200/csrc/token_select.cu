@@ -156,7 +156,7 @@ cudaError_t launch_token_select(const Shape& s, const void* Q, const void* Kp,
                                 const int32_t* page_table, const int32_t* chunk_idx, int n_sel,
                                 int chunk_stride, int chunk_content, int topT, int32_t* tok_pos,
                                 int32_t* tok_cnt, unsigned* err, cudaStream_t st) {
-  if (token_select_tc_supported(s, chunk_stride, chunk_content) && !getenv("DL_TOKEN_SIMT"))
+  if (token_select_tc_supported(s, chunk_stride, chunk_content) && !(kernel_flags() & DL_FLAG_TOKEN_SIMT))
     return launch_token_select_tc(s, Q, Kp, page_table, chunk_idx, n_sel, chunk_stride,
                                   chunk_content, topT, tok_pos, tok_cnt, err, st);
   dim3 grid(n_sel, s.batch * s.H_kv);

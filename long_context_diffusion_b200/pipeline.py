@@ -166,8 +166,16 @@ class DenoiseStep:
         self.lse = [_empty((B, H, L_q), torch.float32, device) for _ in range(n_layers)]
 
     def refresh_pooled_keys(self, layer: int, k_pool, page_table, Kbar, stream=None):
+        """Pooled keys of a whole layer, for a cache whose K rows were all
+        rewritten (built or recomputed)."""
         d = self.desc
         A.dl_pool_keys(d, k_pool, page_table, self.n_blk, d.page, 0, d.page, Kbar, stream)
+
+    def commit_block(self, k_new, v_new, start, k_pool, v_pool, page_table, Kbar, stream=None):
+        """A finished decode block joins one layer's cached context at
+        positions start[b] ..: written into the pools, the touched blocks'
+        pooled keys recomputed in the same pass (dl_cache_write)."""
+        A.dl_cache_write(self.desc, k_new, v_new, start, page_table, k_pool, v_pool, Kbar, stream)
 
     def run(self, conf_prev, still_masked, q_dec: List, k_pool: List, v_pool: List,
             page_table, k_dec: List, v_dec: List, Kbar: List, stream=None,

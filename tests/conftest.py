@@ -19,3 +19,18 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+@pytest.fixture
+def kernel_flags():
+    """Sets the library's kernel-choice flags for one test and restores the
+    previous ones afterwards."""
+    import long_context_diffusion_b200 as dl
+    saved = []
+
+    def set_flags(flags):
+        saved.append(dl.dl_set_kernel_flags(flags))
+
+    yield set_flags
+    if saved:
+        dl.dl_set_kernel_flags(saved[0])

@@ -108,3 +108,12 @@ def test_cache_write_arguments_rejected_before_launch():
     a[0] = ctypes.c_void_p(0x1008)  # K_new off the 16-byte grid
     assert lib.dl_cache_write(ctypes.byref(d), *a) == dl.DL_ERR_INVALID_ARG
     assert "aligned" in lib.dl_last_error_message().decode()
+
+
+def test_kernel_flags_round_trip():
+    prev = dl.dl_set_kernel_flags(dl.DL_FLAG_TOKEN_SIMT | dl.DL_FLAG_GATHER_SIMT)
+    try:
+        assert dl.dl_set_kernel_flags(0) == dl.DL_FLAG_TOKEN_SIMT | dl.DL_FLAG_GATHER_SIMT
+        assert dl.dl_set_kernel_flags(0) == 0
+    finally:
+        dl.dl_set_kernel_flags(prev)

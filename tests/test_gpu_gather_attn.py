@@ -31,9 +31,9 @@ SEED = 20261203
     (32, 32, 64, 128, [[2056] * 16 + [1000, 1, 0, 65] * 4]),
 ])
 @pytest.mark.parametrize("simt", [False, True])
-def test_gather_attention_matches_oracle(H, H_kv, L_q, d, cnts, simt, cuda_device, monkeypatch):
+def test_gather_attention_matches_oracle(H, H_kv, L_q, d, cnts, simt, cuda_device, kernel_flags):
     if simt:
-        monkeypatch.setenv("DL_GATHER_SIMT", "1")
+        kernel_flags(dl.DL_FLAG_GATHER_SIMT)
     batch, page, L_ctx = len(cnts), 64, 4096
     n_pages = L_ctx // page
     n_slots = batch * n_pages

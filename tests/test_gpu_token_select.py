@@ -32,9 +32,9 @@ SEED = 20261202
 ])
 @pytest.mark.parametrize("simt", [False, True])
 def test_token_select_matches_oracle(content, stride, H, H_kv, L_q, topT, n_sel, simt,
-                                     cuda_device, monkeypatch):
+                                     cuda_device, kernel_flags):
     if simt:
-        monkeypatch.setenv("DL_TOKEN_SIMT", "1")
+        kernel_flags(dl.DL_FLAG_TOKEN_SIMT)
     batch, d, page, n_chunks = 2, 128, 64, 3
     G = H // H_kv
     L_ctx = n_chunks * stride
