@@ -180,7 +180,8 @@ def cache_write_bytes(wl, start, n_new):
     e = 2
     j0, j1 = start // wl.B, (start + n_new - 1) // wl.B
     rows = sum(min(wl.B, wl.L_ctx - j * wl.B) for j in range(j0, j1 + 1))
-    per_bg = n_new * wl.d * e * 4 + (rows - n_new) * wl.d * e + (j1 - j0 + 1) * wl.d * 4
+    key_b = wl.d * 4 + wl.d * 5 + 4  # pooled key, its five digit planes, its exponent word
+    per_bg = n_new * wl.d * e * 4 + (rows - n_new) * wl.d * e + (j1 - j0 + 1) * key_b
     return wl.batch * wl.H_kv * per_bg
 
 
@@ -226,6 +227,7 @@ def workload_record(name, device, pk, reps=30):
     ws = pipeline.workspace(desc, device)
     n_units = wl.n_chunks if wl.chunked else wl.n_blk
     Kbar = torch.empty((wl.batch, wl.H_kv, n_units, wl.d), dtype=torch.float32, device=device)
+    Kdig = Kexp = None
     if wl.chunked:  # chunk keys belong to the cache build, not to the step
         dl.dl_pool_keys(desc, inp.k_pool, inp.page_table, wl.n_chunks, wl.chunk_stride, 1,
                         wl.chunk_content, Kbar)
@@ -237,15 +239,17 @@ def workload_record(name, device, pk, reps=30):
                                          topK_chunks=wl.topK_chunks, topT=wl.topT_tokens,
                                          Kbar=Kbar, ws=ws, stream=st)
     else:
-        dl.dl_pool_keys(desc, inp.k_pool, inp.page_table, wl.n_blk, wl.B, 0, wl.B, Kbar)
+        Kdig, Kexp = dl.key_digit_buffers(wl.batch, wl.H_kv, wl.n_blk, wl.d, device)
+        dl.dl_pool_keys(desc, inp.k_pool, inp.page_table, wl.n_blk, wl.B, 0, wl.B, Kbar,
+                        Kdig=Kdig, Kexp=Kexp)
         sinks = inp.sinks_planted[:, :wl.sinks_given].contiguous() if wl.sinks_given else None
 
         def fn(st):
             return pipeline.layer_step(desc, inp.q_dec, inp.k_pool, inp.v_pool, inp.page_table,
                                        inp.k_dec, inp.v_dec, topK=wl.topK,
                                        conf_prev=inp.conf_prev, still_masked=inp.still_masked,
-                                       k=wl.k, w=wl.w, sink_pos=sinks, Kbar=Kbar, ws=ws,
-                                       stream=st)
+                                       k=wl.k, w=wl.w, sink_pos=sinks, Kbar=Kbar, Kdig=Kdig,
+                                       Kexp=Kexp, ws=ws, stream=st)
     us, out = _graph_time_us(fn, device, reps)
     if dl.dl_get_status() != dl.DL_OK:
         raise RuntimeError(f"device status after the {name} step")
@@ -266,7 +270,11 @@ def workload_record(name, device, pk, reps=30):
             last = int((idx[r, :c] == wl.n_blk - 1).sum().item())
             toks += int(c) * wl.B - last * (wl.n_blk * wl.B - wl.L_ctx)
         ctx_tokens = toks / (wl.batch * wl.H_kv)
-        nbytes = (Kbar.numel() * 4 + q_b + wl.batch * wl.H_kv * wl.n_blk * 8 +
+        # the int8 tensor-core selection reads the digit planes; the fp64 one Kbar
+        fast = wl.dtype == "bf16" and wl.d == 128 and wl.G * min(wl.L_q, wl.k * (2 * wl.w + 1)) \
+            <= 32 and wl.n_blk <= 512
+        key_b = Kdig.numel() + Kexp.numel() * 4 if fast else Kbar.numel() * 4
+        nbytes = (key_b + q_b + wl.batch * wl.H_kv * wl.n_blk * 8 +
                   toks * wl.d * e * 2 + dec_b + o_b)
     t = us * 1e-6
     return {"workload": name, "us_per_step": us, "steps_per_s": 1.0 / t,
@@ -398,8 +406,7 @@ def run_ours(args):
     L = wl.n_layers
     step = pipeline.DenoiseStep(desc, L, wl.first_sparse_layer, wl.topK, wl.detect_sinks, wl.k,
                                 wl.w, torch.bfloat16, device)
-    Kbar = [torch.empty((wl.batch, wl.H_kv, wl.n_blk, wl.d), dtype=torch.float32,
-                        device=device) for _ in range(L)]
+    Kbar = [step.key_cache() for _ in range(L)]  # (pooled keys, digits, exponents) per layer
     stream = torch.cuda.Stream(device)
     args_of = lambda: (conf, masked, [x["q"] for x in layers], [x["kp"] for x in layers],  # noqa
                        [x["vp"] for x in layers], pt, [x["kd"] for x in layers],
@@ -445,6 +452,7 @@ def run_ours(args):
     ev1 = torch.cuda.Event(enable_timing=True)
     runtime.barrier(device)
     torch.cuda.synchronize(device)
+    dl.dl_read_counters()  # cleared: the counts below are the timed steps'
     with ClockSampler(local) as clk:
         with torch.cuda.stream(stream):
             ev0.record(stream)
@@ -452,6 +460,7 @@ def run_ours(args):
             ev1.record(stream)
         torch.cuda.synchronize(device)
     runtime.barrier(device)
+    sel_fast, sel_fallback = dl.dl_read_counters()
     ms_total = ev0.elapsed_time(ev1)
     ms_total = runtime.max_over_ranks(ms_total, device)
     ms_step = ms_total / K
@@ -501,7 +510,8 @@ def run_ours(args):
     # step-level roofline: algorithmic bytes of every kernel of one step
     e2b = 2
     cw_b = cache_write_bytes(wl, wl.L_ctx - wl.L_q, wl.L_q)
-    kbar_b = wl.batch * wl.H_kv * n_blk * wl.d * 4
+    # the selection reads the pooled keys as five int8 digit planes + one exponent word
+    kbar_b = wl.batch * wl.H_kv * n_blk * (wl.d * 5 + 4)
     q_b = wl.batch * wl.H * wl.L_q * wl.d * e2b
     # sink search: K counted once (the kernels stream it twice: the row LSEs
     # must be known before any column mass can be summed)
@@ -631,6 +641,8 @@ def run_ours(args):
         "clocks": clk.summary(),
         "e2e": e2e,
         "gpu_launches": launches_per_step * K,
+        "block_select_int8": {"certified": sel_fast, "fp64_fallback": sel_fallback,
+                              "per_step": (sel_fast + sel_fallback) / K},
         "gen_seconds": t_gen,
     }
     # cache refresh on the timed path: one decode block joining one layer
@@ -652,7 +664,7 @@ def run_ours(args):
             ts.append((a_, b_))
     torch.cuda.synchronize(device)
     pool_us = [a_.elapsed_time(b_) * 1e3 for a_, b_ in ts[1:]]
-    pool_b = wl.batch * wl.H_kv * (wl.L_ctx * wl.d * 2 + wl.n_blk * wl.d * 4)
+    pool_b = wl.batch * wl.H_kv * (wl.L_ctx * wl.d * 2 + wl.n_blk * (wl.d * 9 + 4))
     pm = sum(pool_us) / len(pool_us)
     line["full_layer_pool"] = {"call": "dl_pool_keys", "avg_us": pm, "bytes": pool_b,
                                "achieved_GBps": pool_b / (pm * 1e-6) / 1e9,

@@ -38,6 +38,8 @@ def main():
                     required=True)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--batch", type=int, default=4)
+    ap.add_argument("--fp64-select", action="store_true",
+                    help="dl_block_select on the fp64 kernel (DL_FLAG_SCORE_FP64)")
     args = ap.parse_args()
     dev = torch.device("cuda", 0)
     if args.case == "chunk_step":
@@ -57,7 +59,10 @@ def main():
     q_cnt = torch.empty((wl.batch,), dtype=torch.int32, device=dev)
     A.dl_predict_queries(conf, masked, wl.k, wl.w, q_idx, q_cnt)
     Kbar = torch.empty((wl.batch, wl.H_kv, wl.n_blk, wl.d), dtype=torch.float32, device=dev)
-    A.dl_pool_keys(desc, kp, pt, wl.n_blk, wl.B, 0, wl.B, Kbar)
+    Kdig, Kexp = A.key_digit_buffers(wl.batch, wl.H_kv, wl.n_blk, wl.d, dev)
+    A.dl_pool_keys(desc, kp, pt, wl.n_blk, wl.B, 0, wl.B, Kbar, Kdig=Kdig, Kexp=Kexp)
+    if args.fp64_select:
+        A.dl_set_kernel_flags(A.DL_FLAG_SCORE_FP64)
     sinks = torch.empty((wl.batch, wl.detect_sinks), dtype=torch.int32, device=dev)
     A.dl_find_sinks(desc, q, q_idx, q_cnt, kp, pt, kd, wl.detect_sinks, sinks, ws)
     max_sel = min(wl.topK, wl.n_blk) + wl.detect_sinks
@@ -71,7 +76,7 @@ def main():
 
     def block_select():
         A.dl_block_select(desc, q, q_idx, q_cnt, Kbar, wl.n_blk, wl.B, wl.topK, sinks, score,
-                          blk, cnt, ws, max_q=max_q)
+                          blk, cnt, ws, max_q=max_q, Kdig=Kdig, Kexp=Kexp)
 
     calls = {
         "block_select": block_select,
@@ -79,7 +84,8 @@ def main():
                                                 ws),
         "attn_dense": lambda: A.dl_sparse_attn(desc, q, kp, vp, pt, None, None, kd, vd, O, lse,
                                                ws),
-        "pool": lambda: A.dl_pool_keys(desc, kp, pt, wl.n_blk, wl.B, 0, wl.B, Kbar),
+        "pool": lambda: A.dl_pool_keys(desc, kp, pt, wl.n_blk, wl.B, 0, wl.B, Kbar, Kdig=Kdig,
+                                       Kexp=Kexp),
         "sinks": lambda: A.dl_find_sinks(desc, q, q_idx, q_cnt, kp, pt, kd, wl.detect_sinks,
                                          sinks, ws),
     }
@@ -87,6 +93,7 @@ def main():
         block_select()
     fn = calls[args.case]
     torch.cuda.synchronize()
+    A.dl_read_counters()
     times = []
     for _ in range(args.reps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -98,8 +105,10 @@ def main():
     st = A.dl_get_status()
     if st != A.DL_OK:
         raise RuntimeError(f"device status {st}")
+    fast, fallback = A.dl_read_counters()
     print(json.dumps({"case": args.case, "batch": wl.batch, "us_per_call": times,
-                      "mean_us_after_first": sum(times[1:]) / max(1, len(times) - 1)}))
+                      "mean_us_after_first": sum(times[1:]) / max(1, len(times) - 1),
+                      "int8_select_fast": fast, "int8_select_fallback": fallback}))
 
 
 def chunk_step(reps: int, dev):

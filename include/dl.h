@@ -91,6 +91,12 @@ enum { DL_FLAG_TOKEN_SIMT = 1u, DL_FLAG_GATHER_SIMT = 2u, DL_FLAG_PDL = 4u,
        DL_FLAG_SCORE_FP64 = 8u };
 unsigned dl_set_kernel_flags(unsigned flags);
 
+/* Counters of dl_block_select's int8 tensor-core kernel on the current
+ * device since the last call (then cleared): fast = (b, g) selections kept
+ * from the certified integer scores, fallback = (b, g) recomputed in fp64
+ * because the certificate did not hold.  Synchronises the device. */
+dl_status dl_read_counters(unsigned long long* fast, unsigned long long* fallback);
+
 /* Library version (major*10000 + minor*100 + patch). */
 int dl_version(void);
 
@@ -133,10 +139,21 @@ dl_status dl_predict_queries(const float* conf_prev, const uint8_t* still_masked
  * rounded once to fp32 (units with no valid token get 0).  Key blocks use
  * (stride, offset, len) = (page, 0, page); Prefilling-dLLM chunks [P1] with a
  * BOS anchor first use (chunk_stride, 1, chunk_content).
- *   K_pool  see layouts;  Kbar fp32 [batch][H_kv][n_units][d]  (out) */
+ *   K_pool  see layouts;  Kbar fp32 [batch][H_kv][n_units][d]  (out)
+ * Kdig/Kexp (both NULL, or both set): the same pooled keys also written as
+ * integer digits, the form dl_block_select's int8 tensor-core scoring reads
+ * (an implementation format; the pages describe no such thing):
+ *   Kdig int8  [batch][H_kv][5][n_units][d]  (out; 16-byte aligned)
+ *   Kexp int32 [batch][H_kv][n_units]        (out)
+ * With E the largest biased exponent field of the unit's d values (at least
+ * 1), every value x = sign * m * 2^(e - 150) is held as the integer
+ * V = trunc(m * 2^(11 - (E - e))), negated for x < 0, i.e. x~ = V * 2^(E-161),
+ * and V = d0*2^28 + d1*2^21 + d2*2^14 + d3*2^7 + d4 with d0 in [-128, 127]
+ * (plane 0) and d1..d4 in [0, 127] (planes 1..4).  Kexp = E | (number of the
+ * unit's values with x~ != x) << 8. */
 dl_status dl_pool_keys(const dl_attn_desc* desc, const void* K_pool, const int32_t* page_table,
                        int n_units, int unit_stride, int unit_offset, int unit_len,
-                       float* Kbar, void* stream);
+                       float* Kbar, int8_t* Kdig, int32_t* Kexp, void* stream);
 
 /* Cache refresh with the block pooling fused into the write.  [F2 summary:
  * the context is held in a KV cache; blocks are scored by their mean key]
@@ -159,10 +176,13 @@ dl_status dl_pool_keys(const dl_attn_desc* desc, const void* K_pool, const int32
  *   K_new, V_new  [batch][H_kv][n_new][d] (bf16/fp32, 16-byte aligned)
  *   start         int32 [batch] (device)
  *   K_pool, V_pool, page_table  see layouts (written / read)
- *   Kbar          fp32 [batch][H_kv][n_blk][d]  (touched blocks written) */
+ *   Kbar          fp32 [batch][H_kv][n_blk][d]  (touched blocks written)
+ *   Kdig, Kexp    NULL, or the digit form of Kbar as dl_pool_keys writes it
+ *                 (touched blocks rewritten, n_units = n_blk) */
 dl_status dl_cache_write(const dl_attn_desc* desc, const void* K_new, const void* V_new,
                          int n_new, const int32_t* start, const int32_t* page_table,
-                         void* K_pool, void* V_pool, float* Kbar, void* stream);
+                         void* K_pool, void* V_pool, float* Kbar, int8_t* Kdig, int32_t* Kexp,
+                         void* stream);
 
 /* (a3) Block scores with a fused block-level softmax.  [F2 summary]
  * For KV head g, rows r = (h in g's query heads, i in predicted positions):
@@ -205,23 +225,35 @@ dl_status dl_select(const double* score, int batch, int H_kv, int n_units, int u
 
 /* (a3 + a5) Block scores and selection in one call: the results of
  * dl_block_scores followed by dl_select with the same arguments (score is
- * written too), computed by one kernel per (b, g) when G * max_q <= 32 and
- * n_units <= 512 (the scores then stay on chip between the two steps;
- * bf16 or fp32 queries, d 64 or 128), otherwise by the two separate kernels.
- * [F2 summary: the predicted queries rank the blocks; F1 abstract: the sinks
- * are always kept]
+ * written too).  [F2 summary: the predicted queries rank the blocks; F1
+ * abstract: the sinks are always kept]
+ * Kernels, by shape:
+ *  - bf16 queries, d 128, G * max_q <= 32, n_units <= 512 and Kdig/Kexp given
+ *    (the digits of these very Kbar, from dl_pool_keys / dl_cache_write):
+ *    one CTA per (b, g) takes the logits q . Kbar exactly on the int8 tensor
+ *    cores (query digits times key digits, int32 sums), in fp64 from there
+ *    on, with a proven bound on each logit's error (the truncated digits);
+ *    the selection is kept when the gap between the K-th and (K+1)-th score
+ *    exceeds the bound, and otherwise that (b, g) is recomputed by the fp64
+ *    kernel below inside the same CTA.  The selected blocks are then those of
+ *    the exact scores; score holds values within a relative 1e-9 of them.
+ *  - otherwise, G * max_q <= 32 and n_units <= 512: one kernel per (b, g)
+ *    computing the scores in fp64 (the scores then stay on chip between the
+ *    two steps; bf16 or fp32 queries, d 64 or 128);
+ *  - otherwise the two separate kernels.
  * max_q: an upper bound of q_cnt[b] that the caller guarantees (with the
  *   prediction of dl_predict_queries: min(L_q, k * (2w + 1))); 0 = L_q.  The
- *   fused kernel is compiled for that many rows; a sequence with more rows
+ *   fused kernels are compiled for that many rows; a sequence with more rows
  *   is cut to the bound and reported as DL_ERR_BAD_INDEX by dl_get_status.
  * Other arguments, layouts and requirements as for dl_block_scores and
  * dl_select; ws: workspace of dl_workspace_size (used only by the separate
  * kernels). */
 dl_status dl_block_select(const dl_attn_desc* desc, const void* Q_dec, const int32_t* q_idx,
-                          const int32_t* q_cnt, const float* Kbar, int n_units, int unit_size,
-                          int topK, const int32_t* sink_pos, int n_sinks, double* score,
-                          int32_t* blk_idx, int32_t* blk_cnt, int max_sel, int max_q, void* ws,
-                          size_t ws_bytes, void* stream);
+                          const int32_t* q_cnt, const float* Kbar, const int8_t* Kdig,
+                          const int32_t* Kexp, int n_units, int unit_size, int topK,
+                          const int32_t* sink_pos, int n_sinks, double* score, int32_t* blk_idx,
+                          int32_t* blk_cnt, int max_sel, int max_q, void* ws, size_t ws_bytes,
+                          void* stream);
 
 /* (a6) Block-sparse bidirectional attention.  [F1 abstract; F2 summary]
  * For every query head h (KV head g) and decode position i:

@@ -47,18 +47,19 @@ _SIGS = {
     "dl_workspace_size": ([ctypes.POINTER(dl_attn_desc), ctypes.POINTER(ctypes.c_size_t)], _c_int),
     "dl_predict_queries": ([_vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
     "dl_pool_keys": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _c_int, _c_int, _c_int, _c_int,
-                      _vp, _vp], _c_int),
+                      _vp, _vp, _vp, _vp], _c_int),
     "dl_cache_write": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp,
-                        _vp], _c_int),
+                        _vp, _vp, _vp], _c_int),
     "dl_block_scores": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _c_int, _vp, _vp,
                          ctypes.c_size_t, _vp], _c_int),
     "dl_find_sinks": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp,
                        _vp, ctypes.c_size_t, _vp], _c_int),
     "dl_select": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _vp, _c_int,
                    _vp], _c_int),
-    "dl_block_select": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _c_int, _c_int,
-                         _c_int, _vp, _c_int, _vp, _vp, _vp, _c_int, _c_int, _vp,
+    "dl_block_select": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _vp, _vp, _c_int,
+                         _c_int, _c_int, _vp, _c_int, _vp, _vp, _vp, _c_int, _c_int, _vp,
                          ctypes.c_size_t, _vp], _c_int),
+    "dl_read_counters": ([_vp, _vp], _c_int),
     "dl_sparse_attn": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp,
                         _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp], _c_int),
     "dl_token_select": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _c_int, _c_int,
@@ -139,15 +140,30 @@ def dl_predict_queries(conf_prev, still_masked, k, w, q_idx, q_cnt, stream=None)
 
 
 def dl_pool_keys(desc, K_pool, page_table, n_units, unit_stride, unit_offset, unit_len, Kbar,
-                 stream=None):
+                 stream=None, Kdig=None, Kexp=None):
     _check(lib.dl_pool_keys(ctypes.byref(desc), _p(K_pool), _p(page_table), n_units, unit_stride,
-                            unit_offset, unit_len, _p(Kbar), _s(stream)))
+                            unit_offset, unit_len, _p(Kbar), _p(Kdig), _p(Kexp), _s(stream)))
 
 
-def dl_cache_write(desc, K_new, V_new, start, page_table, K_pool, V_pool, Kbar, stream=None):
+def dl_cache_write(desc, K_new, V_new, start, page_table, K_pool, V_pool, Kbar, stream=None,
+                   Kdig=None, Kexp=None):
     _check(lib.dl_cache_write(ctypes.byref(desc), _p(K_new), _p(V_new), K_new.shape[-2],
                               _p(start), _p(page_table), _p(K_pool), _p(V_pool), _p(Kbar),
-                              _s(stream)))
+                              _p(Kdig), _p(Kexp), _s(stream)))
+
+
+def key_digit_buffers(batch, H_kv, n_units, d, device):
+    """Allocates the Kdig / Kexp buffers of dl_pool_keys' digit output."""
+    return (torch.empty((batch, H_kv, 5, n_units, d), dtype=torch.int8, device=device),
+            torch.empty((batch, H_kv, n_units), dtype=torch.int32, device=device))
+
+
+def dl_read_counters():
+    """(fast, fallback) selections of dl_block_select's int8 kernel since the
+    last read."""
+    f, b = ctypes.c_ulonglong(0), ctypes.c_ulonglong(0)
+    _check(lib.dl_read_counters(ctypes.byref(f), ctypes.byref(b)))
+    return int(f.value), int(b.value)
 
 
 def dl_block_scores(desc, Q_dec, q_idx, q_cnt, Kbar, n_units, score, ws, stream=None):
@@ -171,10 +187,11 @@ def dl_select(score, unit_size, topK, sink_pos, blk_idx, blk_cnt, stream=None):
 
 
 def dl_block_select(desc, Q_dec, q_idx, q_cnt, Kbar, n_units, unit_size, topK, sink_pos, score,
-                    blk_idx, blk_cnt, ws, stream=None, max_q=0):
+                    blk_idx, blk_cnt, ws, stream=None, max_q=0, Kdig=None, Kexp=None):
     n_sinks = 0 if sink_pos is None else sink_pos.shape[-1]
     _check(lib.dl_block_select(ctypes.byref(desc), _p(Q_dec), _p(q_idx), _p(q_cnt), _p(Kbar),
-                               n_units, unit_size, topK, _p(sink_pos), n_sinks, _p(score),
+                               _p(Kdig), _p(Kexp), n_units, unit_size, topK, _p(sink_pos),
+                               n_sinks, _p(score),
                                _p(blk_idx), _p(blk_cnt), blk_idx.shape[-1], max_q, _p(ws),
                                ws.numel() * ws.element_size(), _s(stream)))
 

@@ -126,6 +126,14 @@ int dl_version(void) { return 200; }
 
 unsigned dl_set_kernel_flags(unsigned flags) { return g_kernel_flags.exchange(flags); }
 
+dl_status dl_read_counters(unsigned long long* fast, unsigned long long* fallback) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  if ((e = dl::read_select_counts(fast, fallback)) != cudaSuccess)
+    return cuda_fail(e, "dl_read_counters");
+  return ok();
+}
+
 const char* dl_last_error_message(void) { return g_msg; }
 
 dl_status dl_get_status(void* stream) {
@@ -176,11 +184,14 @@ dl_status dl_predict_queries(const float* conf_prev, const uint8_t* still_masked
 
 dl_status dl_pool_keys(const dl_attn_desc* desc, const void* K_pool, const int32_t* page_table,
                        int n_units, int unit_stride, int unit_offset, int unit_len, float* Kbar,
-                       void* stream) {
+                       int8_t* Kdig, int32_t* Kexp, void* stream) {
   dl::Shape s;
   dl_status st = check_desc(desc, &s);
   if (st != DL_OK) return st;
   if (!K_pool || !page_table || !Kbar) return fail(DL_ERR_INVALID_ARG, "dl_pool_keys: NULL pointer");
+  if ((Kdig == nullptr) != (Kexp == nullptr))
+    return fail(DL_ERR_INVALID_ARG, "dl_pool_keys: Kdig and Kexp go together");
+  if (Kdig && !aligned16(Kdig)) return fail(DL_ERR_INVALID_ARG, "Kdig not 16-byte aligned");
   if (!aligned16(K_pool)) return fail(DL_ERR_INVALID_ARG, "K_pool not 16-byte aligned");
   if (n_units < 1 || n_units > (1 << 24)) return fail(DL_ERR_INVALID_ARG, "n_units=%d", n_units);
   if (unit_stride < 1 || unit_offset < 0 || unit_len < 1)
@@ -189,18 +200,21 @@ dl_status dl_pool_keys(const dl_attn_desc* desc, const void* K_pool, const int32
   unsigned* err = nullptr;
   if ((st = error_word(&err)) != DL_OK) return st;
   return launched(dl::launch_pool(s, K_pool, page_table, n_units, unit_stride, unit_offset,
-                                  unit_len, Kbar, err, as_stream(stream)),
+                                  unit_len, Kbar, Kdig, Kexp, err, as_stream(stream)),
                   "dl_pool_keys launch");
 }
 
 dl_status dl_cache_write(const dl_attn_desc* desc, const void* K_new, const void* V_new,
                          int n_new, const int32_t* start, const int32_t* page_table,
-                         void* K_pool, void* V_pool, float* Kbar, void* stream) {
+                         void* K_pool, void* V_pool, float* Kbar, int8_t* Kdig, int32_t* Kexp,
+                         void* stream) {
   dl::Shape s;
   dl_status st = check_desc(desc, &s);
   if (st != DL_OK) return st;
   if (!K_new || !V_new || !start || !page_table || !K_pool || !V_pool || !Kbar)
     return fail(DL_ERR_INVALID_ARG, "dl_cache_write: NULL pointer");
+  if ((Kdig == nullptr) != (Kexp == nullptr))
+    return fail(DL_ERR_INVALID_ARG, "dl_cache_write: Kdig and Kexp go together");
   if (!aligned16(K_new) || !aligned16(V_new) || !aligned16(K_pool) || !aligned16(V_pool))
     return fail(DL_ERR_INVALID_ARG, "dl_cache_write: K/V buffers must be 16-byte aligned");
   if (n_new < 1 || n_new > s.L_ctx)
@@ -208,7 +222,7 @@ dl_status dl_cache_write(const dl_attn_desc* desc, const void* K_new, const void
   unsigned* err = nullptr;
   if ((st = error_word(&err)) != DL_OK) return st;
   return launched(dl::launch_cache_write(s, K_new, V_new, n_new, start, page_table, K_pool,
-                                         V_pool, Kbar, err, as_stream(stream)),
+                                         V_pool, Kbar, Kdig, Kexp, err, as_stream(stream)),
                   "dl_cache_write launch");
 }
 
@@ -273,7 +287,8 @@ dl_status dl_select(const double* score, int batch, int H_kv, int n_units, int u
 }
 
 dl_status dl_block_select(const dl_attn_desc* desc, const void* Q_dec, const int32_t* q_idx,
-                          const int32_t* q_cnt, const float* Kbar, int n_units, int unit_size,
+                          const int32_t* q_cnt, const float* Kbar, const int8_t* Kdig,
+                          const int32_t* Kexp, int n_units, int unit_size,
                           int topK, const int32_t* sink_pos, int n_sinks, double* score,
                           int32_t* blk_idx, int32_t* blk_cnt, int max_sel, int max_q, void* ws,
                           size_t ws_bytes, void* stream) {
@@ -283,6 +298,11 @@ dl_status dl_block_select(const dl_attn_desc* desc, const void* Q_dec, const int
   if (!Q_dec || !Kbar || !score || (q_idx && !q_cnt) || !blk_idx || !blk_cnt ||
       (n_sinks > 0 && !sink_pos))
     return fail(DL_ERR_INVALID_ARG, "dl_block_select: NULL pointer");
+  if ((Kdig == nullptr) != (Kexp == nullptr))
+    return fail(DL_ERR_INVALID_ARG, "dl_block_select: Kdig and Kexp go together");
+  if (Kdig && !aligned16(Kdig)) return fail(DL_ERR_INVALID_ARG, "Kdig not 16-byte aligned");
+  if (!aligned16(Q_dec) || !aligned16(Kbar))
+    return fail(DL_ERR_INVALID_ARG, "dl_block_select: Q_dec and Kbar must be 16-byte aligned");
   if (n_units < 1 || n_units > 16384)
     return fail(DL_ERR_INVALID_ARG, "n_units=%d (need 1..16384)", n_units);
   if (unit_size < 1 || topK < 0 || n_sinks < 0 || n_sinks > 1024)
@@ -294,7 +314,7 @@ dl_status dl_block_select(const dl_attn_desc* desc, const void* Q_dec, const int
   if ((st = need_ws(ws, ws_bytes, dl::scores_workspace(s, n_units))) != DL_OK) return st;
   unsigned* err = nullptr;
   if ((st = error_word(&err)) != DL_OK) return st;
-  return launched(dl::launch_block_select(s, Q_dec, q_idx, q_cnt, Kbar, n_units, score,
+  return launched(dl::launch_block_select(s, Q_dec, q_idx, q_cnt, Kbar, Kdig, Kexp, n_units, score,
                                           unit_size, topK, sink_pos, n_sinks, blk_idx, blk_cnt,
                                           max_sel, max_q, ws, err, as_stream(stream)),
                   "dl_block_select launch");

@@ -730,6 +730,20 @@ bool tc_map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t L_q, u
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// int8 planes of `inner` bytes x rows, stacked `planes` deep; boxes of
+// inner x box_rows x 1, 128-byte swizzle (inner must be 128).
+bool tc_map_i8_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                  uint64_t planes, uint32_t box_rows) {
+  EncodeTiled fn = encoder();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, rows, planes};
+  cuuint64_t strides[2] = {inner, rows * inner};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(inner), box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 int tc_sm_count() {
   int dev = 0, n = 148;

@@ -12,12 +12,14 @@
 // column chunk): its rows of the block, new ones copied from K_new/V_new into
 // the pools, old ones read from the K pool, summed in fp64; the row groups'
 // sums are added in shared memory and the mean over the block's positions
-// below L_ctx is rounded once to fp32.  For bf16 keys the fp64 sum is exact,
+// below L_ctx is rounded once to fp32 (and, when asked, also written as the
+// integer digits of kdigits.cuh).  For bf16 keys the fp64 sum is exact,
 // so the result equals dl_pool_keys bit for bit whatever the order; for fp32
 // keys the fp64 sum is exact only while the 64 values' exponents are close,
 // and the pooled key can then differ from dl_pool_keys' by one fp32 ulp.
 #include "common.cuh"
 #include "internal.h"
+#include "kdigits.cuh"
 #include "launch.cuh"
 
 namespace dl {
@@ -29,7 +31,7 @@ __global__ void __launch_bounds__(kCwThreads)
 cache_write_kernel(Shape s, const T* __restrict__ K_new, const T* __restrict__ V_new, int n_new,
                    const int32_t* __restrict__ start, const int32_t* __restrict__ page_table,
                    T* __restrict__ Kp, T* __restrict__ Vp, float* __restrict__ Kbar,
-                   unsigned* err) {
+                   int8_t* __restrict__ Kdig, int32_t* __restrict__ Kexp, unsigned* err) {
   pdl_trigger();
   pdl_wait();
   constexpr int EPT = Vec16<T>::N;       // elements per 16-byte chunk
@@ -91,23 +93,55 @@ cache_write_kernel(Shape s, const T* __restrict__ K_new, const T* __restrict__ V
 #pragma unroll
   for (int e = 0; e < EPT; ++e) s_sum[rg][c * EPT + e] = acc[e];
   __syncthreads();
+  const int n_blk = (s.L_ctx + B - 1) / B;
+  float mean = 0.0f;
   if (tid < D) {
     double sum = 0.0;
     for (int q = 0; q < RG; ++q) sum += s_sum[q][tid];
     const int n = min(B, s.L_ctx - j * B);
-    const int n_blk = (s.L_ctx + B - 1) / B;
-    Kbar[((size_t)bg * n_blk + j) * D + tid] = __double2float_rn(sum / (double)n);
+    mean = __double2float_rn(sum / (double)n);
+    Kbar[((size_t)bg * n_blk + j) * D + tid] = mean;
+  }
+  if (Kdig == nullptr) return;  // uniform over the grid
+  // the block's pooled key as integer digits (kdigits.cuh): row exponent and
+  // inexact count over the D threads of the first D / 32 warps
+  __shared__ int s_e[kCwThreads / 32], s_n[kCwThreads / 32];
+  const int warp = tid >> 5, lane = tid & 31;
+  int E = tid < D ? exp_field_f32(mean) : 1;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) E = max(E, __shfl_xor_sync(0xffffffffu, E, o));
+  if (lane == 0) s_e[warp] = E;
+  __syncthreads();
+  E = 1;
+  for (int w = 0; w < D / 32; ++w) E = max(E, s_e[w]);
+  int dg[kKeyDigits];
+  int inexact = (tid < D && key_digits(mean, E, dg)) ? 1 : 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) inexact += __shfl_xor_sync(0xffffffffu, inexact, o);
+  if (lane == 0) s_n[warp] = inexact;
+  __syncthreads();
+  if (tid < D) {
+#pragma unroll
+    for (int t = 0; t < kKeyDigits; ++t)
+      Kdig[(((size_t)bg * kKeyDigits + t) * n_blk + j) * D + tid] = (int8_t)dg[t];
+  }
+  if (tid == 0) {
+    int n = 0;
+    for (int w = 0; w < D / 32; ++w) n += s_n[w];
+    Kexp[(size_t)bg * n_blk + j] = E | (n << 8);
   }
 }
 
 cudaError_t launch_cache_write(const Shape& s, const void* K_new, const void* V_new, int n_new,
                                const int32_t* start, const int32_t* page_table, void* Kp,
-                               void* Vp, float* Kbar, unsigned* err, cudaStream_t st) {
+                               void* Vp, float* Kbar, int8_t* Kdig, int32_t* Kexp, unsigned* err,
+                               cudaStream_t st) {
   dim3 grid((n_new + 63) / 64 + 1, s.batch * s.H_kv);
 #define DL_CACHE_WRITE(T, D_)                                                                  \
   DL_LAUNCH(cache_write_kernel<T, D_>, grid, kCwThreads, 0, st, s,                             \
             reinterpret_cast<const T*>(K_new), reinterpret_cast<const T*>(V_new), n_new,      \
-            start, page_table, reinterpret_cast<T*>(Kp), reinterpret_cast<T*>(Vp), Kbar, err)
+            start, page_table, reinterpret_cast<T*>(Kp), reinterpret_cast<T*>(Vp), Kbar, Kdig,   \
+            Kexp, err)
   if (s.dtype == 0) {
     if (s.d == 128) DL_CACHE_WRITE(__nv_bfloat16, 128); else DL_CACHE_WRITE(__nv_bfloat16, 64);
   } else {

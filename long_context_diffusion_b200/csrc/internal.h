@@ -56,8 +56,8 @@ cudaError_t launch_predict(const float* conf, const uint8_t* masked, int batch, 
                            int w, int32_t* q_idx, int32_t* q_cnt, cudaStream_t st);
 
 cudaError_t launch_pool(const Shape& s, const void* Kp, const int32_t* page_table, int n_units,
-                        int stride, int offset, int len, float* Kbar, unsigned* err,
-                        cudaStream_t st);
+                        int stride, int offset, int len, float* Kbar, int8_t* Kdig,
+                        int32_t* Kexp, unsigned* err, cudaStream_t st);
 
 cudaError_t launch_scores(const Shape& s, const void* Q, const int32_t* q_idx,
                           const int32_t* q_cnt, const float* Kbar, int n_units, double* score,
@@ -67,10 +67,20 @@ cudaError_t launch_select(const double* score, int batch, int H_kv, int n_units,
                           int topK, const int32_t* sink_pos, int n_sinks, int32_t* blk_idx,
                           int32_t* blk_cnt, int max_sel, unsigned* err, cudaStream_t st);
 cudaError_t launch_block_select(const Shape& s, const void* Q, const int32_t* q_idx,
-                                const int32_t* q_cnt, const float* Kbar, int n_units,
-                                double* score, int unit_size, int topK, const int32_t* sink_pos,
-                                int n_sinks, int32_t* blk_idx, int32_t* blk_cnt, int max_sel,
-                                int max_q, void* ws, unsigned* err, cudaStream_t st);
+                                const int32_t* q_cnt, const float* Kbar, const int8_t* Kdig,
+                                const int32_t* Kexp, int n_units, double* score, int unit_size,
+                                int topK, const int32_t* sink_pos, int n_sinks, int32_t* blk_idx,
+                                int32_t* blk_cnt, int max_sel, int max_q, void* ws,
+                                unsigned* err, cudaStream_t st);
+
+bool block_select_tc_supported(const Shape& s, int rows, int n_units);
+cudaError_t launch_block_select_tc(const Shape& s, const void* Q, const int32_t* q_idx,
+                                   const int32_t* q_cnt, const float* Kbar, const int8_t* Kdig,
+                                   const int32_t* Kexp, int n_units, double* score,
+                                   int unit_size, int topK, const int32_t* sink_pos,
+                                   int n_sinks, int32_t* blk_idx, int32_t* blk_cnt, int max_sel,
+                                   int rows, unsigned* err, cudaStream_t st);
+cudaError_t read_select_counts(unsigned long long* fast, unsigned long long* fallback);
 
 cudaError_t launch_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
                          const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
@@ -81,7 +91,8 @@ cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
 
 cudaError_t launch_cache_write(const Shape& s, const void* K_new, const void* V_new, int n_new,
                                const int32_t* start, const int32_t* page_table, void* Kp,
-                               void* Vp, float* Kbar, unsigned* err, cudaStream_t st);
+                               void* Vp, float* Kbar, int8_t* Kdig, int32_t* Kexp, unsigned* err,
+                               cudaStream_t st);
 cudaError_t launch_token_select(const Shape& s, const void* Q, const void* Kp,
                                 const int32_t* page_table, const int32_t* chunk_idx, int n_sel,
                                 int chunk_stride, int chunk_content, int topT, int32_t* tok_pos,

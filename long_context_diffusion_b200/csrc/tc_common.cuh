@@ -79,6 +79,10 @@ __device__ __forceinline__ int2 tc_tile_info(const AttnArgs& a, int bg, int tile
 bool tc_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows);
 // decode block K/V: [bg][L_q][d], boxes of 64 x 64 x 1 (rows past L_q read 0)
 bool tc_map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t L_q, uint64_t n_bg);
+// int8 planes [planes][rows][inner] (inner = 128 bytes), boxes of
+// inner x box_rows x 1, 128-byte swizzle.
+bool tc_map_i8_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                  uint64_t planes, uint32_t box_rows);
 int tc_sm_count();
 
 struct TcLaunch {

@@ -48,11 +48,13 @@ class LayerOutputs:
 def layer_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec, v_dec, *,
                topK: int, conf_prev=None, still_masked=None, k: int = 4, w: int = 2,
                q_idx=None, q_cnt=None, sink_pos=None, detect_sinks: int = 0,
-               dense: bool = False, Kbar=None, ws=None, stream=None,
+               dense: bool = False, Kbar=None, Kdig=None, Kexp=None, ws=None, stream=None,
                fused_select: bool = True) -> LayerOutputs:
     """One layer for a batch: (predict,) pool, (find sinks,) score and select
     (one call, or dl_block_scores then dl_select when fused_select is False),
-    attend -- or dense attention.  Mirrors the oracle's layer_step."""
+    attend -- or dense attention.  Mirrors the oracle's layer_step.  When the
+    layer pools its own keys it also writes their integer digits (Kdig, Kexp),
+    which the selection then reads; a caller passing Kbar may pass them too."""
     dev = q_dec.device
     B, L_q, d, H, H_kv = desc.batch, desc.L_q, desc.d, desc.H, desc.H_kv
     n_blk = -(-desc.L_ctx // desc.page)
@@ -70,7 +72,9 @@ def layer_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec, v
         return LayerOutputs(q_idx, q_cnt, None, None, sink_pos, None, None, O, lse)
     if Kbar is None:
         Kbar = _empty((B, H_kv, n_blk, d), torch.float32, dev)
-        A.dl_pool_keys(desc, k_pool, page_table, n_blk, desc.page, 0, desc.page, Kbar, stream)
+        Kdig, Kexp = A.key_digit_buffers(B, H_kv, n_blk, d, dev)
+        A.dl_pool_keys(desc, k_pool, page_table, n_blk, desc.page, 0, desc.page, Kbar, stream,
+                       Kdig=Kdig, Kexp=Kexp)
     score = _empty((B, H_kv, n_blk), torch.float64, dev)
     if detect_sinks:
         sink_pos = _empty((B, detect_sinks), torch.int32, dev)
@@ -84,7 +88,7 @@ def layer_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec, v
         # rows per sequence: the prediction gives at most k windows of 2w+1
         max_q = min(L_q, k * (2 * w + 1)) if conf_prev is not None else 0
         A.dl_block_select(desc, q_dec, q_idx, q_cnt, Kbar, n_blk, desc.page, topK, sink_pos,
-                          score, blk_idx, blk_cnt, ws, stream, max_q=max_q)
+                          score, blk_idx, blk_cnt, ws, stream, max_q=max_q, Kdig=Kdig, Kexp=Kexp)
     else:
         A.dl_block_scores(desc, q_dec, q_idx, q_cnt, Kbar, n_blk, score, ws, stream)
         A.dl_select(score, desc.page, topK, sink_pos, blk_idx, blk_cnt, stream)
@@ -165,23 +169,33 @@ class DenoiseStep:
         self.O = [_empty((B, L_q, H, d), dtype, device) for _ in range(n_layers)]
         self.lse = [_empty((B, H, L_q), torch.float32, device) for _ in range(n_layers)]
 
-    def refresh_pooled_keys(self, layer: int, k_pool, page_table, Kbar, stream=None):
-        """Pooled keys of a whole layer, for a cache whose K rows were all
-        rewritten (built or recomputed)."""
-        d = self.desc
-        A.dl_pool_keys(d, k_pool, page_table, self.n_blk, d.page, 0, d.page, Kbar, stream)
+    def key_cache(self):
+        """Pooled keys of one layer with their integer digits: (Kbar, Kdig,
+        Kexp), to be filled by refresh_pooled_keys / commit_block."""
+        dsc = self.desc
+        Kbar = _empty((dsc.batch, dsc.H_kv, self.n_blk, dsc.d), torch.float32, self.device)
+        return (Kbar, *A.key_digit_buffers(dsc.batch, dsc.H_kv, self.n_blk, dsc.d, self.device))
 
-    def commit_block(self, k_new, v_new, start, k_pool, v_pool, page_table, Kbar, stream=None):
+    def refresh_pooled_keys(self, layer: int, k_pool, page_table, kc, stream=None):
+        """Pooled keys (and digits) of a whole layer, for a cache whose K rows
+        were all rewritten (built or recomputed).  kc = key_cache()."""
+        d = self.desc
+        A.dl_pool_keys(d, k_pool, page_table, self.n_blk, d.page, 0, d.page, kc[0], stream,
+                       Kdig=kc[1], Kexp=kc[2])
+
+    def commit_block(self, k_new, v_new, start, k_pool, v_pool, page_table, kc, stream=None):
         """A finished decode block joins one layer's cached context at
         positions start[b] ..: written into the pools, the touched blocks'
-        pooled keys recomputed in the same pass (dl_cache_write)."""
-        A.dl_cache_write(self.desc, k_new, v_new, start, page_table, k_pool, v_pool, Kbar, stream)
+        pooled keys (and digits) recomputed in the same pass (dl_cache_write)."""
+        A.dl_cache_write(self.desc, k_new, v_new, start, page_table, k_pool, v_pool, kc[0], stream,
+                         Kdig=kc[1], Kexp=kc[2])
 
     def run(self, conf_prev, still_masked, q_dec: List, k_pool: List, v_pool: List,
-            page_table, k_dec: List, v_dec: List, Kbar: List, stream=None,
+            page_table, k_dec: List, v_dec: List, key_caches: List, stream=None,
             attn_events: Optional[list] = None):
-        """Launches the step on `stream`.  If attn_events is a list, a pair of
-        timing events (recorded as graph nodes when captured) brackets every
+        """Launches the step on `stream`.  key_caches[l] = (Kbar, Kdig, Kexp)
+        of layer l (key_cache()).  If attn_events is a list, a pair of timing
+        events (recorded as graph nodes when captured) brackets every
         attention call and (layer, start, end) is appended to it."""
         d = self.desc
         A.dl_predict_queries(conf_prev, still_masked, self.k, self.w, self.q_idx, self.q_cnt,
@@ -196,9 +210,11 @@ class DenoiseStep:
             if l == self.first_sparse:
                 A.dl_find_sinks(d, q_dec[l], self.q_idx, self.q_cnt, k_pool[l], page_table,
                                 k_dec[l], self.n_sinks, self.sink_pos, self.ws, stream)
-            A.dl_block_select(d, q_dec[l], self.q_idx, self.q_cnt, Kbar[l], self.n_blk, d.page,
+            Kbar, Kdig, Kexp = key_caches[l]
+            A.dl_block_select(d, q_dec[l], self.q_idx, self.q_cnt, Kbar, self.n_blk, d.page,
                               self.topK, self.sink_pos, self.score, self.blk_idx[l],
-                              self.blk_cnt[l], self.ws, stream, max_q=self.max_q)
+                              self.blk_cnt[l], self.ws, stream, max_q=self.max_q, Kdig=Kdig,
+                              Kexp=Kexp)
             ev = self._begin(attn_events, stream)
             A.dl_sparse_attn(d, q_dec[l], k_pool[l], v_pool[l], page_table, self.blk_idx[l],
                              self.blk_cnt[l], k_dec[l], v_dec[l], self.O[l], self.lse[l],

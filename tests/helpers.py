@@ -51,3 +51,29 @@ def cut_margin(values, kept, excluded=()):
     if len(a) == 0 or len(b) == 0:
         return float("inf")
     return float(a.min() - b.max())
+
+
+def key_digits_np(kbar):
+    """The integer-digit form of fp32 pooled keys [..., d] that dl_pool_keys
+    documents (include/dl.h): per row the largest exponent field E (at least
+    1), every value as V = trunc(m * 2^(11 - (E - e))), negated when negative,
+    written base 128 with a signed top digit.  Returns (Kdig [..., 5, d] moved
+    to the plane axis by the caller, Kexp [...]) as int8 / int32 arrays with
+    the digit plane as the second-to-last axis."""
+    x = np.ascontiguousarray(np.asarray(kbar, dtype=np.float32))
+    u = x.view(np.uint32).astype(np.int64)
+    sign = (u >> 31) & 1
+    e = (u >> 23) & 0xFF
+    mant = u & 0x7FFFFF
+    m = np.where(e == 0, mant, mant | 0x800000)
+    ee = np.maximum(e, 1)
+    E = ee.max(axis=-1, keepdims=True)
+    sh = E - ee
+    v0 = m << 11
+    v = np.where(sh < 63, v0 >> np.minimum(sh, 62), 0)
+    inexact = (m != 0) & ((sh >= 63) | ((v << np.minimum(sh, 62)) != v0))
+    sv = np.where(sign == 1, -v, v)
+    digs = [sv >> 28] + [(sv >> (7 * (4 - t))) & 127 for t in range(1, 5)]
+    kdig = np.stack(digs, axis=-2).astype(np.int8)   # [..., 5, d]
+    kexp = (E[..., 0] | (inexact.sum(axis=-1) << 8)).astype(np.int32)
+    return kdig, kexp

@@ -69,15 +69,29 @@ def test_null_and_range_arguments_rejected_before_launch():
         dl.DL_ERR_INVALID_ARG
     assert "max_sel" in lib.dl_last_error_message().decode()
     # fused scores + selection: the same checks before any launch
-    assert lib.dl_block_select(ctypes.byref(d), fake, None, None, None, 256, 64, 4, None, 0,
-                               fake, fake, fake, 4, 0, fake, 1 << 40, None) == dl.DL_ERR_INVALID_ARG
-    assert lib.dl_block_select(ctypes.byref(d), fake, None, None, fake, 256, 64, 4, fake, 2,
-                               fake, fake, fake, 5, 0, fake, 1 << 40, None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_block_select(ctypes.byref(d), fake, None, None, None, None, None, 256, 64, 4,
+                               None, 0, fake, fake, fake, 4, 0, fake, 1 << 40,
+                               None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_block_select(ctypes.byref(d), fake, None, None, fake, None, None, 256, 64, 4,
+                               fake, 2, fake, fake, fake, 5, 0, fake, 1 << 40,
+                               None) == dl.DL_ERR_INVALID_ARG
     assert "max_sel" in lib.dl_last_error_message().decode()
-    assert lib.dl_block_select(ctypes.byref(d), fake, None, None, fake, 256, 64, 4, None, 0,
-                               fake, fake, fake, 4, -1, fake, 1 << 40, None) == dl.DL_ERR_INVALID_ARG
-    assert lib.dl_block_select(ctypes.byref(d), fake, None, None, fake, 256, 64, 4, None, 0,
-                               fake, fake, fake, 4, 0, fake, 256, None) == dl.DL_ERR_WORKSPACE
+    assert lib.dl_block_select(ctypes.byref(d), fake, None, None, fake, None, None, 256, 64, 4,
+                               None, 0, fake, fake, fake, 4, -1, fake, 1 << 40,
+                               None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_block_select(ctypes.byref(d), fake, None, None, fake, None, None, 256, 64, 4,
+                               None, 0, fake, fake, fake, 4, 0, fake, 256,
+                               None) == dl.DL_ERR_WORKSPACE
+    # key digits: both or neither, 16-byte aligned
+    assert lib.dl_block_select(ctypes.byref(d), fake, None, None, fake, fake, None, 256, 64, 4,
+                               None, 0, fake, fake, fake, 4, 0, fake, 1 << 40,
+                               None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_block_select(ctypes.byref(d), fake, None, None, fake, ctypes.c_void_p(0x1008),
+                               fake, 256, 64, 4, None, 0, fake, fake, fake, 4, 0, fake, 1 << 40,
+                               None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_pool_keys(ctypes.byref(d), fake, fake, 256, 64, 0, 64, fake, None, fake,
+                            None) == dl.DL_ERR_INVALID_ARG
+    assert "Kdig" in lib.dl_last_error_message().decode()
     # misaligned attention pointers
     odd = ctypes.c_void_p(0x1008)
     st = lib.dl_sparse_attn(ctypes.byref(d), odd, fake, fake, fake, None, None, 0, fake, fake,
@@ -98,7 +112,7 @@ def test_cache_write_arguments_rejected_before_launch():
     lib = _abi.lib
     d = _desc()
     fake = ctypes.c_void_p(0x1000)
-    args = [fake, fake, 32, fake, fake, fake, fake, fake, None]
+    args = [fake, fake, 32, fake, fake, fake, fake, fake, None, None, None]
     assert lib.dl_cache_write(ctypes.byref(d), *args[:1], None, *args[2:]) == dl.DL_ERR_INVALID_ARG
     for n_new in (0, 16385):  # 1 .. L_ctx
         a = list(args)
@@ -108,6 +122,9 @@ def test_cache_write_arguments_rejected_before_launch():
     a[0] = ctypes.c_void_p(0x1008)  # K_new off the 16-byte grid
     assert lib.dl_cache_write(ctypes.byref(d), *a) == dl.DL_ERR_INVALID_ARG
     assert "aligned" in lib.dl_last_error_message().decode()
+    a = list(args)
+    a[8] = fake  # Kdig without Kexp
+    assert lib.dl_cache_write(ctypes.byref(d), *a) == dl.DL_ERR_INVALID_ARG
 
 
 def test_kernel_flags_round_trip():
@@ -117,3 +134,8 @@ def test_kernel_flags_round_trip():
         assert dl.dl_set_kernel_flags(0) == 0
     finally:
         dl.dl_set_kernel_flags(prev)
+
+
+def test_read_counters_is_exported():
+    lib = ctypes.CDLL(_abi.LIB_PATH)
+    assert hasattr(lib, "dl_read_counters")

@@ -147,14 +147,13 @@ def test_multilayer_step_reduced(cuda_device):
     layers = [synth.make_step_inputs(wl, layer=l, device=cuda_device) for l in range(4)]
     step = pipeline.DenoiseStep(desc, 4, wl.first_sparse_layer, wl.topK, wl.detect_sinks, wl.k,
                                 wl.w, torch.bfloat16, cuda_device)
-    Kbar = [torch.empty((wl.batch, wl.H_kv, wl.n_blk, wl.d), dtype=torch.float32,
-                        device=cuda_device) for _ in range(4)]
+    kcs = [step.key_cache() for _ in range(4)]
     for l in range(4):
-        step.refresh_pooled_keys(l, layers[l].k_pool, layers[l].page_table, Kbar[l])
+        step.refresh_pooled_keys(l, layers[l].k_pool, layers[l].page_table, kcs[l])
     x0 = layers[0]
     step.run(x0.conf_prev, x0.still_masked, [x.q_dec for x in layers],
              [x.k_pool for x in layers], [x.v_pool for x in layers], x0.page_table,
-             [x.k_dec for x in layers], [x.v_dec for x in layers], Kbar)
+             [x.k_dec for x in layers], [x.v_dec for x in layers], kcs)
     assert dl.dl_get_status() == dl.DL_OK
     q_idx, q_cnt = oracle.step.predict_all(x0.conf_prev.cpu(), x0.still_masked.cpu(), wl.k, wl.w)
     assert np.array_equal(np_(step.q_idx), q_idx)
