@@ -142,15 +142,24 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- inputs
-def make_inputs(wl, device):
-    """All layers' tensors of the workload, drawn on the device."""
+def make_inputs(wl, device, kv_heads=None):
+    """All layers' tensors of the workload, drawn on the device; with
+    kv_heads = (g0, g1) only those KV heads (and their query heads) are kept,
+    as one rank of a head-sharded run holds them."""
     pt = synth.page_permutation(wl).to(device)
     layers = []
     for l in range(wl.n_layers):
         q = synth.make_q_dec(wl, l, device)
         kd, vd = synth.make_kv_dec(wl, l, device)
         kp, vp = synth.make_layer_kv(wl, l, q, device, pt.cpu())
-        layers.append(dict(q=q, kd=kd, vd=vd, kp=kp, vp=vp))
+        x = dict(q=q, kd=kd, vd=vd, kp=kp, vp=vp)
+        if kv_heads is not None:
+            g0, g1 = kv_heads
+            x = dict(q=q[:, g0 * wl.G:g1 * wl.G].contiguous(), kd=kd[:, g0:g1].contiguous(),
+                     vd=vd[:, g0:g1].contiguous(), kp=kp[:, g0:g1].contiguous(),
+                     vp=vp[:, g0:g1].contiguous())
+            del q, kd, vd, kp, vp
+        layers.append(x)
     confs, masks = zip(*(synth.confidence(wl, b) for b in range(wl.batch)))
     conf = torch.stack(confs).to(device)
     masked = torch.stack(masks).to(device)
@@ -272,7 +281,7 @@ def workload_record(name, device, pk, reps=30):
         ctx_tokens = toks / (wl.batch * wl.H_kv)
         # the int8 tensor-core selection reads the digit planes; the fp64 one Kbar
         fast = wl.dtype == "bf16" and wl.d == 128 and wl.G * min(wl.L_q, wl.k * (2 * wl.w + 1)) \
-            <= 32 and wl.n_blk <= 512
+            <= 24 and wl.n_blk <= 512
         key_b = Kdig.numel() + Kexp.numel() * 4 if fast else Kbar.numel() * 4
         nbytes = (key_b + q_b + wl.batch * wl.H_kv * wl.n_blk * 8 +
                   toks * wl.d * e * 2 + dec_b + o_b)
@@ -381,8 +390,9 @@ def run_reference(args):
     return 0
 
 
-def config_of(wl):
+def config_of(wl, parallelism="replicas"):
     return {"workload": WORKLOAD, "layers": wl.n_layers, "batch_per_gpu": wl.batch,
+            "parallelism": parallelism,
             "heads": wl.H, "kv_heads": wl.H_kv, "head_dim": wl.d, "context": wl.L_ctx,
             "decode_block": wl.L_q, "block": wl.B, "topK": wl.topK, "sinks": wl.detect_sinks,
             "dense_layers": wl.first_sparse_layer, "predict_k": wl.k, "window": wl.w,
@@ -396,16 +406,27 @@ def run_ours(args):
     import long_context_diffusion_b200 as dl
     from long_context_diffusion_b200 import pipeline
 
-    wl = synth.workload(WORKLOAD, n_layers=args.layers, batch=args.batch)
+    wl_full = synth.workload(WORKLOAD, n_layers=args.layers, batch=args.batch)
     torch.manual_seed(0)
-    desc = dl.make_desc(wl.batch, wl.H, wl.H_kv, wl.d, wl.L_ctx, wl.L_q, wl.B, wl.n_pages,
-                        wl.n_slots, dl.DL_BF16)
+    desc = dl.make_desc(wl_full.batch, wl_full.H, wl_full.H_kv, wl_full.d, wl_full.L_ctx,
+                        wl_full.L_q, wl_full.B, wl_full.n_pages, wl_full.n_slots, dl.DL_BF16)
+    heads = args.shard == "heads"
+    kv_heads, sink_group, wl = None, None, wl_full
+    if heads:
+        # this rank holds only its KV heads; the sink mass is all-reduced
+        from long_context_diffusion_b200 import sharded
+        hs = sharded.HeadShard.of(desc, rank, world)
+        desc, kv_heads = hs.desc, (hs.g0, hs.g1)
+        wl = wl_full.replace(H=hs.desc.H, H_kv=hs.desc.H_kv)
+        if world > 1:
+            import torch.distributed as dist
+            sink_group = dist.group.WORLD
     t_gen = time.time()
-    layers, pt, conf, masked = make_inputs(wl, device)
+    layers, pt, conf, masked = make_inputs(wl_full, device, kv_heads)
     t_gen = time.time() - t_gen
     L = wl.n_layers
     step = pipeline.DenoiseStep(desc, L, wl.first_sparse_layer, wl.topK, wl.detect_sinks, wl.k,
-                                wl.w, torch.bfloat16, device)
+                                wl.w, torch.bfloat16, device, sink_group=sink_group)
     Kbar = [step.key_cache() for _ in range(L)]  # (pooled keys, digits, exponents) per layer
     stream = torch.cuda.Stream(device)
     args_of = lambda: (conf, masked, [x["q"] for x in layers], [x["kp"] for x in layers],  # noqa
@@ -485,7 +506,11 @@ def run_ours(args):
             ctx_tokens.append(toks)
     attn_b = [attn_bytes(wl, t) for t in ctx_tokens]
     attn_f = [attn_flops(wl, t) for t in ctx_tokens]
-    kv_tokens = sum(sum(t) / wl.H_kv + wl.batch * wl.L_q for t in ctx_tokens)  # per step
+    # KV tokens attended per step, averaged over the KV heads (of the whole
+    # model when the heads are sharded)
+    tok_sum = runtime.sum_over_ranks(float(sum(sum(t) for t in ctx_tokens)), device) \
+        if heads else float(sum(sum(t) for t in ctx_tokens))
+    kv_tokens = tok_sum / wl_full.H_kv + L * wl.batch * wl.L_q
 
     # dominant kernel: the sparse-layer attention calls, over the timed region
     sparse_ms, dense_ms = [], []
@@ -529,6 +554,10 @@ def run_ours(args):
     # its results copied back, inside the timed graph.  Copies run on their own
     # streams, double-buffered: the inputs of step i+1 go up and the results
     # of step i-1 come down while step i computes.
+    def job_rate(seconds_per_step):
+        # replicas: every rank steps its own batch; heads: the ranks share one step
+        return (1.0 if heads else float(world)) / seconds_per_step if seconds_per_step else 0.0
+
     e2e = None
     if not args.no_e2e:
         keys = ("q", "kd", "vd")
@@ -616,7 +645,7 @@ def run_ours(args):
         torch.cuda.synchronize(device)
         runtime.barrier(device)
         e2e_ms = runtime.max_over_ranks(ev0.elapsed_time(ev1), device) / K
-        e2e = {"value": runtime.weak_throughput([1] * world, e2e_ms / 1e3), "unit": "steps/s",
+        e2e = {"value": job_rate(e2e_ms / 1e3), "unit": "steps/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms,
                "overlap": "inputs of step i+1 and results of step i-1 copied while step i "
@@ -624,13 +653,15 @@ def run_ours(args):
         del g_e2e
 
     launches_per_step = count_launches(wl)
-    value = runtime.weak_throughput([1] * world, t_step)
+    value = job_rate(t_step)
     line = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": K,
-        "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(wl),
-        "kv_tokens_per_s": kv_tokens * world / t_step,
-        "kv_tokens_per_step_per_gpu": kv_tokens,
+        "warmup": W, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong" if heads else "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_of(wl_full, f"heads{world}" if heads else "replicas"),
+        "kv_tokens_per_s": kv_tokens * (1 if heads else world) / t_step,
+        "kv_tokens_per_step": kv_tokens,
         "roofline": roof,
         "step_roofline": {"bytes": step_bytes, "flops": step_flops,
                           "frac_of_measured": t_roof_meas / t_step,
@@ -669,6 +700,33 @@ def run_ours(args):
     line["full_layer_pool"] = {"call": "dl_pool_keys", "avg_us": pm, "bytes": pool_b,
                                "achieved_GBps": pool_b / (pm * 1e-6) / 1e9,
                                "step_ms_if_amortised_per_step": ms_step + (pm - cw_mean) / 1e3}
+    # sinks kept across the steps of one decode block: a block of L_q steps
+    # (one position unmasked per step), the first step finds the sinks and
+    # the others keep them; each step commits one layer's block as above
+    n_blk_steps = wl.L_q
+    g_blk = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_blk, stream=stream):
+        for i in range(n_blk_steps):
+            commit(i, layers[i % L]["kd"], layers[i % L]["vd"])
+            step.run(*args_of(), stream=stream, find_sinks=(i == 0))
+    g_blk.replay()
+    torch.cuda.synchronize(device)
+    runtime.barrier(device)
+    blk_ms = []
+    for _ in range(2):
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            g_blk.replay()
+            ev1.record(stream)
+        torch.cuda.synchronize(device)
+        blk_ms.append(ev0.elapsed_time(ev1))
+    runtime.barrier(device)
+    blk_ms = runtime.max_over_ranks(min(blk_ms), device)
+    del g_blk
+    line["decode_block"] = {
+        "steps": n_blk_steps, "sinks": "found at the block's first step, kept by the others",
+        "ms_per_step": blk_ms / n_blk_steps, "steps_per_s": job_rate(blk_ms / n_blk_steps / 1e3),
+        "ms_per_step_keeping_sinks": (blk_ms - ms_step) / max(1, n_blk_steps - 1)}
     if not args.no_configs:
         line["workloads"] = {n: workload_record(n, device, pk)
                              for n in ("tiny", "llada8k", "dream16k", "chunked32k")}
@@ -684,10 +742,15 @@ def run_ours(args):
 
 
 def count_launches(wl):
-    """Kernels of this library launched per step (from the call sequence)."""
+    """Kernels of this library launched per step (from the call sequence):
+    the cache write, the prediction, one attention kernel per layer (it merges
+    its own split partials; a memset of the merge counts precedes it), the
+    sink search (LSE pass, mass pass, top-n) and one score + select kernel per
+    sparse layer when the group's rows fit a fused kernel (else three)."""
     n_sparse = wl.n_layers - wl.first_sparse_layer
-    pool, predict, attn, sinks = 1, 1, 2, 4
-    fused = wl.G * wl.L_q <= 32 and wl.n_blk <= 512  # dl_block_select: one kernel, else three
+    pool, predict, attn, sinks = 1, 1, 1, 3
+    rows = wl.G * min(wl.L_q, wl.k * (2 * wl.w + 1))
+    fused = rows <= 32 and wl.n_blk <= 512
     score_select = 1 if fused else 3
     return pool + predict + wl.first_sparse_layer * attn + sinks + n_sparse * (
         score_select + attn)
@@ -705,6 +768,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the sub-records of the other workloads")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="replicas: each GPU steps its own batch (weak scaling); heads: the "
+                         "GPUs split the KV heads of one batch and all-reduce the sink mass "
+                         "(strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours" and args.layers == 32:
         args.warmup = 3

@@ -210,6 +210,27 @@ dl_status dl_find_sinks(const dl_attn_desc* desc, const void* Q_dec, const int32
                         const void* K_dec, int n_sinks, int32_t* sink_pos, void* ws,
                         size_t ws_bytes, void* stream);
 
+/* (a4), split in its two halves for head-sharded execution.  The sink mass
+ * is a sum over heads, so a GPU that holds only some KV heads (desc->H_kv
+ * and desc->H of its shard, Q_dec / K_pool / K_dec of those heads only)
+ * computes its shard's part of mass[b][t] with dl_sink_mass; the parts are
+ * summed over the shards (an all-reduce of batch x L_ctx floats) and
+ * dl_sink_topn picks the sinks from the sum.  On one GPU the two calls give
+ * what dl_find_sinks gives.
+ * dl_sink_mass: mass fp32 [batch][L_ctx] (out, device; every element
+ *   written); the same arguments, checks and workspace as dl_find_sinks.
+ * dl_sink_topn: mass fp32 [batch][L_ctx] (device; in, and scratch when
+ *   n_sinks > 8: the chosen columns are overwritten with -inf);
+ *   sink_pos int32 [batch][n_sinks] (out), the n_sinks columns of largest
+ *   mass (ties -> lower index), ascending.  1 <= n_sinks <= 64.
+ *   No workspace.  Returns DL_ERR_INVALID_ARG for NULL pointers or sizes out
+ *   of range, before any launch. */
+dl_status dl_sink_mass(const dl_attn_desc* desc, const void* Q_dec, const int32_t* q_idx,
+                       const int32_t* q_cnt, const void* K_pool, const int32_t* page_table,
+                       const void* K_dec, float* mass, void* ws, size_t ws_bytes, void* stream);
+dl_status dl_sink_topn(float* mass, int batch, int L_ctx, int n_sinks, int32_t* sink_pos,
+                       void* stream);
+
 /* (a5) Sink-aware top-K block selection.  [F1 abstract; F2 summary]
  * For each (b, g): the sink units SB = { sink_pos[b][s] / unit_size : s,
  * sink_pos >= 0 } are always kept; the topK remaining units of largest score
@@ -228,8 +249,9 @@ dl_status dl_select(const double* score, int batch, int H_kv, int n_units, int u
  * written too).  [F2 summary: the predicted queries rank the blocks; F1
  * abstract: the sinks are always kept]
  * Kernels, by shape:
- *  - bf16 queries, d 128, G * max_q <= 32, n_units <= 512 and Kdig/Kexp given
- *    (the digits of these very Kbar, from dl_pool_keys / dl_cache_write):
+ *  - bf16 queries, d 128, G * max_q <= 24, n_units <= 512, Kdig/Kexp given
+ *    (the digits of these very Kbar, from dl_pool_keys / dl_cache_write) and
+ *    DL_FLAG_SCORE_FP64 not set:
  *    one CTA per (b, g) takes the logits q . Kbar exactly on the int8 tensor
  *    cores (query digits times key digits, int32 sums), in fp64 from there
  *    on, with a proven bound on each logit's error (the truncated digits);

@@ -9,7 +9,8 @@ not been built: there is no other implementation to fall back to.
 """
 from ._abi import (  # noqa: F401
     DLError, dl_attn_desc, make_desc, dl_version, dl_set_kernel_flags, dl_get_status, dl_workspace_size,
-    dl_predict_queries, dl_pool_keys, dl_cache_write, dl_block_scores, dl_find_sinks, dl_select,
+    dl_predict_queries, dl_pool_keys, dl_cache_write, dl_block_scores, dl_find_sinks, dl_sink_mass,
+    dl_sink_topn, dl_select,
     dl_block_select, dl_read_counters, key_digit_buffers,
     dl_sparse_attn, dl_token_select, dl_sparse_attn_gather, dl_block_scores_noalloc, LIB_PATH,
     DL_OK, DL_ERR_INVALID_ARG, DL_ERR_UNSUPPORTED, DL_ERR_WORKSPACE, DL_ERR_CUDA,

@@ -56,6 +56,9 @@ _SIGS = {
                        _vp, ctypes.c_size_t, _vp], _c_int),
     "dl_select": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _vp, _c_int,
                    _vp], _c_int),
+    "dl_sink_mass": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                      ctypes.c_size_t, _vp], _c_int),
+    "dl_sink_topn": ([_vp, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
     "dl_block_select": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _vp, _vp, _c_int,
                          _c_int, _c_int, _vp, _c_int, _vp, _vp, _vp, _c_int, _c_int, _vp,
                          ctypes.c_size_t, _vp], _c_int),
@@ -177,6 +180,21 @@ def dl_find_sinks(desc, Q_dec, q_idx, q_cnt, K_pool, page_table, K_dec, n_sinks,
     _check(lib.dl_find_sinks(ctypes.byref(desc), _p(Q_dec), _p(q_idx), _p(q_cnt), _p(K_pool),
                              _p(page_table), _p(K_dec), n_sinks, _p(sink_pos), _p(ws),
                              ws.numel() * ws.element_size(), _s(stream)))
+
+
+def dl_sink_mass(desc, Q_dec, q_idx, q_cnt, K_pool, page_table, K_dec, mass, ws, stream=None):
+    """This shard's part of the sink mass, mass fp32 [batch][L_ctx]."""
+    _check(lib.dl_sink_mass(ctypes.byref(desc), _p(Q_dec), _p(q_idx), _p(q_cnt), _p(K_pool),
+                            _p(page_table), _p(K_dec), _p(mass), _p(ws),
+                            ws.numel() * ws.element_size(), _s(stream)))
+
+
+def dl_sink_topn(mass, sink_pos, stream=None):
+    """sink_pos [batch][n_sinks] from the summed mass [batch][L_ctx]; with
+    more than 8 sinks the chosen columns of mass are overwritten."""
+    batch, L_ctx = mass.shape
+    _check(lib.dl_sink_topn(_p(mass), batch, L_ctx, sink_pos.shape[-1], _p(sink_pos),
+                            _s(stream)))
 
 
 def dl_select(score, unit_size, topK, sink_pos, blk_idx, blk_cnt, stream=None):

@@ -264,6 +264,36 @@ dl_status dl_find_sinks(const dl_attn_desc* desc, const void* Q_dec, const int32
                   "dl_find_sinks launch");
 }
 
+dl_status dl_sink_mass(const dl_attn_desc* desc, const void* Q_dec, const int32_t* q_idx,
+                       const int32_t* q_cnt, const void* K_pool, const int32_t* page_table,
+                       const void* K_dec, float* mass, void* ws, size_t ws_bytes, void* stream) {
+  dl::Shape s;
+  dl_status st = check_desc(desc, &s);
+  if (st != DL_OK) return st;
+  if (!Q_dec || !q_idx || !q_cnt || !K_pool || !page_table || !K_dec || !mass)
+    return fail(DL_ERR_INVALID_ARG, "dl_sink_mass: NULL pointer");
+  if (!aligned16(K_pool) || !aligned16(K_dec))
+    return fail(DL_ERR_INVALID_ARG, "K_pool/K_dec not 16-byte aligned");
+  if (s.L_ctx < 1) return fail(DL_ERR_INVALID_ARG, "dl_sink_mass: empty context");
+  if ((st = need_ws(ws, ws_bytes, dl::sinks_workspace(s))) != DL_OK) return st;
+  unsigned* err = nullptr;
+  if ((st = error_word(&err)) != DL_OK) return st;
+  return launched(dl::launch_sink_mass(s, Q_dec, q_idx, q_cnt, K_pool, page_table, K_dec, mass,
+                                       ws, err, as_stream(stream)),
+                  "dl_sink_mass launch");
+}
+
+dl_status dl_sink_topn(float* mass, int batch, int L_ctx, int n_sinks, int32_t* sink_pos,
+                       void* stream) {
+  if (!mass || !sink_pos) return fail(DL_ERR_INVALID_ARG, "dl_sink_topn: NULL pointer");
+  if (batch < 1 || L_ctx < 1)
+    return fail(DL_ERR_INVALID_ARG, "dl_sink_topn: batch=%d L_ctx=%d", batch, L_ctx);
+  if (n_sinks < 1 || n_sinks > 64) return fail(DL_ERR_INVALID_ARG, "n_sinks=%d (need 1..64)", n_sinks);
+  return launched(dl::launch_sink_topn_mass(mass, batch, L_ctx, n_sinks, sink_pos,
+                                            as_stream(stream)),
+                  "dl_sink_topn launch");
+}
+
 dl_status dl_select(const double* score, int batch, int H_kv, int n_units, int unit_size, int topK,
                     const int32_t* sink_pos, int n_sinks, int32_t* blk_idx, int32_t* blk_cnt,
                     int max_sel, void* stream) {

@@ -168,8 +168,6 @@ attn_combine_kernel(Shape s, int n_split, const void* ws, T* __restrict__ O,
   const int lane = threadIdx.x & 31;
   if (gw >= n_rows) return;
   const int bg = (int)(gw / R), r = (int)(gw % R);
-  const int b = bg / s.H_kv, g = bg % s.H_kv;
-  const int h = g * s.G + r / s.L_q, i = r % s.L_q;
   Partials part = partials_of(const_cast<void*>(ws), s, n_split);
   int n_valid = n_split;
   if (P > 0) {
@@ -180,55 +178,13 @@ attn_combine_kernel(Shape s, int n_split, const void* ws, T* __restrict__ O,
     n_valid = (int)(c1 - c0 + 1);
     n_valid = n_valid < n_split ? n_valid : n_split;
   }
-  constexpr int CPL = D / 32;
-  constexpr int SB = 4;  // slots per batch: their loads are all issued before any is used
-  float o[CPL];
-#pragma unroll
-  for (int c = 0; c < CPL; ++c) o[c] = 0.0f;
-  float M = -INFINITY, L = 0.0f;
-  for (int s0 = 0; s0 < n_valid; s0 += SB) {
-    float2 ml[SB];
-    float ov[SB][CPL];
-#pragma unroll
-    for (int q = 0; q < SB; ++q) {
-      const size_t row = ((size_t)bg * n_split + s0 + q) * R + r;
-      const bool ok = s0 + q < n_valid;
-      ml[q] = ok ? part.ml[row] : make_float2(-INFINITY, 0.0f);
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) ov[q][c] = (ok && O) ? part.o[row * D + lane + 32 * c] : 0.0f;
-    }
-    // merge this batch into the running (M, L, o), as the partials themselves
-    float Mb = M;
-#pragma unroll
-    for (int q = 0; q < SB; ++q) Mb = fmaxf(Mb, ml[q].x);
-    if (Mb == -INFINITY) continue;
-    const float a = M == -INFINITY ? 0.0f : expf(M - Mb);
-    L *= a;
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) o[c] *= a;
-#pragma unroll
-    for (int q = 0; q < SB; ++q) {
-      // an empty run (m = -inf) wrote no output row: skip it, never 0 * garbage
-      if (ml[q].x == -INFINITY) continue;
-      const float wgt = expf(ml[q].x - Mb);
-      L += ml[q].y * wgt;
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) o[c] = fmaf(ov[q][c], wgt, o[c]);
-    }
-    M = Mb;
-  }
-  if (O) {  // O == nullptr: the row LSEs only
-    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-    T* dst = O + (((size_t)b * s.L_q + i) * s.H + h) * D;
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) dst[lane + 32 * c] = from_f32<T>(o[c] * inv);
-  }
-  if (lse && lane == 0) lse[((size_t)b * s.H + h) * s.L_q + i] = L > 0.0f ? M + logf(L) : -INFINITY;
+  merge_row<T, D>(part, s, n_split, bg, r, n_valid, O, lse, lane);
 }
 
 size_t attn_workspace(const Shape& s) {
   const size_t n = (size_t)s.batch * s.H_kv * kMaxSplits * s.G * s.L_q;
-  return round256(n * s.d * sizeof(float)) + round256(n * sizeof(float2));
+  return round256(n * s.d * sizeof(float)) + round256(n * sizeof(float2)) +
+         round256((size_t)s.batch * s.H_kv * sizeof(int));  // merge counters
 }
 
 int attn_splits(const Shape& s, int max_tiles) {

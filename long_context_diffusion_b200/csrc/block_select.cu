@@ -43,8 +43,9 @@ block_select_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
 // The int8 tensor-core kernel (block_select_tc.cu) when the caller passes the
 // key digits and the shape fits it; else fused on the fp64 MMA when the
 // group's query rows (G x the bound max_q on q_cnt, or x L_q) fit four MMA
-// row tiles and the keys one thread each; otherwise block scores then
-// selection, as separate kernels.
+// row tiles and the keys one thread each; else, for more rows over at most
+// 128 units, the CUDA-core kernel of block_select_wide.cu; otherwise block
+// scores then selection, as separate kernels.
 cudaError_t launch_block_select(const Shape& s, const void* Q, const int32_t* q_idx,
                                 const int32_t* q_cnt, const float* Kbar, const int8_t* Kdig,
                                 const int32_t* Kexp, int n_units, double* score, int unit_size,
@@ -57,6 +58,9 @@ cudaError_t launch_block_select(const Shape& s, const void* Q, const int32_t* q_
     return launch_block_select_tc(s, Q, q_idx, q_cnt, Kbar, Kdig, Kexp, n_units, score, unit_size,
                                   topK, sink_pos, n_sinks, blk_idx, blk_cnt, max_sel, rows, err,
                                   st);
+  if (rows > bs::kMaxRows && block_select_wide_supported(s, rows, n_units))
+    return launch_block_select_wide(s, Q, q_idx, q_cnt, Kbar, n_units, score, unit_size, topK,
+                                    sink_pos, n_sinks, blk_idx, blk_cnt, max_sel, rows, err, st);
   if (rows > bs::kMaxRows || n_units > bs::kMaxUnits) {
     cudaError_t e = launch_scores(s, Q, q_idx, q_cnt, Kbar, n_units, score, ws, err, st);
     if (e != cudaSuccess) return e;

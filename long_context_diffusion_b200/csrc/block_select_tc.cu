@@ -37,14 +37,22 @@
 // are taken without subtracting the row maximum: |l| <= B_r <= 700 keeps
 // exp(l) finite and normal, and the softmax does not depend on the shift.
 //
-// Roles (512 threads, 16 warps): thread 480 (warp 15, lane 0) issues the TMA
-// loads of the key digit tiles (128 keys x 5 planes x 128 bytes, double
-// buffered) and the MMAs; warpgroup w (warps 4w .. 4w+3) drains tile w's
-// eight level columns from tensor memory (thread = key = threadIdx.x) into
-// fp64 logits and zeroes them for the tile that reuses them.  All waits are
-// bounded; a role that gives up sets the abort flag and the error word
-// (ERR_TIMEOUT), the CTA waits (bounded) for its loads and MMAs in flight,
-// frees its tensor memory and writes nothing.
+// Roles (512 threads, 16 warps): thread 448 (warp 14, lane 0) streams the
+// key digit planes by TMA through a ring of nine 16 KB stages (128 keys x
+// 128 bytes, one plane each); thread 480 (warp 15, lane 0) copies the
+// group's decode rows, issues the MMAs and commits them, tile by tile, into
+// two alternating sets of accumulator columns.  Warpgroup w < MT drains row
+// block w (query rows 8w .. 8w+7) of every tile: thread = key, the eight
+// level columns read from tensor memory, combined into fp64 logits, the
+// columns zeroed for the tile after next, and the exponentials kept in
+// registers.  With the issuing threads in warpgroup 3, at most three row
+// blocks (24 query rows) are drained; larger groups take the fp64 kernel.
+// After the scores, all 16 warps run the selection (one key per thread).
+// All waits are bounded; a role that gives up sets the abort flag and the
+// error word (ERR_TIMEOUT), the CTA waits (bounded) for its loads and MMAs
+// in flight, frees its tensor memory and writes nothing.  The decision to
+// keep the fast result or recompute in fp64 is taken by one thread and
+// broadcast through shared memory, so every thread takes the same branch.
 #include <cudaTypedefs.h>
 
 #include "block_select_common.cuh"
@@ -96,7 +104,8 @@ __device__ __forceinline__ double warp_rows_sum16(double (&v)[16], int lane) {
   return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 16);
 }
 
-// 2^k as a double, for k in the normal range.
+// 2^k as a double, for k in the normal range [-1022, 1023] (every use here:
+// exponent fields lie in [1, 254]).
 __device__ __forceinline__ double pow2i(int k) {
   return __longlong_as_double((long long)(k + 1023) << 52);
 }
@@ -132,12 +141,24 @@ __device__ __forceinline__ void radix_kth(uint64_t key, bool cand, int take, Rad
     rs.kmax[warp] = mx;
   }
   __syncthreads();
+  if (warp == 0) {  // the 16 warps' extremes, by shuffles
+    mn = lane < bs::kWarps ? rs.kmin[lane] : ~0ull;
+    mx = lane < bs::kWarps ? rs.kmax[lane] : 0ull;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long a = __shfl_xor_sync(0xffffffffu, mn, o);
+      const unsigned long long c = __shfl_xor_sync(0xffffffffu, mx, o);
+      mn = a < mn ? a : mn;
+      mx = c > mx ? c : mx;
+    }
+    if (lane == 0) {
+      rs.kmin[0] = mn;
+      rs.kmax[0] = mx;
+    }
+  }
+  __syncthreads();
   mn = rs.kmin[0];
   mx = rs.kmax[0];
-  for (int w = 1; w < bs::kWarps; ++w) {
-    mn = rs.kmin[w] < mn ? rs.kmin[w] : mn;
-    mx = rs.kmax[w] > mx ? rs.kmax[w] : mx;
-  }
   // bytes above the first one where the smallest and largest candidate differ
   const int lead = mn == mx ? 64 : __clzll((long long)(mn ^ mx));
   const int first_shift = mn == mx ? -8 : 56 - (lead / 8) * 8;
@@ -149,8 +170,7 @@ __device__ __forceinline__ void radix_kth(uint64_t key, bool cand, int take, Rad
     __syncthreads();
     const bool in = (key & fixed) == prefix;
     const unsigned dg = (unsigned)(key >> shift) & 255u;
-    const unsigned grp = __match_any_sync(0xffffffffu, in ? dg : 256u + lane);
-    if (in && lane == __ffs(grp) - 1) atomicAdd(&rs.hist[dg], __popc(grp));
+    if (in) atomicAdd(&rs.hist[dg], 1);
     __syncthreads();
     if (warp == 0) {
       int c[8], loc = 0;
@@ -195,6 +215,30 @@ __device__ __forceinline__ void radix_kth(uint64_t key, bool cand, int take, Rad
   *rem_out = rem;
 }
 
+// Exclusive prefix count of `flag` over the CTA in thread order (kThreads
+// threads), and the total: ballots per warp, the 16 warp counts scanned by
+// warp 0 with shuffles.
+__device__ __forceinline__ int cta_prefix_count(bool flag, int* s_cnt, int* total) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned bal = __ballot_sync(0xffffffffu, flag);
+  if (lane == 0) s_cnt[warp] = __popc(bal);
+  __syncthreads();
+  if (warp == 0) {
+    const int c = lane < bs::kWarps ? s_cnt[lane] : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane < bs::kWarps) s_cnt[32 + lane] = incl - c;
+    if (lane == 31) s_cnt[64] = incl;
+  }
+  __syncthreads();
+  *total = s_cnt[64];
+  return s_cnt[32 + warp] + __popc(bal & ((1u << lane) - 1u));
+}
+
 // Counters of the int8 kernel: CTAs that kept their fast result, CTAs that
 // fell back to fp64 (read and cleared by dl_read_counters).
 __device__ unsigned long long g_select_counts[2];
@@ -213,7 +257,9 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
   using namespace bstc;
   using L = Layout<NQ>;
   constexpr int NR = 8 * MT;  // query rows of the launch (<= NQ)
-  static_assert(NR <= NQ && NQ <= 32, "rows");
+  // row block w is drained by warpgroup w; warpgroup 3 holds the issuing
+  // threads and never drains, so at most three row blocks
+  static_assert(NR <= NQ && NQ <= 32 && MT <= 3, "rows");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -233,7 +279,7 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
   __shared__ int s_qpos[256], s_qcnt;
   __shared__ double s_exp_tab[64];
   __shared__ uint8_t s_sink[bs::kMaxUnits];
-  __shared__ int s_warp[33];
+  __shared__ int s_cnt[72];
   __shared__ unsigned long long s_min[bs::kWarps];
   __shared__ RadixScratch s_rad;
   volatile int* abort_v = &abort_flag;
@@ -241,9 +287,10 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bg = blockIdx.x, b = bg / s.H_kv, g = bg % s.H_kv;
   const int nt = (n_units + kTileKeys - 1) / kTileKeys;  // <= 4
+  const int tl = nt - 1;                                 // the last tile
   const int J = nt * kKeyDigits;                         // digit planes to stream
   const bool q_whole = s.G * s.L_q <= kQRawRows;         // decode rows prefetched whole
-  auto plane_load = [&](int j) {  // control thread only
+  auto plane_load = [&](int j) {  // producer thread only
     const int st = j % kStages;
     mbar_arrive_expect_tx(&full[st], kPlaneBytes);
     tma_load_3d(sK + st * kPlaneBytes, &kdig_map, 0, (j / kKeyDigits) * kTileKeys,
@@ -251,18 +298,18 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
   };
 
   pdl_wait();
-  // small loads first, so that they do not queue behind the key digit
-  // stream: the predicted positions, the sink positions, this thread's key
-  // exponent word, the exponential table; the control thread sets up the
-  // barriers and starts the copy of the group's decode rows
+  // The small loads are issued first (into registers; a barrier does not
+  // wait for them), so that they enter the memory queues ahead of the key
+  // digit stream, which starts right after the barrier.  The control thread
+  // sets up the barriers and copies the group's decode rows.
   if (tid == kCtl) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < 4; ++i) mbar_init(&mma_done[i], 1);
-    mbar_init(&tmem_free[0], 128);
-    mbar_init(&tmem_free[1], 128);
+    mbar_init(&tmem_free[0], 128 * MT);  // the draining warpgroups
+    mbar_init(&tmem_free[1], 128 * MT);
     mbar_init(&qfull, 1);
     abort_flag = 0;
     s_Emax = 1;
@@ -280,13 +327,14 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
   const int key = tid;
   const bool key_ok = key < n_units;
   const int ke = key_ok ? __ldg(Kexp + (size_t)bg * n_units + key) : 0;
+  int qcnt = 0;
   if (warp == 1) {
     for (int i = lane; i < s.L_q; i += 32) s_qpos[i] = q_idx ? q_idx[(size_t)b * s.L_q + i] : i;
-    if (lane == 0) s_qcnt = q_idx ? q_cnt[b] : s.L_q;
+    if (lane == 0) qcnt = q_idx ? q_cnt[b] : s.L_q;
   }
-  s_sink[tid] = 0;
-  if (tid < 64) s_exp_tab[tid] = kPow2Frac64[tid];
   const int sp0 = (warp == 2 && lane < n_sinks) ? sink_pos[(size_t)b * n_sinks + lane] : -1;
+  const double tabv = tid < 64 ? kPow2Frac64[tid] : 0.0;
+  s_sink[tid] = 0;
   if (warp == 0) {
     tmem_alloc(&tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -296,14 +344,14 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  // the key digit stream: the first kStages planes
-  if (tid == kProd) {
+  if (tid == kProd) {  // the key digit stream: the first kStages planes
     const int n0 = J < kStages ? J : kStages;
     for (int j = 0; j < n0; ++j) plane_load(j);
     s_issued_tma = n0;
   }
-  // sink units (kept whatever their score)
-  if (warp == 2 && lane < n_sinks && sp0 >= 0) {
+  if (warp == 1 && lane == 0) s_qcnt = qcnt;
+  if (tid < 64) s_exp_tab[tid] = tabv;
+  if (warp == 2 && lane < n_sinks && sp0 >= 0) {  // sink units (kept whatever their score)
     const long long u = sp0 / unit_size;
     if (u < n_units) s_sink[u] = 1;
     else flag_error(err, ERR_BAD_INDEX);
@@ -318,8 +366,9 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
   }
 
   // every digit-pair MMA accumulates: the two tiles' columns start at zero
-  // (warpgroups 0 and 1, each its buffer; rewritten after each drain)
-  auto zero_cols = [&](int buf) {  // one warpgroup: its warp's 32 lanes x TILE_COLS
+  // (warps 0-7 for both buffers, each its 32 lanes; later rows are zeroed
+  // by the warps that drain them)
+  auto zero_cols = [&](int buf) {  // this warp's 32 lanes of one tile buffer
     uint32_t z[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) z[i] = 0u;
@@ -329,13 +378,6 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
     tmem_st_wait();
   };
   if (warp < 8) zero_cols(warp >> 2);
-
-  int nq = min(max(s_qcnt, 0), s.L_q);
-  if (nq * s.G > NR) {  // more rows than the caller's bound: reported, rows cut
-    if (tid == 0) flag_error(err, ERR_BAD_INDEX);
-    nq = NR / s.G;
-  }
-  const int R = nq * s.G;  // <= NR
 
   // key exponents: block maxima for the bound
   int Eu = 1;
@@ -353,6 +395,13 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
       atomicMax(&s_NK, nk);
     }
   }
+  __syncthreads();  // s_qpos, s_qcnt, s_exp_tab, s_sink
+  int nq = min(max(s_qcnt, 0), s.L_q);
+  if (nq * s.G > NR) {  // more rows than the caller's bound: reported, rows cut
+    if (tid == 0) flag_error(err, ERR_BAD_INDEX);
+    nq = NR / s.G;
+  }
+  const int R = nq * s.G;  // <= NR
 
   // ---- query rows -> four digit planes (row r = tid / 16, dims 8p .. 8p+7)
   {
@@ -425,7 +474,8 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
     const uint64_t kdesc0 = sdesc_sw128(smem_u32(sK), 16, 1024);
     const uint64_t qdesc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
     bool ok = true;
-    for (int j = 0; ok && j < J; ++j) {
+    int j = 0;
+    for (; ok && j < J; ++j) {
       const int t = j / kKeyDigits, tk = j % kKeyDigits, st = j % kStages;
       if (!(ok = mbar_wait(&full[st], (j / kStages) & 1, abort_v))) break;
       if (tk == 0 && t >= 2 &&
@@ -439,74 +489,114 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
                   qdesc0 + (uint64_t)((kk * 32) >> 4), IDESC, 1u);
       mma_commit(&empty[st]);
       if (tk == kKeyDigits - 1) mma_commit(&mma_done[t]);
-      s_issued_mma = j + 1;
     }
+    s_issued_mma = j;
     if (!ok) flag_error(err, ERR_TIMEOUT);
   } else if (tid == kProd) {
     bool ok = true;
-    for (int j = 0; ok && j + kStages < J; ++j) {
+    int j = 0;
+    for (; ok && j + kStages < J; ++j) {
       const int st = j % kStages;
       if (!(ok = mbar_wait(&empty[st], (j / kStages) & 1, abort_v))) break;
       plane_load(j + kStages);
-      s_issued_tma = j + kStages + 1;
     }
+    s_issued_tma = (J < kStages ? J : kStages) + j;
     if (!ok) flag_error(err, ERR_TIMEOUT);
   }
   __syncwarp();
 
-  // ---- drains: warpgroup w turns tile w's eight levels into fp64 logits
-  double lg[NR];
-#pragma unroll
-  for (int r = 0; r < NR; ++r) lg[r] = 0.0;
+  // ---- drains: every tile by every warpgroup w < MT, row block w (rows
+  // 8w .. 8w+7), thread = key 128 t + (threadIdx.x & 127).  Level sums ->
+  // fp64 logits -> softmax numerators p = exp(l) without a shift (|l| <= B_r;
+  // if B_r <= 700 fails below, the fp64 kernel redoes the (b, g)); the p
+  // values stay in registers (one row block of four keys) and each warp adds
+  // its partial row sums to s_red[warp][row].
   const int wg = warp >> 2;
-  if (wg < nt) {
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(&mma_done[wg], 0, abort_v));
-    if (ok) {
-      tc_fence_after();
-      const uint32_t base = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (wg & 1) * L::TILE_COLS;
-      const double sc = s.scale;
+  const double sc = s.scale;
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  double pv[4][8];  // [tile][row of the block]
 #pragma unroll
-      for (int rb = 0; rb < MT; ++rb) {
-        // levels c = 0..7 of rows rb*8 .. rb*8+7, combined two by two:
-        // V = h0 2^42 + h1 2^28 + h2 2^14 + h3, h_k = A_2k * 128 + A_2k+1 (int32)
-        int h[4][8];
+  for (int t = 0; t < 4; ++t)
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint32_t a0[8], a1[8];
-          tmem_ld8(base + (2 * k) * NQ + rb * 8, a0);
-          tmem_ld8(base + (2 * k + 1) * NQ + rb * 8, a1);
+    for (int i = 0; i < 8; ++i) pv[t][i] = 0.0;
+  double zr[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) zr[i] = 0.0;
+  const bool drains = wg < MT;
+  const int row0 = wg * 8;
+  int erow[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) erow[i] = s_rowE[(row0 + i) & 31];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    if (t < nt) {
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&mma_done[t], 0, abort_v));
+      const int tkey = t * kTileKeys + (tid & 127);
+      const bool kok = tkey < n_units;
+      if (ok && drains) {
+        const int ket = kok ? __ldg(Kexp + (size_t)bg * n_units + tkey) : 0;
+        const int et = max(ket & 255, 1);
+        tc_fence_after();
+        const uint32_t base = tmem + lane_base + (t & 1) * L::TILE_COLS + row0;
+        // V = h0 2^42 + h1 2^28 + h2 2^14 + h3, h_k = A_2k * 128 + A_2k+1 (int32),
+        // the eight levels read in two halves
+        double l[8];
+        {
+          uint32_t a[4][8];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld8(base + c * NQ, a[c]);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 8; ++i) h[k][i] = (int)a0[i] * 128 + (int)a1[i];
+          for (int i = 0; i < 8; ++i) {
+            const int h0 = (int)a[0][i] * 128 + (int)a[1][i];
+            const int h1 = (int)a[2][i] * 128 + (int)a[3][i];
+            l[i] = fma((double)h1, 0x1p28, (double)h0 * 0x1p42);
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld8(base + (4 + c) * NQ, a[c]);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int h2 = (int)a[0][i] * 128 + (int)a[1][i];
+            const int h3 = (int)a[2][i] * 128 + (int)a[3][i];
+            const double v = fma((double)h2, 0x1p14, l[i]) + (double)h3;
+            l[i] = v * (sc * pow2i(erow[i] + et - 315));
+          }
+        }
+        if (t + 2 < nt) {  // tile t + 2 accumulates in these columns: zero them
+          uint32_t z[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) z[i] = 0u;
+#pragma unroll
+          for (int c = 0; c < kLevels; ++c) tmem_st8(base + c * NQ, z);
+          tmem_st_wait();
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int r = rb * 8 + i;
-          double v = fma((double)h[1][i], 0x1p28, (double)h[0][i] * 0x1p42);
-          v = fma((double)h[2][i], 0x1p14, v) + (double)h[3][i];
-          lg[r] = v * (sc * pow2i(s_rowE[r] + Eu - 315));
+          const double pe = exp_fp64(l[i], s_exp_tab);
+          pv[t][i] = (kok && row0 + i < R) ? pe : 0.0;
+          zr[i] += pv[t][i];
         }
       }
-      if (wg + 2 < nt) zero_cols(wg & 1);  // tile wg + 2 accumulates here
-    }
-    tc_fence_before();
-    mbar_arrive(&tmem_free[wg & 1]);
-    // softmax numerators without a shift, p = exp(l) (|l| <= B_r; when the
-    // bound B_r <= 700 fails below, the fp64 kernel redoes the (b, g)), and
-    // this warp's partial row sums: overlaps the later tiles' stream
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
-      if (r < R) lg[r] = key_ok ? exp_fp64(lg[r], s_exp_tab) : 0.0;  // r < R: uniform
-      else lg[r] = 0.0;
+      tc_fence_before();
+      if (drains && t + 2 < nt) mbar_arrive(&tmem_free[t & 1]);  // read and zeroed
     }
   }
+  // this warp's partial row sums: the 8 rows of its block over its 32 keys
+  if (drains) {
 #pragma unroll
-  for (int half = 0; half < NR; half += 16) {
-    double v[16];
+    for (int i = 0; i < 8; ++i) {
+      double v = zr[i];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = half + i < NR ? lg[half + i] : 0.0;
-    const double z = warp_rows_sum16(v, lane);
-    if (lane < 16 && half + lane < NR) s_red[warp][half + lane] = z;
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      zr[i] = v;
+    }
+    if (lane < 8) {
+      double v = zr[0];
+#pragma unroll
+      for (int i = 1; i < 8; ++i) v = lane == i ? zr[i] : v;
+      s_red[warp][row0 + lane] = v;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -535,17 +625,20 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
   }
   if (*abort_v) return;
 
-  // ---- bound of the logit errors (rows < R) and of |l|
-  const int Emax = s_Emax, NK = s_NK;
-  if (warp == 1) {
+  // ---- Z_r (sum of the four warps of the row's block) and the bound of the
+  // logit errors
+  if (tid < 32) {
+    const int r = tid, w0 = (r >> 3) * 4;
+    const double z = (r < 8 * MT) ? (s_red[w0][r] + s_red[w0 + 1][r]) + (s_red[w0 + 2][r] + s_red[w0 + 3][r]) : 0.0;
+    s_iZ[r] = (r < R && z > 0.0) ? 1.0 / z : 0.0;
+  } else if (warp == 9) {
+    const int Emax = s_Emax, NK = s_NK;
     double dmax = 0.0, bmax = 0.0;
     if (lane < R) {
       const int er = s_rowE[lane];
-      const double sc = s.scale;
-      const double b_r = sc * (double)s_rowL1[lane] * ldexp(1.0, Emax - 126) * 1.001;
-      const double d_r = sc * ((double)s_rowNq[lane] * ldexp(1.0, er + Emax - 280) +
-                               (double)NK * ldexp(1.0, er + Emax - 287) +
-                               ldexp(1.0, er + Emax - 320)) +
+      const double b_r = sc * (double)s_rowL1[lane] * pow2i(Emax - 126) * 1.001;
+      const double d_r = sc * ((double)s_rowNq[lane] * pow2i(er + Emax - 280) +
+                               (double)NK * pow2i(er + Emax - 287) + pow2i(er + Emax - 320)) +
                          0x1p-49 * b_r;
       dmax = d_r;
       bmax = b_r;
@@ -557,17 +650,22 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
       s_keep_fast = bmax <= 700.0 ? 1 : 0;  // exp(l) stays finite and normal
     }
   }
-  // ---- Z_r = sum over keys of the warps' partial sums
   __syncthreads();
-  if (tid < NR) {
-    double z = 0.0;
-    for (int w = 0; w < bs::kWarps; ++w) z += s_red[w][tid];
-    s_iZ[tid] = (tid < R && z > 0.0) ? 1.0 / z : 0.0;
+  // scores: each warpgroup's row-block partial of its four keys, then the
+  // sum over the row blocks (the ring is free: every MMA is done)
+  double* sPart = reinterpret_cast<double*>(sK);  // [MT][512]
+  if (drains) {
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      double a0 = 0.0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a0 = fma(pv[t][i], s_iZ[row0 + i], a0);
+      sPart[wg * 512 + t * kTileKeys + (tid & 127)] = a0;
+    }
   }
   __syncthreads();
   double my = 0.0;
-#pragma unroll
-  for (int r = 0; r < NR; ++r) my = fma(lg[r], s_iZ[r], my);
+  for (int w = 0; w < MT; ++w) my += sPart[w * 512 + tid];
   const double E = s_E;
   const bool bounded = s_keep_fast != 0;
 
@@ -584,24 +682,32 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
     int rem;
     radix_kth(mykey, key_ok && !is_sink, take, s_rad, &kstar, &rem);
     // the keys equal to k* are taken in thread order, rem of them
-    int n_eq = 0;
-    const int eq_before = block_exclusive_count(mykey == kstar, s_warp, &n_eq);
-    sel = mykey < kstar || (mykey == kstar && eq_before < rem);
+    const int n_eq = __syncthreads_count(mykey == kstar);
+    if (n_eq == 1) {
+      sel = mykey <= kstar;
+    } else {
+      int tot = 0;
+      const int eq_before = cta_prefix_count(mykey == kstar, s_cnt, &tot);
+      sel = mykey < kstar || (mykey == kstar && eq_before < rem);
+    }
     if (take < n_cand && R > 0) {
       // the best key not taken: the next equal one, or the smallest above k*
-      uint64_t above = mykey > kstar ? mykey : ~0ull;
+      unsigned long long above = mykey > kstar ? mykey : ~0ull;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
-        const unsigned long long v = __shfl_xor_sync(0xffffffffu, (unsigned long long)above, o);
+        const unsigned long long v = __shfl_xor_sync(0xffffffffu, above, o);
         above = v < above ? v : above;
       }
       if (lane == 0) s_min[warp] = above;
       __syncthreads();
-      uint64_t next = n_eq > rem ? kstar : ~0ull;
-      for (int w = 0; w < bs::kWarps; ++w) next = s_min[w] < next ? s_min[w] : next;
-      const double s_k = score_of_desc_key(kstar), s_k1 = score_of_desc_key(next);
-      fast = fast && R > 0 && s_k * (1.0 - E) > s_k1 * (1.0 + E);
-      if (R == 0) fast = true;
+      if (tid == 0) {  // one thread decides, for every thread
+        unsigned long long next = n_eq > rem ? kstar : ~0ull;
+        for (int w = 0; w < bs::kWarps; ++w) next = s_min[w] < next ? s_min[w] : next;
+        const double s_k = score_of_desc_key(kstar), s_k1 = score_of_desc_key(next);
+        s_keep_fast = (fast && s_k * (1.0 - E) > s_k1 * (1.0 + E)) ? 1 : 0;
+      }
+      __syncthreads();
+      fast = s_keep_fast != 0;
     }
   }
   if (R == 0) fast = true;  // no rows: every score is exactly 0 on both sides
@@ -609,7 +715,7 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
     if (key_ok) score[(size_t)bg * n_units + key] = my;
     const bool keep = key_ok && (sel || is_sink);
     int total = 0;
-    const int pos = block_exclusive_count(keep, s_warp, &total);
+    const int pos = cta_prefix_count(keep, s_cnt, &total);
     int32_t* out = blk_idx + (size_t)bg * max_sel;
     if (keep && pos < max_sel) out[pos] = key;
     for (int e = total + tid; e < max_sel; e += kThreads) out[e] = -1;
@@ -628,7 +734,7 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
 
 // Whether the int8 kernel takes this call.
 bool block_select_tc_supported(const Shape& s, int rows, int n_units) {
-  return s.dtype == 0 && s.d == 128 && rows <= 32 && n_units <= bs::kMaxUnits &&
+  return s.dtype == 0 && s.d == 128 && rows <= 24 && n_units <= bs::kMaxUnits &&
          !(kernel_flags() & DL_FLAG_SCORE_FP64);
 }
 
@@ -661,8 +767,7 @@ cudaError_t launch_block_select_tc(const Shape& s, const void* Q, const int32_t*
     case 0:
     case 1: DL_BSTC(16, 1) break;
     case 2: DL_BSTC(16, 2) break;
-    case 3: DL_BSTC(32, 3) break;
-    default: DL_BSTC(32, 4) break;
+    default: DL_BSTC(32, 3) break;
   }
 #undef DL_BSTC
   return cudaGetLastError();

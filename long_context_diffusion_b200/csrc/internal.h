@@ -82,6 +82,19 @@ cudaError_t launch_block_select_tc(const Shape& s, const void* Q, const int32_t*
                                    int rows, unsigned* err, cudaStream_t st);
 cudaError_t read_select_counts(unsigned long long* fast, unsigned long long* fallback);
 
+bool block_select_wide_supported(const Shape& s, int rows, int n_units);
+cudaError_t launch_block_select_wide(const Shape& s, const void* Q, const int32_t* q_idx,
+                                     const int32_t* q_cnt, const float* Kbar, int n_units,
+                                     double* score, int unit_size, int topK,
+                                     const int32_t* sink_pos, int n_sinks, int32_t* blk_idx,
+                                     int32_t* blk_cnt, int max_sel, int rows, unsigned* err,
+                                     cudaStream_t st);
+cudaError_t launch_sink_mass(const Shape& s, const void* Q, const int32_t* q_idx,
+                             const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
+                             const void* Kd, float* mass, void* ws, unsigned* err,
+                             cudaStream_t st);
+cudaError_t launch_sink_topn_mass(float* mass, int batch, int L_ctx, int n_sinks,
+                                  int32_t* sink_pos, cudaStream_t st);
 cudaError_t launch_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
                          const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
                          const void* Kd, int n_sinks, int32_t* sink_pos, void* ws,

@@ -378,11 +378,12 @@ static cudaError_t launch_sink_topn(const Shape& s, int n_sinks, const SinkWs& w
 }
 
 template <typename T, int D>
-static cudaError_t run_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
-                             const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
-                             const void* Kd, int n_sinks, int32_t* sink_pos, void* ws,
-                             unsigned* err, cudaStream_t st) {
+static cudaError_t run_sink_mass(const Shape& s, const void* Q, const int32_t* q_idx,
+                                 const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
+                                 const void* Kd, float* mass, void* ws, unsigned* err,
+                                 cudaStream_t st) {
   SinkWs w = sink_ws(ws, s);
+  w.mass = mass;
   const T* q = reinterpret_cast<const T*>(Q);
   const T* kp = reinterpret_cast<const T*>(Kp);
   const T* kd = reinterpret_cast<const T*>(Kd);
@@ -394,8 +395,7 @@ static cudaError_t run_sinks(const Shape& s, const void* Q, const int32_t* q_idx
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   DL_LAUNCH(sink_mass_kernel<T, D>, dim3((s.L_ctx + kSinkTile - 1) / kSinkTile, s.batch), kSinkTile, 0,
                            st, s, q, q_idx, q_cnt, kp, page_table, w, err);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  return launch_sink_topn(s, n_sinks, w, sink_pos, st);
+  return cudaGetLastError();
 }
 
 bool attn_tc_supported(const AttnArgs& a);
@@ -405,14 +405,16 @@ cudaError_t launch_sink_mass_tc(const Shape& s, const void* Q, const int32_t* q_
                                 const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
                                 const float* lse, float* mass, unsigned* err, cudaStream_t st);
 
-// bf16 with at most 256 query rows per KV group: tensor cores (pass 1 = dense
-// attention for the row LSEs -- LSE-only on the key-major kernel, otherwise
-// with V = K and the output discarded --, pass 2 = sinks_tc.cu); otherwise
-// the CUDA-core passes above.
-cudaError_t launch_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
-                         const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
-                         const void* Kd, int n_sinks, int32_t* sink_pos, void* ws,
-                         unsigned* err, cudaStream_t st) {
+// Column masses of the predicted rows of this descriptor's heads into
+// mass[b][L_ctx] (NULL: the workspace's mass array).  bf16 with at most 256
+// query rows per KV group: tensor cores (pass 1 = dense attention for the
+// row LSEs -- LSE-only on the key-major kernel, otherwise with V = K and the
+// output discarded --, pass 2 = sinks_tc.cu); otherwise the CUDA-core passes
+// above.
+cudaError_t launch_sink_mass(const Shape& s, const void* Q, const int32_t* q_idx,
+                             const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
+                             const void* Kd, float* mass, void* ws, unsigned* err,
+                             cudaStream_t st) {
   SinkTcWs tw = sink_tc_ws(ws, s);
   AttnArgs a{};
   a.s = s; a.Q = Q; a.Kp = Kp; a.Vp = Kp; a.page_table = page_table; a.mode = kDense;
@@ -423,21 +425,42 @@ cudaError_t launch_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
     if (attn_tc_kt_supported(a)) a.O = nullptr;
     cudaError_t e = launch_attn(a, st);
     if (e != cudaSuccess) return e;
-    e = launch_sink_mass_tc(s, Q, q_idx, q_cnt, Kp, page_table, tw.lse, tw.mass, err, st);
-    if (e != cudaSuccess) return e;
-    SinkWs w = sink_ws(ws, s);
-    w.mass = tw.mass;
-    return launch_sink_topn(s, n_sinks, w, sink_pos, st);
+    return launch_sink_mass_tc(s, Q, q_idx, q_cnt, Kp, page_table, tw.lse,
+                               mass ? mass : tw.mass, err, st);
   }
+  float* m = mass ? mass : sink_ws(ws, s).mass;
   if (s.dtype == 0)
-    return s.d == 128 ? run_sinks<__nv_bfloat16, 128>(s, Q, q_idx, q_cnt, Kp, page_table, Kd,
-                                                      n_sinks, sink_pos, ws, err, st)
-                      : run_sinks<__nv_bfloat16, 64>(s, Q, q_idx, q_cnt, Kp, page_table, Kd,
-                                                     n_sinks, sink_pos, ws, err, st);
-  return s.d == 128 ? run_sinks<float, 128>(s, Q, q_idx, q_cnt, Kp, page_table, Kd, n_sinks,
-                                            sink_pos, ws, err, st)
-                    : run_sinks<float, 64>(s, Q, q_idx, q_cnt, Kp, page_table, Kd, n_sinks,
-                                           sink_pos, ws, err, st);
+    return s.d == 128 ? run_sink_mass<__nv_bfloat16, 128>(s, Q, q_idx, q_cnt, Kp, page_table, Kd,
+                                                          m, ws, err, st)
+                      : run_sink_mass<__nv_bfloat16, 64>(s, Q, q_idx, q_cnt, Kp, page_table, Kd,
+                                                         m, ws, err, st);
+  return s.d == 128 ? run_sink_mass<float, 128>(s, Q, q_idx, q_cnt, Kp, page_table, Kd, m, ws,
+                                                err, st)
+                    : run_sink_mass<float, 64>(s, Q, q_idx, q_cnt, Kp, page_table, Kd, m, ws,
+                                               err, st);
+}
+
+// The n_sinks columns of largest mass (ties to the lower position), ascending.
+// More than 8 sinks: the chosen columns of mass are overwritten with -inf.
+cudaError_t launch_sink_topn_mass(float* mass, int batch, int L_ctx, int n_sinks,
+                                  int32_t* sink_pos, cudaStream_t st) {
+  Shape s{};
+  s.batch = batch;
+  s.L_ctx = L_ctx;
+  SinkWs w{};
+  w.mass = mass;
+  return launch_sink_topn(s, n_sinks, w, sink_pos, st);
+}
+
+cudaError_t launch_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
+                         const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
+                         const void* Kd, int n_sinks, int32_t* sink_pos, void* ws,
+                         unsigned* err, cudaStream_t st) {
+  const bool tc = s.dtype == 0 && s.G * s.L_q <= 256;
+  float* mass = tc ? sink_tc_ws(ws, s).mass : sink_ws(ws, s).mass;
+  cudaError_t e = launch_sink_mass(s, Q, q_idx, q_cnt, Kp, page_table, Kd, mass, ws, err, st);
+  if (e != cudaSuccess) return e;
+  return launch_sink_topn_mass(mass, s.batch, s.L_ctx, n_sinks, sink_pos, st);
 }
 
 }  // namespace dl

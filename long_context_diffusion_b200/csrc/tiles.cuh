@@ -81,4 +81,73 @@ __host__ __device__ inline Partials partials_of(void* ws, const Shape& s, int n_
   return p;
 }
 
+// Per (b, g), how many of the CTAs that share it have written their partials
+// (the merge inside the persistent tensor-core kernel: the CTA that makes the
+// count complete merges them).  After the partials of kMaxSplits slots; zeroed
+// before each launch.
+__host__ __device__ inline int* merge_counters_of(void* ws, const Shape& s) {
+  const size_t n = (size_t)s.batch * s.H_kv * kMaxSplits * s.G * s.L_q;
+  return reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + round256(n * s.d * sizeof(float)) +
+                                round256(n * sizeof(float2)));
+}
+
+// Merge the split partials of one (b, g, row r) into O and lse: O = sum_s
+// acc_s e^{m_s-M} / L, L = sum_s l_s e^{m_s-M}, lse = M + ln L, over slots
+// [0, n_valid) of the n_split allocated.  One warp per row (lane = columns
+// lane, lane + 32, ...).  The partial loads go through L2 (ld.global.cg):
+// they may have been written by other CTAs of the running kernel.
+template <typename T, int D>
+__device__ __forceinline__ void merge_row(const Partials& part, const Shape& s, int n_split,
+                                          int bg, int r, int n_valid, T* __restrict__ O,
+                                          float* __restrict__ lse, int lane) {
+  const int R = s.G * s.L_q;
+  const int b = bg / s.H_kv, g = bg % s.H_kv;
+  const int h = g * s.G + r / s.L_q, i = r % s.L_q;
+  constexpr int CPL = D / 32;
+  constexpr int SB = 4;  // slots per batch: their loads are all issued before any is used
+  float o[CPL];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) o[c] = 0.0f;
+  float M = -INFINITY, L = 0.0f;
+  for (int s0 = 0; s0 < n_valid; s0 += SB) {
+    float2 ml[SB];
+    float ov[SB][CPL];
+#pragma unroll
+    for (int q = 0; q < SB; ++q) {
+      const size_t row = ((size_t)bg * n_split + s0 + q) * R + r;
+      const bool ok = s0 + q < n_valid;
+      ml[q] = ok ? __ldcg(part.ml + row) : make_float2(-INFINITY, 0.0f);
+#pragma unroll
+      for (int c = 0; c < CPL; ++c)
+        ov[q][c] = (ok && O) ? __ldcg(part.o + row * D + lane + 32 * c) : 0.0f;
+    }
+    // merge this batch into the running (M, L, o), as the partials themselves
+    float Mb = M;
+#pragma unroll
+    for (int q = 0; q < SB; ++q) Mb = fmaxf(Mb, ml[q].x);
+    if (Mb == -INFINITY) continue;
+    const float a = M == -INFINITY ? 0.0f : expf(M - Mb);
+    L *= a;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) o[c] *= a;
+#pragma unroll
+    for (int q = 0; q < SB; ++q) {
+      // an empty run (m = -inf) wrote no output row: skip it, never 0 * garbage
+      if (ml[q].x == -INFINITY) continue;
+      const float wgt = expf(ml[q].x - Mb);
+      L += ml[q].y * wgt;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) o[c] = fmaf(ov[q][c], wgt, o[c]);
+    }
+    M = Mb;
+  }
+  if (O) {  // O == nullptr: the row LSEs only
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    T* dst = O + (((size_t)b * s.L_q + i) * s.H + h) * D;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) dst[lane + 32 * c] = from_f32<T>(o[c] * inv);
+  }
+  if (lse && lane == 0) lse[((size_t)b * s.H + h) * s.L_q + i] = L > 0.0f ? M + logf(L) : -INFINITY;
+}
+
 }  // namespace dl

@@ -150,8 +150,11 @@ class DenoiseStep:
     buffers are allocated once, so `run` can be captured in a CUDA graph."""
 
     def __init__(self, desc: A.dl_attn_desc, n_layers: int, first_sparse: int, topK: int,
-                 n_sinks: int, k: int, w: int, dtype: torch.dtype, device):
+                 n_sinks: int, k: int, w: int, dtype: torch.dtype, device, sink_group=None):
         self.desc, self.n_layers, self.first_sparse = desc, n_layers, first_sparse
+        # head-sharded: desc covers this rank's heads, and the sink mass is
+        # summed over sink_group before the sinks are picked (sharded.py)
+        self.sink_group = sink_group
         self.topK, self.n_sinks, self.k, self.w = topK, n_sinks, k, w
         B, L_q, d, H, H_kv = desc.batch, desc.L_q, desc.d, desc.H, desc.H_kv
         self.n_blk = -(-desc.L_ctx // desc.page)
@@ -162,6 +165,7 @@ class DenoiseStep:
         self.q_idx = _empty((B, L_q), torch.int32, device)
         self.q_cnt = _empty((B,), torch.int32, device)
         self.sink_pos = _empty((B, n_sinks), torch.int32, device)
+        self.mass = _empty((B, desc.L_ctx), torch.float32, device) if sink_group is not None else None
         self.score = _empty((B, H_kv, self.n_blk), torch.float64, device)
         self.blk_idx = [_empty((B, H_kv, self.max_sel), torch.int32, device)
                         for _ in range(n_layers)]
@@ -192,11 +196,14 @@ class DenoiseStep:
 
     def run(self, conf_prev, still_masked, q_dec: List, k_pool: List, v_pool: List,
             page_table, k_dec: List, v_dec: List, key_caches: List, stream=None,
-            attn_events: Optional[list] = None):
+            attn_events: Optional[list] = None, find_sinks: bool = True):
         """Launches the step on `stream`.  key_caches[l] = (Kbar, Kdig, Kexp)
-        of layer l (key_cache()).  If attn_events is a list, a pair of timing
-        events (recorded as graph nodes when captured) brackets every
-        attention call and (layer, start, end) is appended to it."""
+        of layer l (key_cache()).  find_sinks=False keeps the sinks found by
+        an earlier step (sink_pos): the later steps of one decode block reuse
+        the sinks of its first step, until the block is committed to the
+        cache.  If attn_events is a list, a pair of timing events (recorded as
+        graph nodes when captured) brackets every attention call and
+        (layer, start, end) is appended to it."""
         d = self.desc
         A.dl_predict_queries(conf_prev, still_masked, self.k, self.w, self.q_idx, self.q_cnt,
                              stream)
@@ -207,9 +214,8 @@ class DenoiseStep:
                                  k_dec[l], v_dec[l], self.O[l], self.lse[l], self.ws, stream)
                 self._end(attn_events, ev, l, stream)
                 continue
-            if l == self.first_sparse:
-                A.dl_find_sinks(d, q_dec[l], self.q_idx, self.q_cnt, k_pool[l], page_table,
-                                k_dec[l], self.n_sinks, self.sink_pos, self.ws, stream)
+            if l == self.first_sparse and find_sinks:
+                self._find_sinks(q_dec[l], k_pool[l], page_table, k_dec[l], stream)
             Kbar, Kdig, Kexp = key_caches[l]
             A.dl_block_select(d, q_dec[l], self.q_idx, self.q_cnt, Kbar, self.n_blk, d.page,
                               self.topK, self.sink_pos, self.score, self.blk_idx[l],
@@ -220,6 +226,17 @@ class DenoiseStep:
                              self.blk_cnt[l], k_dec[l], v_dec[l], self.O[l], self.lse[l],
                              self.ws, stream)
             self._end(attn_events, ev, l, stream)
+
+    def _find_sinks(self, q_dec, k_pool, page_table, k_dec, stream):
+        d = self.desc
+        if self.sink_group is None:
+            A.dl_find_sinks(d, q_dec, self.q_idx, self.q_cnt, k_pool, page_table, k_dec,
+                            self.n_sinks, self.sink_pos, self.ws, stream)
+            return
+        from .sharded import reduce_and_pick
+        A.dl_sink_mass(d, q_dec, self.q_idx, self.q_cnt, k_pool, page_table, k_dec, self.mass,
+                       self.ws, stream)
+        reduce_and_pick(self.mass, self.sink_pos, self.sink_group, stream=stream)
 
     @staticmethod
     def _begin(events, stream):

@@ -44,6 +44,12 @@ used (each is repeated at the function that applies it):
   R7 chunk path: chunk key = mean of its content tokens (BOS excluded); every
      decode query ranks chunks and tokens; the BOS of each selected chunk is
      always attended.
+  R8 sinks are found once per decode block, at the first step's first sparse
+     layer, and kept by every later step of the block: the pages keep sink
+     locations consistent (reused across layers, and the cached context they
+     index is unchanged until the block is written into the cache).
+  R9 over head shards the sink mass is the sum of the shards' partial masses,
+     each the R4 sum over that shard's heads only.
 """
 from .steps import (  # noqa: F401
     scale_for, predict_queries, pool_mean, pooled_keys, block_scores,
@@ -51,4 +57,6 @@ from .steps import (  # noqa: F401
     gather_context, chunk_pooled_keys, chunk_scores, token_select,
     chunk_attention, dense_attention, topk_lower_index, cache_write,
 )
-from .step import layer_step, chunked_step, StepResult, ChunkResult  # noqa: F401
+from .step import (  # noqa: F401
+    layer_step, chunked_step, denoise_block, StepResult, ChunkResult,
+)

@@ -120,6 +120,40 @@ def layer_step(q_dec, k_pool, v_pool, page_table, k_dec, v_dec, L_ctx: int, B: i
                       blk_idx=blk_idx, blk_cnt=blk_cnt, O=O, lse=lse, sink_mass=mass)
 
 
+def denoise_block(k_pool, v_pool, page_table, steps, L_ctx: int, B: int, topK: int, *,
+                  first_sparse: int, n_sinks: int, k: int = 4, w: int = 2):
+    """The denoising steps of one decode block over a multi-layer model
+    (reading R8).
+
+    k_pool / v_pool: per layer, the cached context, unchanged while the block
+    is decoded; steps: per step, a dict with conf_prev, still_masked and the
+    per-layer lists q_dec, k_dec, v_dec.  Every step predicts its own query
+    positions; layers below first_sparse attend densely; the first step finds
+    the n_sinks sinks at layer first_sparse, and every sparse layer of every
+    step keeps them (the cached context they index does not change before
+    the block is committed).  Returns, per step, the list of per-layer
+    StepResults."""
+    out = []
+    sinks = None
+    for t, st in enumerate(steps):
+        q_idx, q_cnt = predict_all(st["conf_prev"], st["still_masked"], k, w)
+        layers = []
+        for l in range(len(k_pool)):
+            args = (st["q_dec"][l], k_pool[l], v_pool[l], page_table, st["k_dec"][l],
+                    st["v_dec"][l], L_ctx, B, topK)
+            common = dict(q_idx=q_idx, q_cnt=q_cnt, k=k, w=w)
+            if l < first_sparse:
+                r = layer_step(*args, dense=True, **common)
+            elif l == first_sparse and t == 0:
+                r = layer_step(*args, detect_sinks=n_sinks, **common)
+                sinks = r.sink_pos
+            else:
+                r = layer_step(*args, sink_pos=sinks, **common)
+            layers.append(r)
+        out.append(layers)
+    return out
+
+
 @dataclasses.dataclass
 class ChunkResult:
     Kbar: np.ndarray       # fp64 (fp32 values) [batch][H_kv][n_chunks][d]

@@ -23,7 +23,8 @@ def test_header_declares_the_path():
     names = _declared()
     for n in ("dl_predict_queries", "dl_pool_keys", "dl_block_scores", "dl_find_sinks",
               "dl_select", "dl_block_select", "dl_sparse_attn", "dl_token_select",
-              "dl_sparse_attn_gather", "dl_cache_write", "dl_workspace_size", "dl_get_status"):
+              "dl_sparse_attn_gather", "dl_cache_write", "dl_workspace_size", "dl_get_status",
+              "dl_sink_mass", "dl_sink_topn"):
         assert n in names
 
 
@@ -106,6 +107,26 @@ def test_null_and_range_arguments_rejected_before_launch():
                              fake, None, 0, None)
     assert st == dl.DL_ERR_INVALID_ARG
 
+
+
+def test_split_sink_calls_rejected_before_launch():
+    lib = _abi.lib
+    d = _desc()
+    fake = ctypes.c_void_p(0x1000)
+    # the mass half: NULL mass, misaligned keys, workspace too small
+    assert lib.dl_sink_mass(ctypes.byref(d), fake, fake, fake, fake, fake, fake, None, fake,
+                            1 << 40, None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_sink_mass(ctypes.byref(d), fake, fake, fake, ctypes.c_void_p(0x1008), fake,
+                            fake, fake, fake, 1 << 40, None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_sink_mass(ctypes.byref(d), fake, fake, fake, fake, fake, fake, fake, fake,
+                            256, None) == dl.DL_ERR_WORKSPACE
+    # the top-n half: sizes and pointers
+    assert lib.dl_sink_topn(None, 1, 1024, 4, fake, None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_sink_topn(fake, 1, 1024, 4, None, None) == dl.DL_ERR_INVALID_ARG
+    for n_sinks in (0, 65):
+        assert lib.dl_sink_topn(fake, 1, 1024, n_sinks, fake, None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_sink_topn(fake, 0, 1024, 4, fake, None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_sink_topn(fake, 1, 0, 4, fake, None) == dl.DL_ERR_INVALID_ARG
 
 
 def test_cache_write_arguments_rejected_before_launch():

@@ -71,11 +71,12 @@ def test_digits_reconstruct_within_their_bound():
 
 CASES = [  # n_units, H, H_kv, L_q, cnts (predicted rows per sequence), topK, n_sinks
     (512, 4, 4, 32, [20, 15], 128, 4),    # the 32K layer's shape per (b, g)
-    (300, 4, 2, 32, [16, 20], 40, 2),     # ragged third tile, G = 2 (40 rows -> cut at bound)
+    (300, 4, 2, 32, [12, 10], 40, 2),     # ragged third tile, G = 2, 24 rows
     (128, 2, 2, 20, [20, 1], 30, 1),      # one tile, one row
-    (200, 8, 2, 32, [8, 3], 10, 0),       # G = 4, 32 rows, no sinks
+    (200, 8, 2, 32, [6, 3], 10, 0),       # G = 4, 24 rows, no sinks
     (512, 2, 2, 32, [0, 12], 64, 3),      # a sequence with no predicted rows
     (385, 3, 3, 16, [16, 9], 300, 2),     # four tiles, the last with one key; topK near n
+    (256, 2, 2, 32, [8, 8], 16, 1),       # one row block (8 rows)
 ]
 
 
@@ -84,9 +85,7 @@ def test_block_select_tc_matches_oracle(n_units, H, H_kv, L_q, cnts, topK, n_sin
     batch, d = len(cnts), 128
     G = H // H_kv
     max_q = max(cnts)
-    if G * max_q > 32:
-        max_q = 32 // G
-        cnts = [min(c, max_q) for c in cnts]
+    assert G * max_q <= 24  # the int8 kernel's row bound
     sid = 31000 + n_units + 7 * H + L_q
     q = synth.normals(SEED, sid, 0, batch * H * L_q * d).reshape(batch, H, L_q, d).to(
         torch.bfloat16)
@@ -117,6 +116,12 @@ def test_block_select_tc_matches_oracle(n_units, H, H_kv, L_q, cnts, topK, n_sin
     assert dl.dl_get_status() == dl.DL_OK
     fast, fallback = dl.dl_read_counters()
     assert fast + fallback == batch * H_kv
+    _check_against_oracle(q, kbar, q_idx, cnts, sinks, n_sinks, topK, H_kv, G, d, score, blk,
+                          cnt)
+
+
+def _check_against_oracle(q, kbar, q_idx, cnts, sinks, n_sinks, topK, H_kv, G, d, score, blk,
+                          cnt):
     got_s, got_b, got_c = np_(score), np_(blk), np_(cnt)
     scale = oracle.scale_for(d)
     for b, c in enumerate(cnts):
@@ -130,6 +135,39 @@ def test_block_select_tc_matches_oracle(n_units, H, H_kv, L_q, cnts, topK, n_sin
             assert got_c[b, g] == len(sel), (b, g)
             assert got_b[b, g, :len(sel)].tolist() == list(sel), (b, g)
             assert (got_b[b, g, len(sel):] == -1).all()
+
+
+def test_more_than_24_rows_take_the_fp64_kernel(cuda_device):
+    """25 .. 32 rows per group: the fused fp64 kernel (the int8 kernel holds at
+    most three row blocks), same results."""
+    n_units, H, H_kv, L_q, cnts, topK, n_sinks = 300, 8, 2, 32, [8, 7], 40, 2
+    batch, d, G = 2, 128, 4
+    sid = 31500
+    q = synth.normals(SEED, sid, 0, batch * H * L_q * d).reshape(batch, H, L_q, d).to(
+        torch.bfloat16)
+    kbar = (synth.normals(SEED, sid + 1, 0, batch * H_kv * n_units * d) / 8).to(
+        torch.float32).reshape(batch, H_kv, n_units, d)
+    q_idx = torch.full((batch, L_q), -1, dtype=torch.int32)
+    for b, c in enumerate(cnts):
+        keys = synth.uniforms(SEED, sid + 2 + b, 0, L_q)
+        q_idx[b, :c] = torch.sort(torch.argsort(keys)[:c]).values.to(torch.int32)
+    q_cnt = torch.tensor(cnts, dtype=torch.int32)
+    u = synth.uniforms(SEED, sid + 9, 0, batch * n_sinks)
+    sinks = (u * n_units * 64).to(torch.int32).reshape(batch, n_sinks)
+    kdig, kexp = _digits_on(cuda_device, kbar)
+    desc = _desc(batch, H, H_kv, d, L_q, n_units)
+    dev = lambda t: t.to(cuda_device)  # noqa: E731
+    score = torch.empty((batch, H_kv, n_units), dtype=torch.float64, device=cuda_device)
+    blk = torch.empty((batch, H_kv, topK + n_sinks), dtype=torch.int32, device=cuda_device)
+    cnt = torch.empty((batch, H_kv), dtype=torch.int32, device=cuda_device)
+    ws = torch.empty(max(dl.dl_workspace_size(desc), 256), dtype=torch.uint8, device=cuda_device)
+    dl.dl_read_counters()
+    dl.dl_block_select(desc, dev(q), dev(q_idx), dev(q_cnt), dev(kbar), n_units, 64, topK,
+                       dev(sinks), score, blk, cnt, ws, max_q=8, Kdig=kdig, Kexp=kexp)
+    assert dl.dl_get_status() == dl.DL_OK
+    assert dl.dl_read_counters() == (0, 0)
+    _check_against_oracle(q, kbar, q_idx, cnts, sinks, n_sinks, topK, H_kv, G, d, score, blk,
+                          cnt)
 
 
 def test_near_ties_fall_back_to_fp64(cuda_device):

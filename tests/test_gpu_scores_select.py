@@ -3,7 +3,10 @@ through the C ABI, at unit counts that span several 128-unit score tiles
 with a ragged tail, query-row counts that need several 32-row passes, and
 selection sizes that reach each of the selection kernels (one key per
 thread up to 1024 units, the shared-memory network up to 4096, the rank
-count beyond), with tied scores and duplicate sinks."""
+count beyond), with tied scores and duplicate sinks; the fused score +
+select call on each of its kernels (fp64 MMA for up to 32 rows, the wide
+CUDA-core kernel for more rows over at most 128 units, the separate kernels
+beyond)."""
 import numpy as np
 import pytest
 import torch
@@ -109,9 +112,12 @@ def test_select_all_paths(n_units, topK, cuda_device):
     (200, 4, 4, 128, 32, [32, 5], 300, "fp32"),       # fp32 queries, topK beyond the candidates
     (513, 4, 4, 128, 32, [20, 9], 64, "bf16"),        # separate kernels: more than 512 keys
     (100, 8, 2, 128, 32, [20, 32], 10, "bf16"),       # separate kernels: 4 x 32 rows
-    (32, 8, 8, 128, 64, [64, 13], 8, "bf16"),         # separate kernels: few units, 64 rows
-    (128, 8, 4, 64, 40, [40, 1], 20, "fp32"),         # 128 units, 80 rows, d 64, fp32
-    (7, 4, 2, 128, 48, [48, 0], 3, "bf16"),           # 96 rows over 7 units, a sequence with none
+    (32, 8, 8, 128, 64, [64, 13], 8, "bf16"),         # wide kernel: few units, 64 rows
+    (128, 8, 4, 64, 40, [40, 1], 20, "fp32"),         # separate: 80 rows x 128 units > 8192
+    (7, 4, 2, 128, 48, [48, 0], 3, "bf16"),           # wide: 96 rows over 7 units, a sequence with none
+    (20, 8, 1, 128, 32, [32, 11], 5, "fp32"),         # wide: 256 rows (G = 8), fp32, d 128
+    (128, 4, 4, 128, 64, [64, 64], 30, "bf16"),       # wide: 64 rows x 128 units = 8192
+    (33, 6, 2, 64, 40, [40, 23], 33, "bf16"),         # wide: ragged units, topK = all, d 64
 ])
 @pytest.mark.parametrize("tight", [False, True])
 def test_block_select_matches_oracle(n_units, H, H_kv, d, L_q, cnts, topK, dtype, tight,

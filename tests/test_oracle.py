@@ -445,3 +445,79 @@ def test_cache_write_closed_forms_and_untouched_rows():
         v = V2[row[t // B], 0, t % B]
         new = start <= t < start + n
         assert np.all(k == (6.0 if new else 2.0)) and np.all(v == (7.0 if new else -1.0))
+
+
+# ------------------------------------------------- sinks across a decode block
+def _block_inputs(wl, n_layers, seeds):
+    """Cached context of seed seeds[0] (unchanged over the block); the
+    decode-block tensors and confidences of each step from its own seed."""
+    import synth
+    ctx = [synth.make_step_inputs(wl, layer=l) for l in range(n_layers)]
+    steps = []
+    for sd in seeds:
+        xs = [synth.make_step_inputs(wl.replace(seed=sd), layer=l) for l in range(n_layers)]
+        steps.append(dict(conf_prev=xs[0].conf_prev, still_masked=xs[0].still_masked,
+                          q_dec=[x.q_dec for x in xs], k_dec=[x.k_dec for x in xs],
+                          v_dec=[x.v_dec for x in xs]))
+    return ctx, steps
+
+
+def test_denoise_block_keeps_first_step_sinks():
+    """R8: the later steps keep the first step's sinks, not sinks found anew
+    from their own queries (which differ here), and every sparse layer of
+    every step selects the sink blocks."""
+    import synth
+    wl = synth.workload("tiny", batch=2, H=4, H_kv=2, L_ctx=1024, n_layers=3, topK=3)
+    ctx, steps = _block_inputs(wl, 3, [0, 7])
+    res = oracle.denoise_block([x.k_pool for x in ctx], [x.v_pool for x in ctx],
+                               ctx[0].page_table, steps, wl.L_ctx, wl.B, wl.topK,
+                               first_sparse=1, n_sinks=4, k=wl.k, w=wl.w)
+    s0 = res[0][1].sink_pos
+    fresh = []
+    for b in range(wl.batch):
+        Kc = np.stack([S.gather_context(S.f64(ctx[1].k_pool), ctx[1].page_table[b].numpy(), g,
+                                        np.arange(wl.L_ctx), wl.B) for g in range(wl.H_kv)])
+        q_idx, q_cnt = res[1][1].q_idx[b], res[1][1].q_cnt[b]
+        top, _ = S.find_sinks(steps[1]["q_dec"][1][b], Kc, steps[1]["k_dec"][1][b],
+                              q_idx[:q_cnt], 4, S.scale_for(wl.d))
+        fresh.append(top)
+    assert not np.array_equal(np.stack(fresh), s0), "inputs do not tell the readings apart"
+    for t, layers in enumerate(res):
+        # the dense layer selects every block
+        assert np.all(layers[0].blk_cnt == wl.n_blk)
+        for r in layers[1:]:
+            assert np.array_equal(r.sink_pos, s0)
+            for b in range(wl.batch):
+                sink_blocks = set((s0[b] // wl.B).tolist())
+                for g in range(wl.H_kv):
+                    sel = set(r.blk_idx[b, g, : r.blk_cnt[b, g]].tolist())
+                    assert sink_blocks <= sel
+                    # the rest are the topK highest-scoring non-sink blocks
+                    rest = [j for j in np.argsort(-r.score[b, g], kind="stable")
+                            if j not in sink_blocks][: wl.topK]
+                    assert sel == sink_blocks | set(rest)
+    # each step predicts its own queries
+    assert not np.array_equal(res[0][1].q_idx, res[1][1].q_idx)
+
+
+def test_head_shard_masses_sum_to_the_whole():
+    """R9: the sink mass over all heads is the sum of the per-shard masses
+    (any split of the KV heads), computed per head with torch's fp64
+    softmax."""
+    r = np.random.default_rng(5)
+    H, H_kv, L_ctx, L_q, d = 6, 3, 40, 8, 16
+    Q = r.standard_normal((H, L_q, d))
+    Kc = r.standard_normal((H_kv, L_ctx, d))
+    Kd = r.standard_normal((H_kv, L_q, d))
+    rows = np.array([1, 2, 5])
+    scale = S.scale_for(d)
+    G = H // H_kv
+    want = torch.zeros(L_ctx, dtype=torch.float64)
+    for h in range(H):
+        keys = torch.from_numpy(np.concatenate([Kc[h // G], Kd[h // G]]))
+        p = torch.softmax(scale * torch.from_numpy(Q[h, rows]) @ keys.T, dim=-1)
+        want += p[:, :L_ctx].sum(0)
+    for split in ([0, 1, 3], [0, 2, 3], [0, 1, 2, 3]):
+        parts = [S.find_sinks(Q[a * G:b * G], Kc[a:b], Kd[a:b], rows, 2, scale)[1]
+                 for a, b in zip(split, split[1:])]
+        assert np.allclose(sum(parts), want.numpy(), rtol=1e-13, atol=0)
