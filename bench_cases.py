@@ -64,7 +64,7 @@ def main():
     if args.fp64_select:
         A.dl_set_kernel_flags(A.DL_FLAG_SCORE_FP64)
     sinks = torch.empty((wl.batch, wl.detect_sinks), dtype=torch.int32, device=dev)
-    A.dl_find_sinks(desc, q, q_idx, q_cnt, kp, pt, kd, wl.detect_sinks, sinks, ws)
+    A.dl_find_sinks(desc, q, q_idx, q_cnt, kp, pt, kd, wl.detect_sinks, sinks, ws, Kexp=Kexp)
     max_sel = min(wl.topK, wl.n_blk) + wl.detect_sinks
     score = torch.empty((wl.batch, wl.H_kv, wl.n_blk), dtype=torch.float64, device=dev)
     blk = torch.empty((wl.batch, wl.H_kv, max_sel), dtype=torch.int32, device=dev)
@@ -87,7 +87,7 @@ def main():
         "pool": lambda: A.dl_pool_keys(desc, kp, pt, wl.n_blk, wl.B, 0, wl.B, Kbar, Kdig=Kdig,
                                        Kexp=Kexp),
         "sinks": lambda: A.dl_find_sinks(desc, q, q_idx, q_cnt, kp, pt, kd, wl.detect_sinks,
-                                         sinks, ws),
+                                         sinks, ws, Kexp=Kexp),
     }
     if args.case.startswith("attn"):
         block_select()

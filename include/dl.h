@@ -204,11 +204,20 @@ dl_status dl_block_scores(const dl_attn_desc* desc, const void* Q_dec, const int
  * sink_pos[b] = the n_sinks columns of largest mass (ties -> lower index),
  * ascending.  Computed once, at the first sparse layer, and passed unchanged
  * to dl_select of every deeper layer.
+ *   Kexp  int32 [batch][H_kv][ceil(L_ctx / page)] or NULL: the exponent words
+ *         that dl_pool_keys (unit = page) or dl_cache_write wrote for this
+ *         layer's current K pool; their norm field bounds every key's norm.
+ *         Given, the cut is certified: the masses are taken in fp32, and
+ *         where a proven bound on their error does not separate the n-th
+ *         largest from the next, the undecided columns (or, past 512 of
+ *         them, every column) get their masses again in fp64 and the sinks
+ *         are those of the fp64 masses (exact up to fp64 rounding).  NULL:
+ *         the top n of the fp32 masses (relative error about 1e-6).
  *   sink_pos int32 [batch][n_sinks]  (out);  1 <= n_sinks <= 64 */
 dl_status dl_find_sinks(const dl_attn_desc* desc, const void* Q_dec, const int32_t* q_idx,
                         const int32_t* q_cnt, const void* K_pool, const int32_t* page_table,
-                        const void* K_dec, int n_sinks, int32_t* sink_pos, void* ws,
-                        size_t ws_bytes, void* stream);
+                        const void* K_dec, const int32_t* Kexp, int n_sinks, int32_t* sink_pos,
+                        void* ws, size_t ws_bytes, void* stream);
 
 /* (a4), split in its two halves for head-sharded execution.  The sink mass
  * is a sum over heads, so a GPU that holds only some KV heads (desc->H_kv
@@ -219,6 +228,8 @@ dl_status dl_find_sinks(const dl_attn_desc* desc, const void* Q_dec, const int32
  * what dl_find_sinks gives.
  * dl_sink_mass: mass fp32 [batch][L_ctx] (out, device; every element
  *   written); the same arguments, checks and workspace as dl_find_sinks.
+ *   The split calls take the top n of the fp32 sum without the certified
+ *   recheck of dl_find_sinks.
  * dl_sink_topn: mass fp32 [batch][L_ctx] (device; in, and scratch when
  *   n_sinks > 8: the chosen columns are overwritten with -inf);
  *   sink_pos int32 [batch][n_sinks] (out), the n_sinks columns of largest

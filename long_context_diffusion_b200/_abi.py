@@ -52,8 +52,8 @@ _SIGS = {
                         _vp, _vp, _vp], _c_int),
     "dl_block_scores": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _c_int, _vp, _vp,
                          ctypes.c_size_t, _vp], _c_int),
-    "dl_find_sinks": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp,
-                       _vp, ctypes.c_size_t, _vp], _c_int),
+    "dl_find_sinks": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int,
+                       _vp, _vp, ctypes.c_size_t, _vp], _c_int),
     "dl_select": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _vp, _c_int,
                    _vp], _c_int),
     "dl_sink_mass": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -176,9 +176,11 @@ def dl_block_scores(desc, Q_dec, q_idx, q_cnt, Kbar, n_units, score, ws, stream=
 
 
 def dl_find_sinks(desc, Q_dec, q_idx, q_cnt, K_pool, page_table, K_dec, n_sinks, sink_pos, ws,
-                  stream=None):
+                  stream=None, Kexp=None):
+    """Kexp: the layer's key exponent words (key_digit_buffers, filled by
+    dl_pool_keys / dl_cache_write); given, the sink cut is certified."""
     _check(lib.dl_find_sinks(ctypes.byref(desc), _p(Q_dec), _p(q_idx), _p(q_cnt), _p(K_pool),
-                             _p(page_table), _p(K_dec), n_sinks, _p(sink_pos), _p(ws),
+                             _p(page_table), _p(K_dec), _p(Kexp), n_sinks, _p(sink_pos), _p(ws),
                              ws.numel() * ws.element_size(), _s(stream)))
 
 

@@ -245,8 +245,8 @@ dl_status dl_block_scores(const dl_attn_desc* desc, const void* Q_dec, const int
 
 dl_status dl_find_sinks(const dl_attn_desc* desc, const void* Q_dec, const int32_t* q_idx,
                         const int32_t* q_cnt, const void* K_pool, const int32_t* page_table,
-                        const void* K_dec, int n_sinks, int32_t* sink_pos, void* ws,
-                        size_t ws_bytes, void* stream) {
+                        const void* K_dec, const int32_t* Kexp, int n_sinks, int32_t* sink_pos,
+                        void* ws, size_t ws_bytes, void* stream) {
   dl::Shape s;
   dl_status st = check_desc(desc, &s);
   if (st != DL_OK) return st;
@@ -259,8 +259,8 @@ dl_status dl_find_sinks(const dl_attn_desc* desc, const void* Q_dec, const int32
   if ((st = need_ws(ws, ws_bytes, dl::sinks_workspace(s))) != DL_OK) return st;
   unsigned* err = nullptr;
   if ((st = error_word(&err)) != DL_OK) return st;
-  return launched(dl::launch_sinks(s, Q_dec, q_idx, q_cnt, K_pool, page_table, K_dec, n_sinks,
-                                   sink_pos, ws, err, as_stream(stream)),
+  return launched(dl::launch_sinks(s, Q_dec, q_idx, q_cnt, K_pool, page_table, K_dec, Kexp,
+                                   n_sinks, sink_pos, ws, err, as_stream(stream)),
                   "dl_find_sinks launch");
 }
 

@@ -386,7 +386,7 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
     if (key_ok) {
       Eu = max(ke & 255, 1);
       em = Eu;
-      nk = ke >> 8;
+      nk = (ke >> 8) & 255;
     }
     em = __reduce_max_sync(0xffffffffu, em);
     nk = __reduce_max_sync(0xffffffffu, nk);

@@ -39,6 +39,7 @@ cache_write_kernel(Shape s, const T* __restrict__ K_new, const T* __restrict__ V
   constexpr int RG = kCwThreads / TPR;   // row groups
   constexpr int B = 64;                  // positions per block (= page)
   __shared__ double s_sum[RG][D];
+  __shared__ float s_sq[RG][TPR];  // per row group and chunk: max sum of squares
   const int bg = blockIdx.y;
   const int b = bg / s.H_kv, g = bg % s.H_kv;
   const int tid = threadIdx.x, c = tid % TPR, rg = tid / TPR;
@@ -58,6 +59,7 @@ cache_write_kernel(Shape s, const T* __restrict__ K_new, const T* __restrict__ V
   double acc[EPT];
 #pragma unroll
   for (int e = 0; e < EPT; ++e) acc[e] = 0.0;
+  float sq_max = 0.0f;
 #pragma unroll
   for (int r = rg; r < B; r += RG) {
     const int p = j * B + r;
@@ -89,9 +91,14 @@ cache_write_kernel(Shape s, const T* __restrict__ K_new, const T* __restrict__ V
     }
 #pragma unroll
     for (int e = 0; e < EPT; ++e) acc[e] += (double)v[e];
+    float q = 0.0f;
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) q = __fmaf_rn(v[e], v[e], q);
+    sq_max = fmaxf(sq_max, q);
   }
 #pragma unroll
   for (int e = 0; e < EPT; ++e) s_sum[rg][c * EPT + e] = acc[e];
+  s_sq[rg][c] = sq_max;
   __syncthreads();
   const int n_blk = (s.L_ctx + B - 1) / B;
   float mean = 0.0f;
@@ -128,7 +135,14 @@ cache_write_kernel(Shape s, const T* __restrict__ K_new, const T* __restrict__ V
   if (tid == 0) {
     int n = 0;
     for (int w = 0; w < D / 32; ++w) n += s_n[w];
-    Kexp[(size_t)bg * n_blk + j] = E | (n << 8);
+    // norm bound: per chunk the max over the row groups, added in chunk order
+    float sq_sum = 0.0f;
+    for (int q = 0; q < TPR; ++q) {
+      float m = 0.0f;
+      for (int r = 0; r < RG; ++r) m = fmaxf(m, s_sq[r][q]);
+      sq_sum += m;
+    }
+    Kexp[(size_t)bg * n_blk + j] = E | (n << 8) | key_norm_field(sq_sum);
   }
 }
 

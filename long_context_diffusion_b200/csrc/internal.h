@@ -97,8 +97,15 @@ cudaError_t launch_sink_topn_mass(float* mass, int batch, int L_ctx, int n_sinks
                                   int32_t* sink_pos, cudaStream_t st);
 cudaError_t launch_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
                          const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
-                         const void* Kd, int n_sinks, int32_t* sink_pos, void* ws,
-                         unsigned* err, cudaStream_t st);
+                         const void* Kd, const int32_t* Kexp, int n_sinks, int32_t* sink_pos,
+                         void* ws, unsigned* err, cudaStream_t st);
+size_t sink_cert_workspace(const Shape& s);
+bool sink_cert_supported(const Shape& s, int n_sinks);
+cudaError_t launch_sink_cert(const Shape& s, const void* Q, const int32_t* q_idx,
+                             const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
+                             const void* Kd, const int32_t* Kexp, int n_units, const float* mass,
+                             int n_sinks, int32_t* sink_pos, void* ws, unsigned* err,
+                             cudaStream_t st);
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
 

@@ -20,6 +20,12 @@
 // Device layouts written by dl_pool_keys / dl_cache_write:
 //   Kdig int8  [b][g][kKeyDigits][n_units][d]   digit plane t of every unit
 //   Kexp int32 [b][g][n_units]                  E | (inexact values << 8)
+//                                               | (norm bound << 16)
+// The norm bound is the bf16 bit pattern of an upper bound of the largest
+// Euclidean norm of the unit's pooled key rows, max_t ||k_t||_2 (rounded up;
+// the sink search bounds its fp32 logits with it).  It is computed as
+// sqrt(sum_c max_t s_tc) with s_tc the sum of squares of row t's 16-byte
+// column chunk c, which is at least max_t sum_c s_tc.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -75,6 +81,19 @@ __device__ __forceinline__ bool query_digits(uint32_t h, int E, int (&dg)[kQuery
   dg[2] = (sv >> 7) & 127;
   dg[3] = sv & 127;
   return inexact;
+}
+
+// The Kexp norm field from sum_c max_t s_tc (fp32 sums of squares, chunk
+// sums added in chunk order): the fp32 rounding of the squares, of the sums
+// and of the square root is covered by the factor 1 + 2^-14 on the sum, and
+// the result is rounded up to bf16.
+__device__ __forceinline__ int key_norm_field(float sq_sum) {
+  const float n = sqrtf(sq_sum * (1.0f + 0x1p-14f));
+  return (int)__bfloat16_as_ushort(__float2bfloat16_ru(n)) << 16;
+}
+// The norm bound a Kexp word holds.
+__device__ __forceinline__ float key_norm_of(int kexp) {
+  return __bfloat162float(__ushort_as_bfloat16((unsigned short)((unsigned)kexp >> 16)));
 }
 
 __device__ __forceinline__ uint32_t pack4_i8(int a, int b, int c, int d) {

@@ -45,6 +45,14 @@ pool_kernel(const T* __restrict__ Kp, const int32_t* __restrict__ page_table, Sh
   double acc[EPT];
 #pragma unroll
   for (int e = 0; e < EPT; ++e) acc[e] = 0.0;
+  float sq_max = 0.0f;  // max over the rows of this chunk's sum of squares
+  const bool norms = Kdig != nullptr;
+  auto sq = [](const float(&v)[EPT]) {
+    float q = 0.0f;
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) q = __fmaf_rn(v[e], v[e], q);
+    return q;
+  };
   for (long long t = lo; t < hi;) {
     const int lp = (int)(t / s.page);
     const int row0 = (int)(t % s.page);
@@ -65,12 +73,17 @@ pool_kernel(const T* __restrict__ Kp, const int32_t* __restrict__ page_table, Sh
       for (int q = 0; q < 8; ++q)
 #pragma unroll
         for (int e = 0; e < EPT; ++e) acc[e] += (double)v[q][e];
+      if (norms) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) sq_max = fmaxf(sq_max, sq(v[q]));
+      }
     }
     for (; r < rows; ++r) {
       float v[EPT];
       Vec16<T>::load(src + (size_t)r * D, v);
 #pragma unroll
       for (int e = 0; e < EPT; ++e) acc[e] += (double)v[e];
+      if (norms) sq_max = fmaxf(sq_max, sq(v));
     }
   }
   const long long n = hi > lo ? hi - lo : 0;
@@ -94,6 +107,11 @@ pool_kernel(const T* __restrict__ Kp, const int32_t* __restrict__ page_table, Sh
   for (int e = 0; e < EPT; ++e) inexact += key_digits(mean[e], E, dg[e]) ? 1 : 0;
 #pragma unroll
   for (int o = 1; o < TPR; o <<= 1) inexact += __shfl_xor_sync(0xffffffffu, inexact, o);
+  // norm bound: the chunks' maxima added in chunk order (as dl_cache_write)
+  const int lane0 = (threadIdx.x & 31) & ~(TPR - 1);
+  float sq_sum = 0.0f;
+#pragma unroll
+  for (int q = 0; q < TPR; ++q) sq_sum += __shfl_sync(0xffffffffu, sq_max, lane0 + q);
   if (!active) return;
 #pragma unroll
   for (int t = 0; t < kKeyDigits; ++t) {
@@ -106,7 +124,7 @@ pool_kernel(const T* __restrict__ Kp, const int32_t* __restrict__ page_table, Sh
       *reinterpret_cast<uint32_t*>(plane) = pack4_i8(dg[0][t], dg[1][t], dg[2][t], dg[3][t]);
     }
   }
-  if (c == 0) Kexp[(size_t)bg * n_units + u] = E | (inexact << 8);
+  if (c == 0) Kexp[(size_t)bg * n_units + u] = E | (inexact << 8) | key_norm_field(sq_sum);
 }
 
 cudaError_t launch_pool(const Shape& s, const void* Kp, const int32_t* page_table, int n_units,

@@ -68,7 +68,8 @@ static SinkTcWs sink_tc_ws(void* ws, const Shape& s) {
   return w;
 }
 
-size_t sinks_workspace(const Shape& s) {
+// [mass-pass workspace (CUDA-core or tensor-core layout)][certified cut]
+static size_t sinks_mass_workspace(const Shape& s) {
   const size_t simt = round256((size_t)s.batch * s.H * sink_tiles(s) * s.L_q * sizeof(float2)) +
                       round256((size_t)s.batch * s.H * s.L_q * sizeof(float)) +
                       round256((size_t)s.batch * s.L_ctx * sizeof(float));
@@ -77,6 +78,8 @@ size_t sinks_workspace(const Shape& s) {
                     round256((size_t)s.batch * s.L_ctx * sizeof(float));
   return simt > tc ? simt : tc;
 }
+
+size_t sinks_workspace(const Shape& s) { return sinks_mass_workspace(s) + sink_cert_workspace(s); }
 
 // Loads key row `t` of KV head g (context t < L_ctx, else decode key t-L_ctx)
 // into k[]; returns false when the row holds no key.
@@ -452,14 +455,20 @@ cudaError_t launch_sink_topn_mass(float* mass, int batch, int L_ctx, int n_sinks
   return launch_sink_topn(s, n_sinks, w, sink_pos, st);
 }
 
+// With Kexp (the norm bounds of this layer's pooled keys) the cut is
+// certified (sinks_cert.cu); without it, the top-n of the fp32 masses.
 cudaError_t launch_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
                          const int32_t* q_cnt, const void* Kp, const int32_t* page_table,
-                         const void* Kd, int n_sinks, int32_t* sink_pos, void* ws,
-                         unsigned* err, cudaStream_t st) {
+                         const void* Kd, const int32_t* Kexp, int n_sinks, int32_t* sink_pos,
+                         void* ws, unsigned* err, cudaStream_t st) {
   const bool tc = s.dtype == 0 && s.G * s.L_q <= 256;
   float* mass = tc ? sink_tc_ws(ws, s).mass : sink_ws(ws, s).mass;
   cudaError_t e = launch_sink_mass(s, Q, q_idx, q_cnt, Kp, page_table, Kd, mass, ws, err, st);
   if (e != cudaSuccess) return e;
+  if (Kexp && sink_cert_supported(s, n_sinks))
+    return launch_sink_cert(s, Q, q_idx, q_cnt, Kp, page_table, Kd, Kexp,
+                            (s.L_ctx + s.page - 1) / s.page, mass, n_sinks, sink_pos,
+                            reinterpret_cast<char*>(ws) + sinks_mass_workspace(s), err, st);
   return launch_sink_topn_mass(mass, s.batch, s.L_ctx, n_sinks, sink_pos, st);
 }
 

@@ -79,7 +79,7 @@ def layer_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec, v
     if detect_sinks:
         sink_pos = _empty((B, detect_sinks), torch.int32, dev)
         A.dl_find_sinks(desc, q_dec, q_idx, q_cnt, k_pool, page_table, k_dec, detect_sinks,
-                        sink_pos, ws, stream)
+                        sink_pos, ws, stream, Kexp=Kexp)
     n_s = 0 if sink_pos is None else sink_pos.shape[-1]
     max_sel = min(topK, n_blk) + n_s
     blk_idx = _empty((B, H_kv, max(max_sel, 1)), torch.int32, dev)
@@ -215,7 +215,8 @@ class DenoiseStep:
                 self._end(attn_events, ev, l, stream)
                 continue
             if l == self.first_sparse and find_sinks:
-                self._find_sinks(q_dec[l], k_pool[l], page_table, k_dec[l], stream)
+                self._find_sinks(q_dec[l], k_pool[l], page_table, k_dec[l], key_caches[l][2],
+                                 stream)
             Kbar, Kdig, Kexp = key_caches[l]
             A.dl_block_select(d, q_dec[l], self.q_idx, self.q_cnt, Kbar, self.n_blk, d.page,
                               self.topK, self.sink_pos, self.score, self.blk_idx[l],
@@ -227,11 +228,11 @@ class DenoiseStep:
                              self.ws, stream)
             self._end(attn_events, ev, l, stream)
 
-    def _find_sinks(self, q_dec, k_pool, page_table, k_dec, stream):
+    def _find_sinks(self, q_dec, k_pool, page_table, k_dec, Kexp, stream):
         d = self.desc
         if self.sink_group is None:
             A.dl_find_sinks(d, q_dec, self.q_idx, self.q_cnt, k_pool, page_table, k_dec,
-                            self.n_sinks, self.sink_pos, self.ws, stream)
+                            self.n_sinks, self.sink_pos, self.ws, stream, Kexp=Kexp)
             return
         from .sharded import reduce_and_pick
         A.dl_sink_mass(d, q_dec, self.q_idx, self.q_cnt, k_pool, page_table, k_dec, self.mass,

@@ -77,3 +77,28 @@ def key_digits_np(kbar):
     kdig = np.stack(digs, axis=-2).astype(np.int8)   # [..., 5, d]
     kexp = (E[..., 0] | (inexact.sum(axis=-1) << 8)).astype(np.int32)
     return kdig, kexp
+
+
+def check_norm_field(kexp, k_pool, page_table, L_ctx, B):
+    """The norm field (bits 16-31, bf16) of every Kexp word: at least the
+    largest Euclidean norm of the block's key rows (fp64 on the host), and at
+    most the documented quantity sqrt(sum over 16-byte column chunks of the
+    largest sum of squares in the chunk) by more than bf16 rounding plus the
+    stated fp32 allowance."""
+    kexp = np.asarray(kexp)
+    bits = ((kexp.astype(np.int64) >> 16) & 0xFFFF).astype(np.uint32) << 16
+    bound = bits.view(np.float32).astype(np.float64)
+    K = np.asarray(torch.as_tensor(k_pool).to(torch.float64))
+    pt = np.asarray(page_table).astype(np.int64)
+    batch, H_kv, n_blk = kexp.shape
+    d = K.shape[-1]
+    ept = 8 if torch.as_tensor(k_pool).dtype == torch.bfloat16 else 4
+    for b in range(batch):
+        for g in range(H_kv):
+            for j in range(n_blk):
+                n = min(B, L_ctx - j * B)
+                rows = K[pt[b, j], g, :n]
+                true = np.sqrt((rows ** 2).sum(axis=1)).max()
+                chunk = (rows ** 2).reshape(n, d // ept, ept).sum(axis=2).max(axis=0).sum()
+                assert bound[b, g, j] >= true, (b, g, j)
+                assert bound[b, g, j] <= np.sqrt(chunk) * (1 + 2 ** -6), (b, g, j)

@@ -13,7 +13,7 @@ import torch
 import long_context_diffusion_b200 as dl
 import oracle
 import synth
-from tests.helpers import key_digits_np, np_
+from tests.helpers import check_norm_field, key_digits_np, np_
 
 pytestmark = pytest.mark.gpu
 
@@ -46,7 +46,9 @@ def test_pool_writes_key_digits(dtype, d, cuda_device):
     assert dl.dl_get_status() == dl.DL_OK
     ref_dig, ref_exp = key_digits_np(kbar.cpu().numpy())
     assert np.array_equal(kdig.cpu().numpy(), np.moveaxis(ref_dig, -2, 2))
-    assert np.array_equal(kexp.cpu().numpy(), ref_exp)
+    assert np.array_equal(kexp.cpu().numpy() & 0xFFFF, ref_exp)
+    check_norm_field(kexp.cpu().numpy(), inp.k_pool.cpu(), inp.page_table.cpu(), wl.L_ctx,
+                     wl.B)
 
 
 def test_digits_reconstruct_within_their_bound():
@@ -272,7 +274,13 @@ def test_cache_write_updates_key_digits(cuda_device):
     assert dl.dl_get_status() == dl.DL_OK
     ref_dig, ref_exp = key_digits_np(kbar.cpu().numpy())
     assert np.array_equal(kdig.cpu().numpy(), np.moveaxis(ref_dig, -2, 2))
-    assert np.array_equal(kexp.cpu().numpy(), ref_exp)
+    assert np.array_equal(kexp.cpu().numpy() & 0xFFFF, ref_exp)
+    check_norm_field(kexp.cpu().numpy(), K_dev.cpu(), page_table, L_ctx, page)
+    # the cache write's words equal a fresh pooling of the updated pool's
+    kbar2 = torch.empty_like(kbar)
+    kdig2, kexp2 = dl.key_digit_buffers(batch, H_kv, n_pages, d, cuda_device)
+    dl.dl_pool_keys(desc, K_dev, pt, n_pages, page, 0, page, kbar2, Kdig=kdig2, Kexp=kexp2)
+    assert torch.equal(kexp2, kexp)
     after = kdig.cpu().numpy()
     touched = {0: {1, 2}, 1: {9}}
     for b in range(batch):

@@ -2,6 +2,8 @@
 same seeded inputs.  Index outputs (predicted positions, pooled keys, block
 and token selections, sinks) must match exactly; attention outputs within
 the stated tolerances."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -52,25 +54,44 @@ def test_single_layer_workloads(name, cuda_device):
     _compare_layer(out, ref, wl.dtype == "fp32", name)
 
 
+def _key_exps(wl, desc, inp, dev):
+    """The layer's pooled-key exponent words (with their norm bounds)."""
+    Kbar = torch.empty((wl.batch, wl.H_kv, wl.n_blk, wl.d), dtype=torch.float32, device=dev)
+    Kdig, Kexp = dl.key_digit_buffers(wl.batch, wl.H_kv, wl.n_blk, wl.d, dev)
+    dl.dl_pool_keys(desc, inp.k_pool, inp.page_table, wl.n_blk, wl.B, 0, wl.B, Kbar, Kdig=Kdig,
+                    Kexp=Kexp)
+    return Kexp
+
+
+def _oracle_sinks(wl, inp, q_idx, q_cnt, n, b):
+    Kc = np.stack([S.gather_context(np_(inp.k_pool), np_(inp.page_table)[b], g,
+                                    np.arange(wl.L_ctx), wl.B) for g in range(wl.H_kv)])
+    qi, qc = np_(q_idx), np_(q_cnt)
+    return S.find_sinks(np_(inp.q_dec)[b], Kc, np_(inp.k_dec)[b], qi[b, : qc[b]], n,
+                        S.scale_for(wl.d))
+
+
+def _find(wl, inp, dev, n, certified=True):
+    desc = desc_for(wl)
+    q_idx = torch.empty((wl.batch, wl.L_q), dtype=torch.int32, device=dev)
+    q_cnt = torch.empty((wl.batch,), dtype=torch.int32, device=dev)
+    dl.dl_predict_queries(inp.conf_prev, inp.still_masked, wl.k, wl.w, q_idx, q_cnt)
+    ws = pipeline.workspace(desc, dev)
+    sinks = torch.full((wl.batch, n), -7, dtype=torch.int32, device=dev)
+    Kexp = _key_exps(wl, desc, inp, dev) if certified else None
+    dl.dl_find_sinks(desc, inp.q_dec, q_idx, q_cnt, inp.k_pool, inp.page_table, inp.k_dec, n,
+                     sinks, ws, Kexp=Kexp)
+    assert dl.dl_get_status() == dl.DL_OK
+    return sinks, q_idx, q_cnt
+
+
 @pytest.mark.parametrize("name", ["llada8k", "dream16k"])
 def test_find_sinks_recovers_planted(name, cuda_device):
     wl = synth.workload(name)
     inp = synth.make_step_inputs(wl, device=cuda_device)
-    desc = desc_for(wl)
-    q_idx = torch.empty((wl.batch, wl.L_q), dtype=torch.int32, device=cuda_device)
-    q_cnt = torch.empty((wl.batch,), dtype=torch.int32, device=cuda_device)
-    dl.dl_predict_queries(inp.conf_prev, inp.still_masked, wl.k, wl.w, q_idx, q_cnt)
-    ws = pipeline.workspace(desc, cuda_device)
-    sinks = torch.empty((wl.batch, 4), dtype=torch.int32, device=cuda_device)
-    dl.dl_find_sinks(desc, inp.q_dec, q_idx, q_cnt, inp.k_pool, inp.page_table, inp.k_dec, 4,
-                     sinks, ws)
-    assert dl.dl_get_status() == dl.DL_OK
-    qi, qc = np_(q_idx), np_(q_cnt)
+    sinks, q_idx, q_cnt = _find(wl, inp, cuda_device, 4)
     for b in range(wl.batch):
-        Kc = np.stack([S.gather_context(np_(inp.k_pool), np_(inp.page_table)[b], g,
-                                        np.arange(wl.L_ctx), wl.B) for g in range(wl.H_kv)])
-        top, _ = S.find_sinks(np_(inp.q_dec)[b], Kc, np_(inp.k_dec)[b], qi[b, : qc[b]], 4,
-                              S.scale_for(wl.d))
+        top, _ = _oracle_sinks(wl, inp, q_idx, q_cnt, 4, b)
         assert np_(sinks)[b].tolist() == top.tolist()
         if wl.G == 1:
             # with one query head per KV head the planted boost (3 x the mean
@@ -80,28 +101,29 @@ def test_find_sinks_recovers_planted(name, cuda_device):
 
 
 @pytest.mark.parametrize("name,n", [("tiny", 1), ("tiny", 12), ("llada8k", 1), ("llada8k", 8),
-                                    ("llada8k", 12)])
+                                    ("llada8k", 12), ("llada8k", 64), ("dream16k", 20)])
 def test_find_sinks_top_n(name, n, cuda_device):
-    """n sinks through both top-n kernels (one pass for n <= 8, rounds of a
-    scan beyond): ascending, distinct, equal to the oracle's where its cut has
-    a margin above the fp32 mass error, else within that error of the cut."""
+    """n sinks with the certified cut: exactly the oracle's, whatever the
+    margin at the cut (columns the fp32 bound cannot separate are recomputed
+    in fp64)."""
     wl = synth.workload(name)
     inp = synth.make_step_inputs(wl, device=cuda_device)
-    desc = desc_for(wl)
-    q_idx = torch.empty((wl.batch, wl.L_q), dtype=torch.int32, device=cuda_device)
-    q_cnt = torch.empty((wl.batch,), dtype=torch.int32, device=cuda_device)
-    dl.dl_predict_queries(inp.conf_prev, inp.still_masked, wl.k, wl.w, q_idx, q_cnt)
-    ws = pipeline.workspace(desc, cuda_device)
-    sinks = torch.empty((wl.batch, n), dtype=torch.int32, device=cuda_device)
-    dl.dl_find_sinks(desc, inp.q_dec, q_idx, q_cnt, inp.k_pool, inp.page_table, inp.k_dec, n,
-                     sinks, ws)
-    assert dl.dl_get_status() == dl.DL_OK
-    qi, qc = np_(q_idx), np_(q_cnt)
+    sinks, q_idx, q_cnt = _find(wl, inp, cuda_device, n)
     for b in range(wl.batch):
-        Kc = np.stack([S.gather_context(np_(inp.k_pool), np_(inp.page_table)[b], g,
-                                        np.arange(wl.L_ctx), wl.B) for g in range(wl.H_kv)])
-        top, mass = S.find_sinks(np_(inp.q_dec)[b], Kc, np_(inp.k_dec)[b], qi[b, : qc[b]], n,
-                                 S.scale_for(wl.d))
+        top, _ = _oracle_sinks(wl, inp, q_idx, q_cnt, n, b)
+        assert np_(sinks)[b].tolist() == top.tolist(), b
+
+
+@pytest.mark.parametrize("name,n", [("tiny", 12), ("llada8k", 12)])
+def test_find_sinks_fp32_cut(name, n, cuda_device):
+    """Without the exponent words: the top n of the fp32 masses (both top-n
+    kernels): ascending, distinct, equal to the oracle's where its cut has a
+    margin above the fp32 mass error, else within that error of the cut."""
+    wl = synth.workload(name)
+    inp = synth.make_step_inputs(wl, device=cuda_device)
+    sinks, q_idx, q_cnt = _find(wl, inp, cuda_device, n, certified=False)
+    for b in range(wl.batch):
+        top, mass = _oracle_sinks(wl, inp, q_idx, q_cnt, n, b)
         got = np_(sinks)[b]
         assert got.tolist() == sorted(set(got.tolist())) and len(got) == n
         assert got.min() >= 0 and got.max() < wl.L_ctx
@@ -110,6 +132,54 @@ def test_find_sinks_top_n(name, n, cuda_device):
             assert got.tolist() == top.tolist()
         else:
             assert (mass[got] >= np.sort(mass)[-n] - tol).all()
+
+
+@pytest.mark.parametrize("exact_tie", [False, True])
+def test_find_sinks_near_tie_at_the_cut(exact_tie, cuda_device):
+    """Two context keys built to have (nearly or exactly) the same mass, just
+    below the planted sinks and above every other column, so that the cut at
+    n = planted + 1 falls between them: a copy of one key with one value moved
+    by a bf16 ulp (masses apart by less than the certification bound, so the
+    fp64 recheck decides), or an exact copy (a tie: the lower position).  The
+    certified cut equals the oracle's."""
+    wl = synth.workload("llada8k", L_ctx=4096)
+    inp = synth.make_step_inputs(wl, device=cuda_device)
+    dev = cuda_device
+    kp = inp.k_pool.clone()
+    pt = np_(inp.page_table)
+    planted = np_(inp.sinks_planted)[0].tolist()
+    t1, t2 = 1000, 3000
+    assert t1 not in planted and t2 not in planted
+    q = inp.q_dec[0].to(torch.float32)
+    for g in range(wl.H_kv):
+        qbar = q[g].mean(dim=0)  # the head's mean decode query (G = 1)
+        r1 = (int(pt[0, t1 // wl.B]), g, t1 % wl.B)
+        r2 = (int(pt[0, t2 // wl.B]), g, t2 % wl.B)
+        kp[r1] = (kp[r1].to(torch.float32) + 1.5 * qbar).to(torch.bfloat16)
+        kp[r2] = kp[r1]
+        if not exact_tie:
+            row = kp[r2].clone()
+            row[5] = _bf16_step(row[5])
+            kp[r2] = row
+    inp2 = dataclasses.replace(inp, k_pool=kp)
+    n = len(planted) + 1
+    sinks, q_idx, q_cnt = _find(wl, inp2, dev, n)
+    top, mass = _oracle_sinks(wl, inp2, q_idx, q_cnt, n, 0)
+    order = np.argsort(-mass, kind="stable")
+    assert set(order[:n - 1].tolist()) == set(planted)        # the planted lead
+    assert set(order[n - 1:n + 1].tolist()) == {t1, t2}       # the pair straddles the cut
+    gap = abs(mass[t1] - mass[t2]) / mass[t1]
+    # inside the certification band (far below the bound on the fp32 error)
+    assert (0.0 < gap < 1e-3) if not exact_tie else gap == 0.0
+    assert np_(sinks)[0].tolist() == top.tolist()
+    if exact_tie:
+        assert t1 in top.tolist() and t2 not in top.tolist()
+
+
+def _bf16_step(x):
+    """x moved to the next larger-magnitude bf16 value."""
+    b = x.view(torch.int16) + 1
+    return b.view(torch.bfloat16)
 
 
 def test_chunked_prefix_workload(cuda_device):
