@@ -238,15 +238,16 @@ def workload_record(name, device, pk, reps=30):
     Kbar = torch.empty((wl.batch, wl.H_kv, n_units, wl.d), dtype=torch.float32, device=device)
     Kdig = Kexp = None
     if wl.chunked:  # chunk keys belong to the cache build, not to the step
+        Kdig, Kexp = dl.key_digit_buffers(wl.batch, wl.H_kv, wl.n_chunks, wl.d, device)
         dl.dl_pool_keys(desc, inp.k_pool, inp.page_table, wl.n_chunks, wl.chunk_stride, 1,
-                        wl.chunk_content, Kbar)
+                        wl.chunk_content, Kbar, Kdig=Kdig, Kexp=Kexp)
 
         def fn(st):
             return pipeline.chunked_step(desc, inp.q_dec, inp.k_pool, inp.v_pool, inp.page_table,
                                          inp.k_dec, inp.v_dec, n_chunks=wl.n_chunks,
                                          stride=wl.chunk_stride, content=wl.chunk_content,
                                          topK_chunks=wl.topK_chunks, topT=wl.topT_tokens,
-                                         Kbar=Kbar, ws=ws, stream=st)
+                                         Kbar=Kbar, Kexp=Kexp, ws=ws, stream=st)
     else:
         Kdig, Kexp = dl.key_digit_buffers(wl.batch, wl.H_kv, wl.n_blk, wl.d, device)
         dl.dl_pool_keys(desc, inp.k_pool, inp.page_table, wl.n_blk, wl.B, 0, wl.B, Kbar,

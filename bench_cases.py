@@ -119,15 +119,16 @@ def chunk_step(reps: int, dev):
                        wl.n_slots, A.DL_BF16)
     ws = torch.empty(A.dl_workspace_size(desc), dtype=torch.uint8, device=dev)
     Kbar = torch.empty((wl.batch, wl.H_kv, wl.n_chunks, wl.d), dtype=torch.float32, device=dev)
+    Kdig, Kexp = A.key_digit_buffers(wl.batch, wl.H_kv, wl.n_chunks, wl.d, dev)
     A.dl_pool_keys(desc, inp.k_pool, inp.page_table, wl.n_chunks, wl.chunk_stride, 1,
-                   wl.chunk_content, Kbar)
+                   wl.chunk_content, Kbar, Kdig=Kdig, Kexp=Kexp)
 
     def fn():
         return pipeline.chunked_step(desc, inp.q_dec, inp.k_pool, inp.v_pool, inp.page_table,
                                      inp.k_dec, inp.v_dec, n_chunks=wl.n_chunks,
                                      stride=wl.chunk_stride, content=wl.chunk_content,
                                      topK_chunks=wl.topK_chunks, topT=wl.topT_tokens,
-                                     Kbar=Kbar, ws=ws)
+                                     Kbar=Kbar, Kexp=Kexp, ws=ws)
     out = fn()
     torch.cuda.synchronize()
     # algorithmic bytes per step: pooled chunk keys, Q, the content K rows of

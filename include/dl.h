@@ -314,12 +314,22 @@ dl_status dl_sparse_attn(const dl_attn_desc* desc, const void* Q_dec, const void
  * logical positions of the n_sel selected chunks, ascending; tok_cnt[b][g]
  * their number (n_sel * (min(topT, chunk_content) + 1)).
  *   chunk_idx int32 [batch][H_kv][n_sel] (from dl_select over chunks)
+ *   Kexp      int32 [batch][H_kv][ceil(L_ctx / chunk_stride)] or NULL: the
+ *             exponent words of the chunk keys (dl_pool_keys over the chunks'
+ *             content tokens); their norm field bounds the content keys'
+ *             norms.  Given (tensor-core kernel: bf16, d 128), the top-T cut
+ *             is certified: where a proven bound on the fp32 masses' error
+ *             does not separate the T-th from the next, the CTA recomputes
+ *             the undecided tokens' masses in fp64 and keeps the top T of
+ *             those.  NULL (or the CUDA-core kernel): the top T of the fp32
+ *             masses.
  *   tok_pos   int32 [batch][H_kv][n_sel*(topT+1)]  (out)
  * Requires 1 <= chunk_content <= 1024, 0 <= topT <= chunk_content. */
 dl_status dl_token_select(const dl_attn_desc* desc, const void* Q_dec, const void* K_pool,
                           const int32_t* page_table, const int32_t* chunk_idx, int n_sel,
-                          int chunk_stride, int chunk_content, int topT, int32_t* tok_pos,
-                          int32_t* tok_cnt, void* ws, size_t ws_bytes, void* stream);
+                          int chunk_stride, int chunk_content, int topT, const int32_t* Kexp,
+                          int32_t* tok_pos, int32_t* tok_cnt, void* ws, size_t ws_bytes,
+                          void* stream);
 
 /* (a7) Attention over gathered, non-contiguous cached tokens plus the decode
  * block.  [P1 abstract: a kernel that parallelises decoding over the

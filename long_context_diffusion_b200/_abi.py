@@ -66,7 +66,7 @@ _SIGS = {
     "dl_sparse_attn": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp,
                         _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp], _c_int),
     "dl_token_select": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _c_int, _c_int,
-                         _c_int, _c_int, _vp, _vp, _vp, ctypes.c_size_t, _vp], _c_int),
+                         _c_int, _c_int, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp], _c_int),
     "dl_block_scores_noalloc": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _c_int, _vp,
                                  _vp], _c_int),
     "dl_sparse_attn_gather": ([ctypes.POINTER(dl_attn_desc), _vp, _vp, _vp, _vp, _vp, _vp,
@@ -226,11 +226,13 @@ def dl_sparse_attn(desc, Q_dec, K_pool, V_pool, page_table, blk_idx, blk_cnt, K_
 
 
 def dl_token_select(desc, Q_dec, K_pool, page_table, chunk_idx, chunk_stride, chunk_content, topT,
-                    tok_pos, tok_cnt, ws=None, stream=None):
+                    tok_pos, tok_cnt, ws=None, stream=None, Kexp=None):
+    """Kexp: the chunk keys' exponent words (dl_pool_keys over the chunks);
+    given, the top-T cut is certified."""
     n_sel = chunk_idx.shape[-1]
     wsz = 0 if ws is None else ws.numel() * ws.element_size()
     _check(lib.dl_token_select(ctypes.byref(desc), _p(Q_dec), _p(K_pool), _p(page_table),
-                               _p(chunk_idx), n_sel, chunk_stride, chunk_content, topT,
+                               _p(chunk_idx), n_sel, chunk_stride, chunk_content, topT, _p(Kexp),
                                _p(tok_pos), _p(tok_cnt), _p(ws), wsz, _s(stream)))
 
 

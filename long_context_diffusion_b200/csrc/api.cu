@@ -400,8 +400,9 @@ dl_status dl_sparse_attn_gather(const dl_attn_desc* desc, const void* Q_dec, con
 
 dl_status dl_token_select(const dl_attn_desc* desc, const void* Q_dec, const void* K_pool,
                           const int32_t* page_table, const int32_t* chunk_idx, int n_sel,
-                          int chunk_stride, int chunk_content, int topT, int32_t* tok_pos,
-                          int32_t* tok_cnt, void* ws, size_t ws_bytes, void* stream) {
+                          int chunk_stride, int chunk_content, int topT, const int32_t* Kexp,
+                          int32_t* tok_pos, int32_t* tok_cnt, void* ws, size_t ws_bytes,
+                          void* stream) {
   (void)ws;
   (void)ws_bytes;
   dl::Shape s;
@@ -420,8 +421,8 @@ dl_status dl_token_select(const dl_attn_desc* desc, const void* Q_dec, const voi
   unsigned* err = nullptr;
   if ((st = error_word(&err)) != DL_OK) return st;
   return launched(dl::launch_token_select(s, Q_dec, K_pool, page_table, chunk_idx, n_sel,
-                                          chunk_stride, chunk_content, topT, tok_pos, tok_cnt,
-                                          err, as_stream(stream)),
+                                          chunk_stride, chunk_content, topT, Kexp, tok_pos,
+                                          tok_cnt, err, as_stream(stream)),
                   "dl_token_select launch");
 }
 

@@ -115,8 +115,9 @@ cudaError_t launch_cache_write(const Shape& s, const void* K_new, const void* V_
                                cudaStream_t st);
 cudaError_t launch_token_select(const Shape& s, const void* Q, const void* Kp,
                                 const int32_t* page_table, const int32_t* chunk_idx, int n_sel,
-                                int chunk_stride, int chunk_content, int topT, int32_t* tok_pos,
-                                int32_t* tok_cnt, unsigned* err, cudaStream_t st);
+                                int chunk_stride, int chunk_content, int topT,
+                                const int32_t* Kexp, int32_t* tok_pos, int32_t* tok_cnt,
+                                unsigned* err, cudaStream_t st);
 
 // Shared by entry points in several files (defined in api.cu).
 dl_status api_check_desc(const dl_attn_desc* d, Shape* s);

@@ -147,18 +147,20 @@ token_select_kernel(Shape s, const T* __restrict__ Q, const T* __restrict__ Kp,
 bool token_select_tc_supported(const Shape& s, int chunk_stride, int chunk_content);
 cudaError_t launch_token_select_tc(const Shape& s, const void* Q, const void* Kp,
                                    const int32_t* page_table, const int32_t* chunk_idx, int n_sel,
-                                   int chunk_stride, int chunk_content, int topT, int32_t* tok_pos,
-                                   int32_t* tok_cnt, unsigned* err, cudaStream_t st);
+                                   int chunk_stride, int chunk_content, int topT,
+                                   const int32_t* Kexp, int32_t* tok_pos, int32_t* tok_cnt,
+                                   unsigned* err, cudaStream_t st);
 
 // bf16, d 128, page-aligned chunks of at most 64 rows per group: the tensor
 // cores (token_select_tc.cu); otherwise the CUDA-core kernel above.
 cudaError_t launch_token_select(const Shape& s, const void* Q, const void* Kp,
                                 const int32_t* page_table, const int32_t* chunk_idx, int n_sel,
-                                int chunk_stride, int chunk_content, int topT, int32_t* tok_pos,
-                                int32_t* tok_cnt, unsigned* err, cudaStream_t st) {
+                                int chunk_stride, int chunk_content, int topT,
+                                const int32_t* Kexp, int32_t* tok_pos, int32_t* tok_cnt,
+                                unsigned* err, cudaStream_t st) {
   if (token_select_tc_supported(s, chunk_stride, chunk_content) && !(kernel_flags() & DL_FLAG_TOKEN_SIMT))
     return launch_token_select_tc(s, Q, Kp, page_table, chunk_idx, n_sel, chunk_stride,
-                                  chunk_content, topT, tok_pos, tok_cnt, err, st);
+                                  chunk_content, topT, Kexp, tok_pos, tok_cnt, err, st);
   dim3 grid(n_sel, s.batch * s.H_kv);
   if (s.dtype == 0) {
     auto* q = reinterpret_cast<const __nv_bfloat16*>(Q);

@@ -30,6 +30,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "kdigits.cuh"
 #include "sm100.cuh"
 #include "launch.cuh"
 
@@ -105,6 +106,142 @@ __device__ __forceinline__ int block_exclusive_sum(int v, int* s_scan, int* tota
   return before + inc - v;
 }
 
+// fp64 recheck of one chunk's undecided cut (certified cut, see the kernel):
+// the LSE of every row over the chunk's usable content tokens, then the mass
+// of every candidate (s_key[i] - 1 >= thr as fp32 bits), and keep[i] = the
+// candidate is among the T largest fp64 masses (ties to the lower position).
+// scratch: >= R * D + R + MAXC doubles (the K ring, free after streaming).
+// Every thread of the CTA calls it.
+__device__ __noinline__ void token_recheck_fp64(
+    const Shape& s, const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ Kp,
+    const int32_t* __restrict__ page_table, int b, int g, long long base, int n, int T,
+    double thr, const uint32_t* s_key, const int* s_pv, double* scratch, uint8_t* keep_bits) {
+  constexpr int RG = 16;  // rows per LSE pass
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int R = s.G * s.L_q;
+  double* q64 = scratch;              // [R][D]
+  double* lse = q64 + R * D;          // [R]
+  double* tau = lse + R;              // [MAXC]: fp64 mass of each candidate, -1 otherwise
+  __shared__ double s_m[THREADS / 32][RG], s_z[THREADS / 32][RG];
+  for (int e = tid; e < R * D; e += THREADS) {
+    const int r = e / D, c = e % D;
+    const int h = g * s.G + r / s.L_q, i = r % s.L_q;
+    q64[e] = (double)__bfloat162float(Q[(((size_t)b * s.H + h) * s.L_q + i) * D + c]);
+  }
+  __syncthreads();
+  auto usable = [&](int i) {  // content index i <-> offset i + 1
+    return i < n && s_key[i] != 0u;
+  };
+  auto key_src = [&](int i) {
+    const long long pos = base + 1 + i;
+    const int slot = page_table[(size_t)b * s.n_pages + pos / 64];
+    return Kp + (((size_t)slot * s.H_kv + g) * 64 + pos % 64) * D;
+  };
+  // fp64 logits of rows r0 .. r0+nr-1 against key i (dimension order)
+  auto logits = [&](const __nv_bfloat16* k, int r0, int nr, double(&acc)[RG]) {
+#pragma unroll
+    for (int j = 0; j < RG; ++j) acc[j] = 0.0;
+    for (int c = 0; c < D; c += 8) {
+      float kv[8];
+      Vec16<__nv_bfloat16>::load(k + c, kv);
+#pragma unroll
+      for (int j = 0; j < RG; ++j) {
+        if (j < nr) {
+          const double* q = q64 + (r0 + j) * D + c;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[j] = fma(q[e], (double)kv[e], acc[j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < RG; ++j) acc[j] *= s.scale;
+  };
+  // row LSEs over the usable content tokens
+  for (int r0 = 0; r0 < R; r0 += RG) {
+    const int nr = min(RG, R - r0);
+    double m[RG], z[RG];
+#pragma unroll
+    for (int j = 0; j < RG; ++j) {
+      m[j] = -INFINITY;
+      z[j] = 0.0;
+    }
+    for (int i = tid; i < n; i += THREADS) {
+      if (!usable(i)) continue;
+      double l[RG];
+      logits(key_src(i), r0, nr, l);
+#pragma unroll
+      for (int j = 0; j < RG; ++j) {
+        if (j >= nr) continue;
+        if (l[j] > m[j]) {
+          z[j] = z[j] * exp(m[j] - l[j]) + 1.0;
+          m[j] = l[j];
+        } else {
+          z[j] += exp(l[j] - m[j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < RG; ++j) {  // merge over the warp, then over the warps
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double om = __shfl_xor_sync(0xffffffffu, m[j], o);
+        const double oz = __shfl_xor_sync(0xffffffffu, z[j], o);
+        const double mm = fmax(m[j], om);
+        z[j] = (m[j] == -INFINITY ? 0.0 : z[j] * exp(m[j] - mm)) +
+               (om == -INFINITY ? 0.0 : oz * exp(om - mm));
+        m[j] = mm;
+      }
+      if (lane == 0) {
+        s_m[warp][j] = m[j];
+        s_z[warp][j] = z[j];
+      }
+    }
+    __syncthreads();
+    if (tid < nr) {
+      double mm = -INFINITY;
+      for (int w = 0; w < THREADS / 32; ++w) mm = fmax(mm, s_m[w][tid]);
+      double zz = 0.0;
+      for (int w = 0; w < THREADS / 32; ++w)
+        if (s_m[w][tid] != -INFINITY) zz += s_z[w][tid] * exp(s_m[w][tid] - mm);
+      lse[r0 + tid] = mm + log(zz);
+    }
+    __syncthreads();
+  }
+  // candidates' fp64 masses, summed over the rows in order
+  for (int i = tid; i < MAXC; i += THREADS) {
+    double t = -1.0;
+    if (usable(i) && (double)__uint_as_float(s_key[i] - 1u) >= thr) {
+      const __nv_bfloat16* k = key_src(i);
+      t = 0.0;
+      for (int r0 = 0; r0 < R; r0 += RG) {
+        const int nr = min(RG, R - r0);
+        double l[RG];
+        logits(k, r0, nr, l);
+#pragma unroll
+        for (int j = 0; j < RG; ++j)
+          if (j < nr) t += exp(l[j] - lse[r0 + j]);
+      }
+    }
+    tau[i] = t;
+  }
+  __syncthreads();
+  // keep: a candidate with fewer than T better ones (mass desc, position asc)
+  for (int i = tid; i < MAXC; i += THREADS) {
+    bool kp = false;
+    const double ti = tau[i];
+    if (ti >= 0.0) {
+      int better = 0;
+      for (int j = 0; j < MAXC; ++j) {
+        const double tj = tau[j];
+        better += (tj > ti || (tj == ti && j < i)) ? 1 : 0;
+      }
+      kp = better < T;
+    }
+    keep_bits[i] = kp ? 1 : 0;
+  }
+  __syncthreads();
+}
+
 }  // namespace ts
 
 template <int N>
@@ -113,7 +250,8 @@ token_select_tc_kernel(const __grid_constant__ CUtensorMap tm_k, Shape s,
                        const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ Kp,
                        const int32_t* __restrict__ page_table,
                        const int32_t* __restrict__ chunk_idx, int n_sel, int stride, int content,
-                       int topT, int32_t* __restrict__ tok_pos, int32_t* __restrict__ tok_cnt,
+                       int topT, const int32_t* __restrict__ Kexp, int n_chunks,
+                       int32_t* __restrict__ tok_pos, int32_t* __restrict__ tok_cnt,
                        unsigned* err) {
   using namespace ts;
   using L = Layout<N>;
@@ -440,6 +578,53 @@ token_select_tc_kernel(const __grid_constant__ CUtensorMap tm_k, Shape s,
       k_rem -= s_scan[33];
       __syncthreads();
     }
+    // Certified cut (with the chunk's exponent word): the fp32 masses are
+    // within a relative eps of the exact ones (the bound of the sink search,
+    // sinks_cert.cu: logits d 2^-23 ||q|| ||k|| scale, the exponentials and
+    // sums on top).  Tokens below thr = v_T (1 - eps) / (1 + eps) are not in
+    // the top T; if more than T reach thr, the CTA recomputes those in fp64.
+    __shared__ int s_cnt_thr;
+    __shared__ float s_qmax;
+    __shared__ double s_thr;
+    bool recheck = false;
+    if (Kexp != nullptr && T > 0 && T < n) {
+      if (warp == 0) {  // largest row norm of the group (rounded up)
+        float qm = 0.0f;
+        for (int r = lane; r < R; r += 32) {
+          const int h = g * s.G + r / s.L_q, i = r % s.L_q;
+          const __nv_bfloat16* qr = Q + (((size_t)b * s.H + h) * s.L_q + i) * D;
+          float sq = 0.0f;
+          for (int c2i = 0; c2i < D; ++c2i) {
+            const float v = __bfloat162float(qr[c2i]);
+            sq = __fmaf_rn(v, v, sq);
+          }
+          qm = fmaxf(qm, __fsqrt_ru(sq * (1.0f + 0x1p-14f)));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, o));
+        if (lane == 0) {
+          s_qmax = qm;
+          s_cnt_thr = 0;
+          const double kn = (double)key_norm_of(Kexp[(size_t)bg * n_chunks + c]);
+          const double delta = s.scale * (double)qm * kn * (1.0 + 0x1p-20) * (D + 2) * 0x1p-23;
+          const double eps = 4.0 * delta + ((double)n / 32.0 + R + 512.0) * 0x1p-24 + 0x1p-20;
+          const double vT = (double)__uint_as_float(prefix - 1u);
+          s_thr = vT * (1.0 - eps) / (1.0 + eps);
+        }
+      }
+      __syncthreads();
+      int cnt = 0;
+      for (int i = threadIdx.x; i < n; i += blockDim.x)
+        cnt += (s_key[i] != 0u && (double)__uint_as_float(s_key[i] - 1u) >= s_thr) ? 1 : 0;
+      atomicAdd(&s_cnt_thr, cnt);
+      __syncthreads();
+      recheck = s_cnt_thr != T;
+    }
+    uint8_t* keep_bits = reinterpret_cast<uint8_t*>(s_hist);  // 1024 flags over hist + scan
+    if (recheck) {
+      ts::token_recheck_fp64(s, Q, Kp, page_table, b, g, base, n, T, s_thr, s_key, s_pv,
+                             reinterpret_cast<double*>(sK), keep_bits);
+    }
     // keep: above the cut, or at it among the first k_rem in position order
     constexpr int PER_T = MAXC / THREADS;  // positions per thread, contiguous
     const int i0 = threadIdx.x * PER_T;
@@ -457,7 +642,9 @@ token_select_tc_kernel(const __grid_constant__ CUtensorMap tm_k, Shape s,
     for (int q = 0; q < PER_T; ++q) {
       const int i = i0 + q;
       bool k = false;
-      if (T > 0 && i < n) {
+      if (recheck) {
+        k = i < n && keep_bits[i] != 0;
+      } else if (T > 0 && i < n) {
         const uint32_t v = s_key[i];
         if (v > prefix) {
           k = true;
@@ -501,9 +688,11 @@ bool token_select_tc_supported(const Shape& s, int chunk_stride, int chunk_conte
 
 cudaError_t launch_token_select_tc(const Shape& s, const void* Q, const void* Kp,
                                    const int32_t* page_table, const int32_t* chunk_idx, int n_sel,
-                                   int chunk_stride, int chunk_content, int topT, int32_t* tok_pos,
-                                   int32_t* tok_cnt, unsigned* err, cudaStream_t st) {
+                                   int chunk_stride, int chunk_content, int topT,
+                                   const int32_t* Kexp, int32_t* tok_pos, int32_t* tok_cnt,
+                                   unsigned* err, cudaStream_t st) {
   CUtensorMap mk;
+  const int n_chunks = (s.L_ctx + chunk_stride - 1) / chunk_stride;
   if (!tc_map_2d(&mk, Kp, ts::D, (uint64_t)s.n_slots * s.H_kv * 64, 64)) return cudaErrorInvalidValue;
   dim3 grid(n_sel, s.batch * s.H_kv);
   auto* q = reinterpret_cast<const __nv_bfloat16*>(Q);
@@ -515,14 +704,16 @@ cudaError_t launch_token_select_tc(const Shape& s, const void* Q, const void* Kp
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
       return e;
     DL_LAUNCH(token_select_tc_kernel<32>, grid, ts::THREADS, smem, st, mk, s, q, k, page_table,
-              chunk_idx, n_sel, chunk_stride, chunk_content, topT, tok_pos, tok_cnt, err);
+              chunk_idx, n_sel, chunk_stride, chunk_content, topT, Kexp, n_chunks, tok_pos,
+              tok_cnt, err);
   } else {
     constexpr int smem = ts::Layout<64>::SMEM;
     if ((e = cudaFuncSetAttribute(token_select_tc_kernel<64>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
       return e;
     DL_LAUNCH(token_select_tc_kernel<64>, grid, ts::THREADS, smem, st, mk, s, q, k, page_table,
-              chunk_idx, n_sel, chunk_stride, chunk_content, topT, tok_pos, tok_cnt, err);
+              chunk_idx, n_sel, chunk_stride, chunk_content, topT, Kexp, n_chunks, tok_pos,
+              tok_cnt, err);
   }
   return cudaGetLastError();
 }

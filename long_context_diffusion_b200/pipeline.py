@@ -111,7 +111,7 @@ class ChunkOutputs:
 
 def chunked_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec, v_dec, *,
                  n_chunks: int, stride: int, content: int, topK_chunks: int, topT: int,
-                 Kbar=None, ws=None, stream=None) -> ChunkOutputs:
+                 Kbar=None, Kexp=None, ws=None, stream=None) -> ChunkOutputs:
     """Chunked-prefix step: chunk keys (BOS excluded), chunk scores from
     every decode query, top-K chunks, top-T tokens per chunk plus its BOS,
     attention over the gathered tokens and the decode block."""
@@ -120,8 +120,11 @@ def chunked_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec,
     if ws is None:
         ws = workspace(desc, dev)
     if Kbar is None:
+        # chunk keys with their exponent words (the token cut is certified with them)
         Kbar = _empty((B, H_kv, n_chunks, d), torch.float32, dev)
-        A.dl_pool_keys(desc, k_pool, page_table, n_chunks, stride, 1, content, Kbar, stream)
+        Kdig, Kexp = A.key_digit_buffers(B, H_kv, n_chunks, d, dev)
+        A.dl_pool_keys(desc, k_pool, page_table, n_chunks, stride, 1, content, Kbar, stream,
+                       Kdig=Kdig, Kexp=Kexp)
     score = _empty((B, H_kv, n_chunks), torch.float64, dev)
     kc = min(topK_chunks, n_chunks)
     chunk_idx = _empty((B, H_kv, kc), torch.int32, dev)
@@ -132,7 +135,7 @@ def chunked_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec,
     tok_pos = _empty((B, H_kv, kc * (topT + 1)), torch.int32, dev)
     tok_cnt = _empty((B, H_kv), torch.int32, dev)
     A.dl_token_select(desc, q_dec, k_pool, page_table, chunk_idx, stride, content, topT, tok_pos,
-                      tok_cnt, ws, stream)
+                      tok_cnt, ws, stream, Kexp=Kexp)
     O = _empty((B, L_q, H, d), q_dec.dtype, dev)
     lse = _empty((B, H, L_q), torch.float32, dev)
     A.dl_sparse_attn_gather(desc, q_dec, k_pool, v_pool, page_table, tok_pos, tok_cnt, k_dec,

@@ -103,8 +103,8 @@ def test_null_and_range_arguments_rejected_before_launch():
                             fake, None, ctypes.c_void_p(0x10000), 256, None)
     assert st == dl.DL_ERR_WORKSPACE
     # unsupported token-select sizes
-    st = lib.dl_token_select(ctypes.byref(d), fake, fake, fake, fake, 8, 1088, 2048, 256, fake,
-                             fake, None, 0, None)
+    st = lib.dl_token_select(ctypes.byref(d), fake, fake, fake, fake, 8, 1088, 2048, 256, None,
+                             fake, fake, None, 0, None)
     assert st == dl.DL_ERR_INVALID_ARG
 
 

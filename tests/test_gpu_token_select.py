@@ -3,9 +3,11 @@ directly through the C ABI: chunks of 1024 content tokens (eight key tiles
 and the token past them), ragged chunks, one and two query heads per KV
 group, 16 to 64 query rows, T from 0 to the whole chunk, and a chunk stride
 off the page grid (the CUDA-core kernel).  Every page-aligned case also runs
-through the CUDA-core kernel.  Kept tokens must equal the oracle's wherever
-its cut has a margin above the fp32 error of the masses, and be within that
-error of the cut otherwise."""
+through the CUDA-core kernel.  With the chunk keys' exponent words the
+tensor-core kernel's cut is certified and the kept tokens must equal the
+oracle's exactly; otherwise (fp32 cut) they must equal them wherever the
+oracle's cut has a margin above the fp32 error of the masses, and be within
+that error of the cut elsewhere."""
 
 import numpy as np
 import pytest
@@ -22,6 +24,17 @@ pytestmark = pytest.mark.gpu
 SEED = 20261202
 
 
+def _chunk_exps(desc, kp, page_table, n_chunks, stride, content, dev):
+    """Exponent words (with the norm bounds) of the chunk keys: each chunk's
+    content tokens pooled, the BOS left out."""
+    batch, H_kv, d = desc.batch, desc.H_kv, desc.d
+    kbar = torch.empty((batch, H_kv, n_chunks, d), dtype=torch.float32, device=dev)
+    kdig, kexp = dl.key_digit_buffers(batch, H_kv, n_chunks, d, dev)
+    dl.dl_pool_keys(desc, kp.to(dev), page_table.to(dev), n_chunks, stride, 1, content, kbar,
+                    Kdig=kdig, Kexp=kexp)
+    return kexp
+
+
 @pytest.mark.parametrize("content,stride,H,H_kv,L_q,topT,n_sel", [
     (1024, 1088, 4, 4, 64, 256, 2),   # the benchmark's chunk shape: 64 rows
     (1000, 1024, 4, 2, 16, 100, 2),   # G = 2, 32 rows, ragged last tile
@@ -30,8 +43,8 @@ SEED = 20261202
     (64, 128, 3, 3, 48, 1, 2),        # one tile, 48 rows
     (300, 301, 2, 2, 32, 37, 2),      # stride off the page grid
 ])
-@pytest.mark.parametrize("simt", [False, True])
-def test_token_select_matches_oracle(content, stride, H, H_kv, L_q, topT, n_sel, simt,
+@pytest.mark.parametrize("simt,certified", [(False, True), (False, False), (True, False)])
+def test_token_select_matches_oracle(content, stride, H, H_kv, L_q, topT, n_sel, simt, certified,
                                      cuda_device, kernel_flags):
     if simt:
         kernel_flags(dl.DL_FLAG_TOKEN_SIMT)
@@ -57,9 +70,13 @@ def test_token_select_matches_oracle(content, stride, H, H_kv, L_q, topT, n_sel,
     per = topT + 1
     tok_pos = torch.full((batch, H_kv, n_sel * per), -7, dtype=torch.int32, device=cuda_device)
     tok_cnt = torch.full((batch, H_kv), -7, dtype=torch.int32, device=cuda_device)
+    Kexp = _chunk_exps(desc, kp, page_table, n_chunks, stride, content, cuda_device) \
+        if certified else None
     dl.dl_token_select(desc, q.to(cuda_device), kp.to(cuda_device), page_table.to(cuda_device),
-                       chunk_idx.to(cuda_device), stride, content, topT, tok_pos, tok_cnt, ws)
+                       chunk_idx.to(cuda_device), stride, content, topT, tok_pos, tok_cnt, ws,
+                       Kexp=Kexp)
     torch.cuda.synchronize()
+    exact = certified and stride % page == 0  # the tensor-core kernel takes page-aligned chunks
     assert dl.dl_get_status() == dl.DL_OK
     got, cnt = np_(tok_pos), np_(tok_cnt)
     assert (cnt == n_sel * per).all()
@@ -81,7 +98,83 @@ def test_token_select_matches_oracle(content, stride, H, H_kv, L_q, topT, n_sel,
                 mine = kept[: len(off)] - base - 1
                 assert np.all(np.diff(mine) > 0), (b, g, j)
                 tol = 1e-5 * tau.max()
-                if cut_margin(tau, off) > tol:
+                if exact:
+                    assert mine.tolist() == off.tolist(), (b, g, j)
+                elif cut_margin(tau, off) > tol:
                     assert mine.tolist() == off.tolist(), (b, g, j)
                 else:
                     assert (tau[mine] >= np.sort(tau)[-topT] - tol).all(), (b, g, j)
+
+
+@pytest.mark.parametrize("exact_tie", [False, True])
+def test_token_select_near_tie_at_the_cut(exact_tie, cuda_device):
+    """Two content tokens of one chunk built to have (nearly or exactly) the
+    same mass and to straddle the top-T cut: token a's key is raised so that
+    it ranks T-th, token b is a copy of it (a tie: the lower position is
+    kept), or the copy with one value moved by a bf16 ulp (masses apart by
+    less than the certification bound, so the fp64 recheck decides).  The
+    certified cut equals the oracle's."""
+    batch, H, H_kv, d, L_q, page = 1, 2, 2, 128, 32, 64
+    content, stride, n_chunks, topT = 1024, 1088, 2, 64
+    L_ctx = n_chunks * stride
+    n_pages = -(-L_ctx // page)
+    n_slots = batch * n_pages
+    q = synth.normals(SEED, 12990, 0, batch * H * L_q * d).reshape(batch, H, L_q, d).to(
+        torch.bfloat16)
+    kp = synth.normals(SEED, 12991, 0, n_slots * H_kv * page * d).reshape(
+        n_slots, H_kv, page, d).to(torch.bfloat16)
+    page_table = torch.arange(n_slots, dtype=torch.int32).reshape(batch, n_pages)
+    chunk_idx = torch.tensor([[[1], [1]]], dtype=torch.int32)
+    base = 1 * stride
+    desc = dl.make_desc(batch=batch, H=H, H_kv=H_kv, d=d, L_ctx=L_ctx, L_q=L_q, page=page,
+                        n_pages=n_pages, n_slots=n_slots, dtype=dl.DL_BF16)
+    scale = oracle.scale_for(d)
+    a, bpos = 100, 900  # content offsets (positions base + 1 + offset)
+    for g in range(H_kv):
+        rows = S.f64(q[0, g])
+        keys = S.gather_context(S.f64(kp), page_table[0].numpy(), g,
+                                base + 1 + np.arange(content), page)
+        _, tau = S.token_select(rows, keys, topT, scale)
+        target = np.sort(tau)[-topT]  # the T-th mass: raise a's key until it reaches it
+        qbar = q[0, g].to(torch.float32).mean(dim=0)
+        ra = (int(page_table[0, (base + 1 + a) // page]), g, (base + 1 + a) % page)
+        rb = (int(page_table[0, (base + 1 + bpos) // page]), g, (base + 1 + bpos) % page)
+        orig = kp[ra].to(torch.float32).clone()
+        lo, hi = 0.0, 20.0
+        for _ in range(40):
+            mid = (lo + hi) / 2
+            kp[ra] = (orig + mid * qbar).to(torch.bfloat16)
+            keys = S.gather_context(S.f64(kp), page_table[0].numpy(), g,
+                                    base + 1 + np.arange(content), page)
+            _, tau = S.token_select(rows, keys, topT, scale)
+            if tau[a] > target:
+                hi = mid
+            else:
+                lo = mid
+        kp[ra] = (orig + hi * qbar).to(torch.bfloat16)
+        kp[rb] = kp[ra]
+        if not exact_tie:
+            row = kp[rb].clone()
+            row[7] = (row[7].view(torch.int16) + 1).view(torch.bfloat16)
+            kp[rb] = row
+    dev = cuda_device
+    ws = torch.empty(max(dl.dl_workspace_size(desc), 256), dtype=torch.uint8, device=dev)
+    per = topT + 1
+    tok_pos = torch.full((batch, H_kv, per), -7, dtype=torch.int32, device=dev)
+    tok_cnt = torch.full((batch, H_kv), -7, dtype=torch.int32, device=dev)
+    Kexp = _chunk_exps(desc, kp, page_table, n_chunks, stride, content, dev)
+    dl.dl_token_select(desc, q.to(dev), kp.to(dev), page_table.to(dev), chunk_idx.to(dev),
+                       stride, content, topT, tok_pos, tok_cnt, ws, Kexp=Kexp)
+    assert dl.dl_get_status() == dl.DL_OK
+    got = np_(tok_pos)
+    for g in range(H_kv):
+        rows = S.f64(q[0, g])
+        keys = S.gather_context(S.f64(kp), page_table[0].numpy(), g,
+                                base + 1 + np.arange(content), page)
+        off, tau = S.token_select(rows, keys, topT, scale)
+        order = np.argsort(-tau, kind="stable")
+        assert {a, bpos} & set(order[topT - 1:topT + 1].tolist()), g  # at the cut
+        gap = abs(tau[a] - tau[bpos]) / tau[a]
+        assert (0.0 < gap < 1e-3) if not exact_tie else gap == 0.0
+        mine = got[0, g, 1:] - base - 1
+        assert mine.tolist() == off.tolist(), g
