@@ -744,12 +744,14 @@ def run_ours(args):
 
 def count_launches(wl):
     """Kernels of this library launched per step (from the call sequence):
-    the cache write, the prediction, one attention kernel per layer (it merges
-    its own split partials; a memset of the merge counts precedes it), the
-    sink search (LSE pass, mass pass, top-n) and one score + select kernel per
-    sparse layer when the group's rows fit a fused kernel (else three)."""
+    the cache write, the prediction, attention and combine per layer, the
+    certified sink search, and one score + select kernel per sparse layer when
+    the group's rows fit a fused kernel (else three)."""
     n_sparse = wl.n_layers - wl.first_sparse_layer
-    pool, predict, attn, sinks = 1, 1, 1, 3
+    # sinks: LSE pass + combine, mass, top-n, and the certification (band,
+    # fp64 LSE, merge, candidate masses, pick: the last four return at once
+    # when the cut is certified)
+    pool, predict, attn, sinks = 1, 1, 2, 9
     rows = wl.G * min(wl.L_q, wl.k * (2 * wl.w + 1))
     fused = rows <= 32 and wl.n_blk <= 512
     score_select = 1 if fused else 3

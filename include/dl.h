@@ -230,8 +230,7 @@ dl_status dl_find_sinks(const dl_attn_desc* desc, const void* Q_dec, const int32
  *   written); the same arguments, checks and workspace as dl_find_sinks.
  *   The split calls take the top n of the fp32 sum without the certified
  *   recheck of dl_find_sinks.
- * dl_sink_topn: mass fp32 [batch][L_ctx] (device; in, and scratch when
- *   n_sinks > 8: the chosen columns are overwritten with -inf);
+ * dl_sink_topn: mass fp32 [batch][L_ctx] (device; in, not modified);
  *   sink_pos int32 [batch][n_sinks] (out), the n_sinks columns of largest
  *   mass (ties -> lower index), ascending.  1 <= n_sinks <= 64.
  *   No workspace.  Returns DL_ERR_INVALID_ARG for NULL pointers or sizes out

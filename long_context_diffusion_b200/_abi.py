@@ -192,8 +192,7 @@ def dl_sink_mass(desc, Q_dec, q_idx, q_cnt, K_pool, page_table, K_dec, mass, ws,
 
 
 def dl_sink_topn(mass, sink_pos, stream=None):
-    """sink_pos [batch][n_sinks] from the summed mass [batch][L_ctx]; with
-    more than 8 sinks the chosen columns of mass are overwritten."""
+    """sink_pos [batch][n_sinks] from the summed mass [batch][L_ctx]."""
     batch, L_ctx = mass.shape
     _check(lib.dl_sink_topn(_p(mass), batch, L_ctx, sink_pos.shape[-1], _p(sink_pos),
                             _s(stream)))

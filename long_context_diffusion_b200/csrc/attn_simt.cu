@@ -183,8 +183,7 @@ attn_combine_kernel(Shape s, int n_split, const void* ws, T* __restrict__ O,
 
 size_t attn_workspace(const Shape& s) {
   const size_t n = (size_t)s.batch * s.H_kv * kMaxSplits * s.G * s.L_q;
-  return round256(n * s.d * sizeof(float)) + round256(n * sizeof(float2)) +
-         round256((size_t)s.batch * s.H_kv * sizeof(int));  // merge counters
+  return round256(n * s.d * sizeof(float)) + round256(n * sizeof(float2));
 }
 
 int attn_splits(const Shape& s, int max_tiles) {

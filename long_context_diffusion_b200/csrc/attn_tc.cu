@@ -42,8 +42,7 @@
 // their TMA path.
 // The G*L_q query rows of a KV group are padded to M-tiles of 128 rows (the
 // path is HBM-bound: padding costs tensor time, not bytes).  Partials of the
-// splits of one (b, g) are merged at the end of the kernel by the CTA whose
-// partial completes the (b, g) (a count in the workspace; no waiting).
+// splits of one (b, g) are merged by the combine kernel of attn_simt.cu.
 //
 // Every wait is bounded: a role that gives up raises the shared abort flag
 // and the device error word (ERR_TIMEOUT) and leaves its loop; the CTA then
@@ -680,27 +679,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
-  // ---- merge: the CTA whose partials complete a (b, g) merges that (b, g)
-  // (a count per (b, g); no CTA waits for another).  An aborted CTA adds no
-  // count: its (b, g) stay unmerged, and the error word says so.
-  if (*abort_flag || u1 <= u0) return;
-  __threadfence();  // this thread's partials, before the count that publishes them
-  __syncthreads();
-  __shared__ int s_last;
-  int* counts = merge_counters_of(a.ws, s);
-  for (int bg = (int)(u0 / plan.S); bg <= (int)((u1 - 1) / plan.S); ++bg) {
-    const long long base = (long long)bg * plan.S;
-    const int nv = tc_owner(base + plan.S - 1, U, gridDim.x) - tc_owner(base, U, gridDim.x) + 1;
-    if (threadIdx.x == 0) s_last = atomicAdd(counts + bg, 1) == nv - 1;
-    __syncthreads();
-    if (s_last) {
-      __threadfence();  // the other CTAs' partials, after their counts
-      for (int r = warp; r < R; r += C::THREADS / 32)
-        merge_row<__nv_bfloat16, D>(part, s, plan.nslot, bg, r, nv,
-                                    reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, lane);
-    }
-    __syncthreads();
-  }
 }
 
 // ---------------------------------------------------------------- host side
@@ -818,11 +796,9 @@ static cudaError_t run_tc(const AttnArgs& a, int max_tiles, cudaStream_t st) {
   auto kern = attn_tc_kernel<D, NM, REP, ST, QB, OB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  // the merge counts start at zero (the kernel merges; no combine launch)
-  if ((e = cudaMemsetAsync(merge_counters_of(a.ws, s), 0, n_bg * sizeof(int), st)) != cudaSuccess)
-    return e;
   DL_LAUNCH(kern, L.grid, C::THREADS, C::SMEM, st, mq, mk, mv, mkd, mvd, a, L.plan);
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return launch_combine(a, L.plan.nslot, st, L.plan.S, L.grid);
 }
 
 // Whether the tensor-core kernel takes this call (bf16, block or dense keys,

@@ -32,9 +32,9 @@
 // Roles: warp 0 one thread: TMA of Q (per segment) and of the K ring;
 // warp 2 one thread: the V ring; warp 1 one thread: S^T MMAs; warp 3 one
 // thread: O^T MMAs; warps 4..7: softmax.  Work is split over the SMs in tile
-// slots exactly as in attn_tc.cu; a CTA writes one partial per (b, g) it
-// touches, and the CTA whose partial completes a (b, g) (a count in the
-// workspace) merges that (b, g)'s partials into O and the LSEs at its end.
+// slots exactly as in attn_tc.cu; partials go to the same combine kernel.
+// (Merging inside this kernel, by the CTA whose partial completes a (b, g),
+// measured slower: the merges land on the last CTAs, at the tail.)
 // Every wait is bounded and the softmax warps exchange through mbarriers (no
 // named barriers), so a role that gives up cannot leave another waiting.
 // With O == nullptr only the row LSEs are produced (the first pass of the
@@ -546,28 +546,6 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
-  // ---- merge: the CTA whose partials complete a (b, g) merges that (b, g)
-  // (a count per (b, g); no CTA waits for another).  An aborted CTA adds no
-  // count: its (b, g) stay unmerged, and the error word says so.
-  if (*abort_flag) return;
-  __threadfence();  // this thread's partials, before the count that publishes them
-  __syncthreads();
-  __shared__ int s_last;
-  int* counts = merge_counters_of(a.ws, s);
-  for (int i = 0; i < nb; ++i) {
-    const int bg = bg_lo + i;
-    const long long base = (long long)bg * plan.S;
-    const int nv = tc_owner(base + plan.S - 1, U, gridDim.x) - tc_owner(base, U, gridDim.x) + 1;
-    if (threadIdx.x == 0) s_last = atomicAdd(counts + bg, 1) == nv - 1;
-    __syncthreads();
-    if (s_last) {
-      __threadfence();  // the other CTAs' partials, after their counts
-      for (int r = warp; r < R; r += THREADS / 32)
-        merge_row<__nv_bfloat16, D>(part, s, plan.nslot, bg, r, nv,
-                                    reinterpret_cast<__nv_bfloat16*>(a.O), a.lse, lane);
-    }
-    __syncthreads();
-  }
 }
 
 // Whether the key-major kernel takes this call: bf16, head dim 128, block or
@@ -592,9 +570,6 @@ cudaError_t launch_attn_tc_kt(const AttnArgs& a, int max_tiles, cudaStream_t st)
   const TcLaunch L = tc_plan((int)n_bg, max_tiles, tc_sm_count());
   if (L.plan.nslot > kMaxSplits) return cudaErrorInvalidValue;  // workspace bound
   cudaError_t e;
-  // the merge counts start at zero (the kernel merges; no combine launch)
-  if ((e = cudaMemsetAsync(merge_counters_of(a.ws, s), 0, n_bg * sizeof(int), st)) != cudaSuccess)
-    return e;
   if (a.O == nullptr) {  // the row LSEs only
     constexpr int smem = kt::Layout<true>::SMEM;
     if ((e = cudaFuncSetAttribute(attn_tc_kt_kernel<true>,
@@ -610,7 +585,8 @@ cudaError_t launch_attn_tc_kt(const AttnArgs& a, int max_tiles, cudaStream_t st)
     DL_LAUNCH(attn_tc_kt_kernel<false>, L.grid, kt::THREADS, smem, st, mq, mk, mv, mkd, mvd, a,
               L.plan);
   }
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return launch_combine(a, L.plan.nslot, st, L.plan.S, L.grid);
 }
 
 }  // namespace dl

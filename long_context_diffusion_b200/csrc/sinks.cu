@@ -232,7 +232,9 @@ sink_mass_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q
 }
 
 // Top-n columns by mass (ties to the lower position), ascending.  Any n:
-// n rounds of a block argmax over a scan of the masses.
+// n rounds of a block argmax over a scan of the masses, round k over the
+// columns strictly after round k-1's winner in (mass desc, position asc)
+// order (the masses are left as they are).
 __global__ void __launch_bounds__(1024)
 sink_topn_scan_kernel(Shape s, int n_sinks, SinkWs w, int32_t* __restrict__ sink_pos) {
   pdl_trigger();
@@ -241,22 +243,23 @@ sink_topn_scan_kernel(Shape s, int n_sinks, SinkWs w, int32_t* __restrict__ sink
   __shared__ int si[32];
   __shared__ int chosen[64];
   const int b = blockIdx.x;
-  float* mass = w.mass + (size_t)b * s.L_ctx;
+  const float* mass = w.mass + (size_t)b * s.L_ctx;
+  float pv = INFINITY;  // the previous winner
+  int pi = -1;
   for (int round = 0; round < n_sinks; ++round) {
     float v = -INFINITY;
     int idx = 0x7fffffff;
     for (int t = threadIdx.x; t < s.L_ctx; t += blockDim.x) {
       const float m = mass[t];
-      if (m > v || (m == v && t < idx)) { v = m; idx = t; }
+      const bool after = m < pv || (m == pv && t > pi);
+      if (after && (m > v || (m == v && t < idx))) { v = m; idx = t; }
     }
     float bv;
     int bi;
     block_argmax(v, idx, sv, si, bv, bi);
-    if (threadIdx.x == 0) {
-      chosen[round] = bi < s.L_ctx ? bi : -1;
-      if (bi < s.L_ctx) mass[bi] = -INFINITY;
-    }
-    __threadfence_block();
+    if (threadIdx.x == 0) chosen[round] = bi < s.L_ctx ? bi : -1;
+    pv = bv;
+    pi = bi;
     __syncthreads();
   }
   if (threadIdx.x == 0) {
@@ -444,7 +447,6 @@ cudaError_t launch_sink_mass(const Shape& s, const void* Q, const int32_t* q_idx
 }
 
 // The n_sinks columns of largest mass (ties to the lower position), ascending.
-// More than 8 sinks: the chosen columns of mass are overwritten with -inf.
 cudaError_t launch_sink_topn_mass(float* mass, int batch, int L_ctx, int n_sinks,
                                   int32_t* sink_pos, cudaStream_t st) {
   Shape s{};
@@ -465,11 +467,13 @@ cudaError_t launch_sinks(const Shape& s, const void* Q, const int32_t* q_idx,
   float* mass = tc ? sink_tc_ws(ws, s).mass : sink_ws(ws, s).mass;
   cudaError_t e = launch_sink_mass(s, Q, q_idx, q_cnt, Kp, page_table, Kd, mass, ws, err, st);
   if (e != cudaSuccess) return e;
-  if (Kexp && sink_cert_supported(s, n_sinks))
+  if ((e = launch_sink_topn_mass(mass, s.batch, s.L_ctx, n_sinks, sink_pos, st)) != cudaSuccess)
+    return e;
+  if (Kexp && sink_cert_supported(s, n_sinks))  // certify the top n (sinks_cert.cu)
     return launch_sink_cert(s, Q, q_idx, q_cnt, Kp, page_table, Kd, Kexp,
                             (s.L_ctx + s.page - 1) / s.page, mass, n_sinks, sink_pos,
                             reinterpret_cast<char*>(ws) + sinks_mass_workspace(s), err, st);
-  return launch_sink_topn_mass(mass, s.batch, s.L_ctx, n_sinks, sink_pos, st);
+  return cudaSuccess;
 }
 
 }  // namespace dl

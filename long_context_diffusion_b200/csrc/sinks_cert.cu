@@ -33,8 +33,10 @@
 // are exact up to fp64 rounding (products of bf16 or fp32 values are exact
 // in fp64).
 //
-// Kernels: band (one CTA per sequence: norms, eps, radix select of v_n, the
-// candidates in position order); lse64 (CTA per (512-key chunk, b, h): fp64
+// Kernels (after the top-n kernel of sinks.cu has written its n columns):
+// band (one CTA per sequence: norms, eps, v_n = the smallest of the n
+// masses, the count reaching thr, and when it is not n the candidates in
+// position order); lse64 (CTA per (512-key chunk, b, h): fp64
 // logits of up to 32 predicted rows at a time in shared memory, the chunk's
 // (max, sum) per row); lse64 merge; candidate mass (CTA per (candidate, b));
 // pick (one CTA per sequence: n rounds of a block argmax in (mass desc,
@@ -125,9 +127,6 @@ sink_band_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q
   __shared__ int s_kn[sc::kMaxKvHeads];  // float bits (non-negative: int order = float order)
   __shared__ int s_qk;                   // float bits of max scale ||q|| ||k||
   __shared__ int s_warp[33];
-  __shared__ int s_hist[256];
-  __shared__ unsigned s_prefix;
-  __shared__ int s_rank;
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NW = sc::kBandThreads / 32;
   const int L = s.L_ctx;
@@ -135,7 +134,7 @@ sink_band_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q
   const int nq = min(max(q_cnt[b], 0), s.L_q);
   int32_t* out = sink_pos + (size_t)b * n_sinks;
 
-  if (nq == 0) {  // no predicted rows: every mass is exactly zero
+  if (nq == 0) {  // no predicted rows: every mass is exactly zero, the top n are 0 .. n-1
     if (tid < n_sinks) out[tid] = tid;
     if (tid == 0) w.flag[b] = 0;
     return;
@@ -186,74 +185,67 @@ sink_band_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q
   const double eps = 4.0 * delta + ((double)L / 32.0 + (double)s.H * nq + 512.0) * 0x1p-24 +
                      0x1p-20;
 
-  // ---- v_n: radix select of the n-th largest mass (non-negative fp32 bits)
-  unsigned prefix = 0u, pmask = 0u;
-  int rank = n_sinks;  // 1-based rank among the keys matching the prefix
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += blockDim.x) s_hist[i] = 0;
-    __syncthreads();
-    for (int t = tid; t < L; t += blockDim.x) {
-      const unsigned u = __float_as_uint(fmaxf(m[t], 0.0f));
-      if ((u & pmask) == prefix) atomicAdd(&s_hist[(u >> shift) & 255u], 1);
+  // ---- v_n: the smallest mass among the top n (sink_pos holds them)
+  __shared__ float s_vn;
+  __shared__ int s_cnt;
+  if (tid == 0) {
+    float vn = INFINITY;
+    for (int i = 0; i < n_sinks; ++i) {
+      const int p = out[i];
+      vn = fminf(vn, (p >= 0 && p < L) ? fmaxf(m[p], 0.0f) : 0.0f);
     }
-    __syncthreads();
-    if (tid == 0) {
-      int acc = 0, d = 255;
-      for (; d > 0; --d) {
-        if (acc + s_hist[d] >= rank) break;
-        acc += s_hist[d];
-      }
-      s_prefix = prefix | ((unsigned)d << shift);
-      s_rank = rank - acc;
-    }
-    __syncthreads();
-    prefix = s_prefix;
-    rank = s_rank;
-    pmask |= 255u << shift;
-    __syncthreads();
+    s_vn = vn;
+    s_cnt = 0;
   }
-  const double vn = (double)__uint_as_float(prefix);
-  const double thr = vn * (1.0 - eps) / (1.0 + eps);
-
-  // ---- the columns reaching thr, in position order
-  int total = 0;
-  for (int t0 = 0; t0 < L; t0 += blockDim.x) {
+  __syncthreads();
+  const double thr = (double)s_vn * (1.0 - eps) / (1.0 + eps);
+  // ---- how many columns reach thr: exactly n -> the top n are certified
+  int cnt = 0;
+  for (int t = tid; t < L; t += blockDim.x) cnt += (double)fmaxf(m[t], 0.0f) >= thr ? 1 : 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if (lane == 0) atomicAdd(&s_cnt, cnt);
+  __syncthreads();
+  const int total = s_cnt;
+  if (total == n_sinks) {
+    if (tid == 0) w.flag[b] = 0;
+    return;
+  }
+  // ---- undecided: the columns reaching thr, in position order
+  int done = 0;
+  for (int t0 = 0; t0 < L && total <= sc::kCap; t0 += blockDim.x) {
     const int t = t0 + tid;
     const bool in = t < L && (double)fmaxf(m[t], 0.0f) >= thr;
     int chunk_total = 0;
-    const int pos = total + block_exclusive_count(in, s_warp, &chunk_total);
-    if (in) {
-      if (pos < n_sinks) out[pos] = t;  // the sinks when exactly n columns reach thr
-      if (pos < sc::kCap) w.cand[(size_t)b * sc::kCap + pos] = t;
-    }
-    total += chunk_total;
+    const int pos = done + block_exclusive_count(in, s_warp, &chunk_total);
+    if (in && pos < sc::kCap) w.cand[(size_t)b * sc::kCap + pos] = t;
+    done += chunk_total;
   }
   if (tid == 0) {
     w.count[b] = total;
-    w.flag[b] = total == n_sinks ? 0 : (total <= sc::kCap ? 1 : 2);
+    w.flag[b] = total <= sc::kCap ? 1 : 2;
   }
 }
 
 // ---------------------------------------------------------------- fp64 LSE
-// CTA (chunk c, b*H + h): keys c*kChunk .. of the concatenation (context,
-// decode block); fp64 logits of kRows predicted rows at a time.
+// One 512-key chunk of the concatenation (context, decode block) for
+// (b, h): fp64 logits of kRows predicted rows at a time in shared memory,
+// then the chunk's (max, sum) of each row.
 template <typename T, int D>
-__global__ void __launch_bounds__(sc::kThreads)
-sink_lse64_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
-                  const int32_t* __restrict__ q_cnt, const T* __restrict__ Kp,
-                  const int32_t* __restrict__ page_table, const T* __restrict__ Kd,
-                  SinkCertWs w, unsigned* err) {
-  pdl_trigger();
-  pdl_wait();
-  const int bh = blockIdx.y, b = bh / s.H, h = bh % s.H, g = h / s.G;
-  if (w.flag[b] == 0) return;
+__device__ __forceinline__ void sink_lse64_chunk(const Shape& s, const T* __restrict__ Q,
+                                                 const int32_t* __restrict__ q_idx,
+                                                 const int32_t* __restrict__ q_cnt,
+                                                 const T* __restrict__ Kp,
+                                                 const int32_t* __restrict__ page_table,
+                                                 const T* __restrict__ Kd, const SinkCertWs& w,
+                                                 unsigned* err, int b, int h, int g, int bh,
+                                                 int chunk, int nch) {
   extern __shared__ __align__(16) uint8_t smem_b[];
   double* sQ = reinterpret_cast<double*>(smem_b);  // [kRows][D]
   double* sL = sQ + sc::kRows * D;                  // [kRows][kChunk]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nq = min(max(q_cnt[b], 0), s.L_q);
-  const int nch = gridDim.x;
-  const long long t0 = (long long)blockIdx.x * sc::kChunk;
+  const long long t0 = (long long)chunk * sc::kChunk;
   const long long L_tot = (long long)s.L_ctx + s.L_q;
   for (int r0 = 0; r0 < nq; r0 += sc::kRows) {
     const int nr = min(sc::kRows, nq - r0);
@@ -307,8 +299,27 @@ sink_lse64_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ 
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
       if (lane == 0)
-        w.part[((size_t)bh * nch + blockIdx.x) * s.L_q + r0 + rr] = make_double2(mx, sum);
+        w.part[((size_t)bh * nch + chunk) * s.L_q + r0 + rr] = make_double2(mx, sum);
     }
+  }
+}
+
+// CTA (x, b*H + h): chunks x, x + gridDim.x, ... of (b, h); returns at once
+// for a certified sequence.
+template <typename T, int D>
+__global__ void __launch_bounds__(sc::kThreads)
+sink_lse64_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
+                  const int32_t* __restrict__ q_cnt, const T* __restrict__ Kp,
+                  const int32_t* __restrict__ page_table, const T* __restrict__ Kd,
+                  SinkCertWs w, int nch, unsigned* err) {
+  pdl_trigger();
+  pdl_wait();
+  const int bh = blockIdx.y, b = bh / s.H, h = bh % s.H, g = h / s.G;
+  if (w.flag[b] == 0) return;
+  for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
+    __syncthreads();
+    sink_lse64_chunk<T, D>(s, Q, q_idx, q_cnt, Kp, page_table, Kd, w, err, b, h, g, bh, chunk,
+                           nch);
   }
 }
 
@@ -333,21 +344,16 @@ sink_lse64_merge_kernel(Shape s, const int32_t* __restrict__ q_cnt, int nch, Sin
 }
 
 // ---------------------------------------------------------------- fp64 mass
-// CTA (candidate c, b): the candidate's fp64 mass, summed in (h, r) order
-// (per thread, then over the threads in a fixed tree).
+// Candidate c of sequence b: its fp64 mass, summed in (h, r) order (per
+// thread, then over the threads in a fixed tree).
 template <typename T, int D>
-__global__ void __launch_bounds__(sc::kThreads)
-sink_cand_mass_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
-                      const int32_t* __restrict__ q_cnt, const T* __restrict__ Kp,
-                      const int32_t* __restrict__ page_table, SinkCertWs w, unsigned* err) {
-  pdl_trigger();
-  pdl_wait();
-  __shared__ double s_red[sc::kThreads / 32];
-  const int b = blockIdx.y, c = blockIdx.x;
-  const int flag = w.flag[b];
-  if (flag == 0) return;
-  if (flag == 1 && c >= w.count[b]) return;
-  if (flag == 2 && c >= s.L_ctx) return;
+__device__ __forceinline__ void sink_cand_mass_one(const Shape& s, const T* __restrict__ Q,
+                                                   const int32_t* __restrict__ q_idx,
+                                                   const int32_t* __restrict__ q_cnt,
+                                                   const T* __restrict__ Kp,
+                                                   const int32_t* __restrict__ page_table,
+                                                   const SinkCertWs& w, unsigned* err, int b,
+                                                   int c, int flag, double* s_red) {
   const int t = flag == 1 ? w.cand[(size_t)b * sc::kCap + c] : c;
   const int nq = min(max(q_cnt[b], 0), s.L_q);
   const int slot = page_table[(size_t)b * s.n_pages + t / s.page];
@@ -382,6 +388,26 @@ sink_cand_mass_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restric
     double tot = 0.0;
     for (int i = 0; i < sc::kThreads / 32; ++i) tot += s_red[i];
     w.m64[(size_t)b * cert_m64_len(s) + c] = tot;
+  }
+}
+
+// CTA (x, b): candidates x, x + gridDim.x, ... (every column when there are
+// more than kCap); returns at once for a certified sequence.
+template <typename T, int D>
+__global__ void __launch_bounds__(sc::kThreads)
+sink_cand_mass_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
+                      const int32_t* __restrict__ q_cnt, const T* __restrict__ Kp,
+                      const int32_t* __restrict__ page_table, SinkCertWs w, unsigned* err) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ double s_red[sc::kThreads / 32];
+  const int b = blockIdx.y;
+  const int flag = w.flag[b];
+  if (flag == 0) return;
+  const int n_cols = flag == 1 ? w.count[b] : s.L_ctx;
+  for (int c = blockIdx.x; c < n_cols; c += gridDim.x) {
+    __syncthreads();
+    sink_cand_mass_one<T, D>(s, Q, q_idx, q_cnt, Kp, page_table, w, err, b, c, flag, s_red);
   }
 }
 
@@ -481,13 +507,13 @@ static cudaError_t run_cert(const Shape& s, const void* Q, const int32_t* q_idx,
   if ((e = cudaFuncSetAttribute(sink_lse64_kernel<T, D>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
     return e;
-  DL_LAUNCH(sink_lse64_kernel<T, D>, dim3(nch, s.batch * s.H), sc::kThreads, smem, st, s, q,
-            q_idx, q_cnt, kp, page_table, kd, w, err);
+  DL_LAUNCH(sink_lse64_kernel<T, D>, dim3(nch < 8 ? nch : 8, s.batch * s.H), sc::kThreads, smem,
+            st, s, q, q_idx, q_cnt, kp, page_table, kd, w, nch, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   DL_LAUNCH(sink_lse64_merge_kernel, s.batch * s.H, 256, 0, st, s, q_cnt, nch, w);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  DL_LAUNCH(sink_cand_mass_kernel<T, D>, dim3(cert_m64_len(s), s.batch), sc::kThreads, 0, st, s,
-            q, q_idx, q_cnt, kp, page_table, w, err);
+  DL_LAUNCH(sink_cand_mass_kernel<T, D>, dim3(sc::kCap, s.batch), sc::kThreads, 0, st, s, q,
+            q_idx, q_cnt, kp, page_table, w, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   DL_LAUNCH(sink_pick_kernel, s.batch, 1024, 0, st, s, n_sinks, w, sink_pos);
   return cudaGetLastError();

@@ -81,21 +81,10 @@ __host__ __device__ inline Partials partials_of(void* ws, const Shape& s, int n_
   return p;
 }
 
-// Per (b, g), how many of the CTAs that share it have written their partials
-// (the merge inside the persistent tensor-core kernel: the CTA that makes the
-// count complete merges them).  After the partials of kMaxSplits slots; zeroed
-// before each launch.
-__host__ __device__ inline int* merge_counters_of(void* ws, const Shape& s) {
-  const size_t n = (size_t)s.batch * s.H_kv * kMaxSplits * s.G * s.L_q;
-  return reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + round256(n * s.d * sizeof(float)) +
-                                round256(n * sizeof(float2)));
-}
-
 // Merge the split partials of one (b, g, row r) into O and lse: O = sum_s
 // acc_s e^{m_s-M} / L, L = sum_s l_s e^{m_s-M}, lse = M + ln L, over slots
 // [0, n_valid) of the n_split allocated.  One warp per row (lane = columns
-// lane, lane + 32, ...).  The partial loads go through L2 (ld.global.cg):
-// they may have been written by other CTAs of the running kernel.
+// lane, lane + 32, ...).
 template <typename T, int D>
 __device__ __forceinline__ void merge_row(const Partials& part, const Shape& s, int n_split,
                                           int bg, int r, int n_valid, T* __restrict__ O,
@@ -116,10 +105,10 @@ __device__ __forceinline__ void merge_row(const Partials& part, const Shape& s, 
     for (int q = 0; q < SB; ++q) {
       const size_t row = ((size_t)bg * n_split + s0 + q) * R + r;
       const bool ok = s0 + q < n_valid;
-      ml[q] = ok ? __ldcg(part.ml + row) : make_float2(-INFINITY, 0.0f);
+      ml[q] = ok ? part.ml[row] : make_float2(-INFINITY, 0.0f);
 #pragma unroll
       for (int c = 0; c < CPL; ++c)
-        ov[q][c] = (ok && O) ? __ldcg(part.o + row * D + lane + 32 * c) : 0.0f;
+        ov[q][c] = (ok && O) ? part.o[row * D + lane + 32 * c] : 0.0f;
     }
     // merge this batch into the running (M, L, o), as the partials themselves
     float Mb = M;

@@ -111,10 +111,18 @@ class ChunkOutputs:
 
 def chunked_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec, v_dec, *,
                  n_chunks: int, stride: int, content: int, topK_chunks: int, topT: int,
-                 Kbar=None, Kexp=None, ws=None, stream=None) -> ChunkOutputs:
+                 Kbar=None, Kexp=None, ws=None, stream=None,
+                 certify_tokens: bool = False) -> ChunkOutputs:
     """Chunked-prefix step: chunk keys (BOS excluded), chunk scores from
     every decode query, top-K chunks, top-T tokens per chunk plus its BOS,
-    attention over the gathered tokens and the decode block."""
+    attention over the gathered tokens and the decode block.
+
+    certify_tokens: the top-T cut certified with the chunk keys' exponent
+    words (an undecided cut recomputed in fp64 inside the token kernel).  Off
+    by default: the bound on the fp32 tensor-core logits is about 1e-3 of the
+    masses, wider than the spacing of the masses at the cut of dense chunks,
+    so nearly every chunk would take the fp64 recheck (about 20 times the
+    step's time on the 32-chunk workload)."""
     dev = q_dec.device
     B, L_q, d, H, H_kv = desc.batch, desc.L_q, desc.d, desc.H, desc.H_kv
     if ws is None:
@@ -135,7 +143,7 @@ def chunked_step(desc: A.dl_attn_desc, q_dec, k_pool, v_pool, page_table, k_dec,
     tok_pos = _empty((B, H_kv, kc * (topT + 1)), torch.int32, dev)
     tok_cnt = _empty((B, H_kv), torch.int32, dev)
     A.dl_token_select(desc, q_dec, k_pool, page_table, chunk_idx, stride, content, topT, tok_pos,
-                      tok_cnt, ws, stream, Kexp=Kexp)
+                      tok_cnt, ws, stream, Kexp=Kexp if certify_tokens else None)
     O = _empty((B, L_q, H, d), q_dec.dtype, dev)
     lse = _empty((B, H, L_q), torch.float32, dev)
     A.dl_sparse_attn_gather(desc, q_dec, k_pool, v_pool, page_table, tok_pos, tok_cnt, k_dec,

@@ -182,14 +182,16 @@ def _bf16_step(x):
     return b.view(torch.bfloat16)
 
 
-def test_chunked_prefix_workload(cuda_device):
+@pytest.mark.parametrize("certify", [False, True])
+def test_chunked_prefix_workload(certify, cuda_device):
     wl = synth.workload("chunked32k")
     inp = synth.make_step_inputs(wl, device=cuda_device)
     desc = desc_for(wl)
     out = pipeline.chunked_step(desc, inp.q_dec, inp.k_pool, inp.v_pool, inp.page_table,
                                 inp.k_dec, inp.v_dec, n_chunks=wl.n_chunks,
                                 stride=wl.chunk_stride, content=wl.chunk_content,
-                                topK_chunks=wl.topK_chunks, topT=wl.topT_tokens)
+                                topK_chunks=wl.topK_chunks, topT=wl.topT_tokens,
+                                certify_tokens=certify)
     assert dl.dl_get_status() == dl.DL_OK
     ref = oracle.chunked_step(inp.q_dec.cpu(), inp.k_pool.cpu(), inp.v_pool.cpu(),
                               inp.page_table.cpu(), inp.k_dec.cpu(), inp.v_dec.cpu(),

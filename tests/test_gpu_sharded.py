@@ -74,15 +74,15 @@ def test_shard_masses_sum_to_the_sinks(name, world, cuda_device):
     for b in range(wl.batch):
         if cut_margin(mass[b], top[b]) > 1e-5 * mass[b].max():
             assert np_(sinks)[b].tolist() == top[b].tolist()
-    if wl.G == 1:
+    if wl.G == 1 and inp.sinks_planted.shape[-1] == n:
         assert np_(sinks).tolist() == np_(inp.sinks_planted).tolist()
 
 
 @pytest.mark.parametrize("n", [4, 12])
 def test_split_calls_equal_find_sinks(n, cuda_device):
     """One shard of every head: dl_sink_mass then dl_sink_topn give exactly
-    what dl_find_sinks gives (the same kernels); with more than 8 sinks the
-    top-n scan overwrites the chosen columns of the mass with -inf."""
+    what dl_find_sinks without exponent words gives (the same kernels), and
+    both top-n kernels leave the mass as it is."""
     wl = synth.workload("llada8k")
     inp = synth.make_step_inputs(wl, device=cuda_device)
     desc = desc_for(wl)
@@ -99,13 +99,7 @@ def test_split_calls_equal_find_sinks(n, cuda_device):
     dl.dl_sink_topn(mass, sinks)
     assert dl.dl_get_status() == dl.DL_OK
     assert torch.equal(sinks, ref)
-    chosen = torch.zeros_like(mass, dtype=torch.bool)
-    chosen.scatter_(1, sinks.long(), True)
-    if n > 8:
-        assert torch.isneginf(mass[chosen]).all()
-        assert torch.equal(mass[~chosen], before[~chosen])
-    else:
-        assert torch.equal(mass, before)
+    assert torch.equal(mass, before)
 
 
 def test_sink_group_of_one_rank_takes_the_split_path(cuda_device):
