@@ -140,7 +140,8 @@ def test_sink_group_of_one_rank_takes_the_split_path(cuda_device):
         assert torch.equal(a.sink_pos, b.sink_pos)
         assert np_(a.sink_pos).tolist() == np_(x0.sinks_planted).tolist()
         for l in range(3):
-            assert torch.equal(a.blk_idx[l], b.blk_idx[l])
+            if l >= wl.first_sparse_layer:  # dense layers select nothing
+                assert torch.equal(a.blk_idx[l], b.blk_idx[l])
             assert torch.equal(a.O[l], b.O[l])
     finally:
         if group_owner:
