@@ -748,10 +748,10 @@ def count_launches(wl):
     certified sink search, and one score + select kernel per sparse layer when
     the group's rows fit a fused kernel (else three)."""
     n_sparse = wl.n_layers - wl.first_sparse_layer
-    # sinks: LSE pass + combine, mass, top-n, and the certification (band,
-    # fp64 LSE, merge, candidate masses, pick: the last four return at once
-    # when the cut is certified)
-    pool, predict, attn, sinks = 1, 1, 2, 9
+    # sinks: LSE pass + combine, mass, top-n, and the certification (bound,
+    # band count, band final, fp64 LSE, merge, candidate masses, pick: the
+    # last four return at once when the cut is certified)
+    pool, predict, attn, sinks = 1, 1, 2, 11
     rows = wl.G * min(wl.L_q, wl.k * (2 * wl.w + 1))
     fused = rows <= 32 and wl.n_blk <= 512
     score_select = 1 if fused else 3

@@ -34,9 +34,10 @@
 // in fp64).
 //
 // Kernels (after the top-n kernel of sinks.cu has written its n columns):
-// band (one CTA per sequence: norms, eps, v_n = the smallest of the n
-// masses, the count reaching thr, and when it is not n the candidates in
-// position order); lse64 (CTA per (512-key chunk, b, h): fp64
+// bound (CTA per (b, g): the group's largest ||q|| ||k||), band count (CTAs
+// over slices of the columns: eps, v_n = the smallest of the n masses, the
+// columns reaching thr), band final (CTA per sequence: certified, or the
+// candidates in position order); lse64 (CTA per (512-key chunk, b, h): fp64
 // logits of up to 32 predicted rows at a time in shared memory, the chunk's
 // (max, sum) per row); lse64 merge; candidate mass (CTA per (candidate, b));
 // pick (one CTA per sequence: n rounds of a block argmax in (mass desc,
@@ -61,6 +62,8 @@ constexpr int kMaxKvHeads = 256;
 struct SinkCertWs {
   int* flag;      // [b]: 0 certified, 1 candidates, 2 every column
   int* count;     // [b]: columns reaching the threshold
+  float* qk;      // [b][H_kv]: largest ||q|| ||k|| bound of the KV group
+  double* thr;    // [b]: the threshold
   int* cand;      // [b][kCap], ascending positions
   double* m64;    // [b][max(kCap, L_ctx)]: fp64 masses of the candidates
   double2* part;  // [b*H][n_chunks][L_q]: (max, sum) of each chunk
@@ -77,6 +80,8 @@ __host__ __device__ inline int cert_m64_len(const Shape& s) {
 size_t sink_cert_workspace(const Shape& s) {
   const size_t bh = (size_t)s.batch * s.H;
   return round256((size_t)s.batch * 2 * sizeof(int)) +
+         round256((size_t)s.batch * s.H_kv * sizeof(float)) +
+         round256((size_t)s.batch * sizeof(double)) +
          round256((size_t)s.batch * sc::kCap * sizeof(int)) +
          round256((size_t)s.batch * cert_m64_len(s) * sizeof(double)) +
          round256(bh * cert_chunks(s) * s.L_q * sizeof(double2)) +
@@ -90,6 +95,10 @@ static SinkCertWs sink_cert_ws(void* ws, const Shape& s) {
   w.flag = reinterpret_cast<int*>(p);
   w.count = w.flag + s.batch;
   p += round256((size_t)s.batch * 2 * sizeof(int));
+  w.qk = reinterpret_cast<float*>(p);
+  p += round256((size_t)s.batch * s.H_kv * sizeof(float));
+  w.thr = reinterpret_cast<double*>(p);
+  p += round256((size_t)s.batch * sizeof(double));
   w.cand = reinterpret_cast<int*>(p);
   p += round256((size_t)s.batch * sc::kCap * sizeof(int));
   w.m64 = reinterpret_cast<double*>(p);
@@ -116,41 +125,32 @@ __device__ __forceinline__ float norm_up(float sq_sum) {
 }
 
 // ---------------------------------------------------------------- band
+// (1) CTA per (b, g): the group's bound ||q|| ||k|| -- the largest key norm
+// (the blocks' norm fields and the decode keys) times the largest norm of the
+// predicted rows of the group's heads.  Also clears the sequence's count.
 template <typename T, int D>
-__global__ void __launch_bounds__(sc::kBandThreads)
-sink_band_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
-                 const int32_t* __restrict__ q_cnt, const T* __restrict__ Kd,
-                 const int32_t* __restrict__ Kexp, int n_units, const float* __restrict__ mass,
-                 int n_sinks, SinkCertWs w, int32_t* __restrict__ sink_pos) {
+__global__ void __launch_bounds__(256)
+sink_bound_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
+                  const int32_t* __restrict__ q_cnt, const T* __restrict__ Kd,
+                  const int32_t* __restrict__ Kexp, int n_units, SinkCertWs w) {
   pdl_trigger();
   pdl_wait();
-  __shared__ int s_kn[sc::kMaxKvHeads];  // float bits (non-negative: int order = float order)
-  __shared__ int s_qk;                   // float bits of max scale ||q|| ||k||
-  __shared__ int s_warp[33];
-  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int NW = sc::kBandThreads / 32;
-  const int L = s.L_ctx;
-  const float* m = mass + (size_t)b * L;
-  const int nq = min(max(q_cnt[b], 0), s.L_q);
-  int32_t* out = sink_pos + (size_t)b * n_sinks;
-
-  if (nq == 0) {  // no predicted rows: every mass is exactly zero, the top n are 0 .. n-1
-    if (tid < n_sinks) out[tid] = tid;
-    if (tid == 0) w.flag[b] = 0;
-    return;
+  __shared__ int s_kn, s_qn;  // float bits (non-negative: int order = float order)
+  const int bg = blockIdx.x, b = bg / s.H_kv, g = bg % s.H_kv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = 256 / 32;
+  if (tid == 0) {
+    s_kn = 0;
+    s_qn = 0;
+    if (g == 0) w.count[b] = 0;
   }
-  // ---- key norms per KV head: the context blocks' bounds and the decode keys
-  for (int g = tid; g < s.H_kv; g += blockDim.x) s_kn[g] = 0;
-  if (tid == 0) s_qk = 0;
   __syncthreads();
-  for (long long e = tid; e < (long long)s.H_kv * n_units; e += blockDim.x) {
-    const int g = (int)(e / n_units);
-    const float kn = key_norm_of(__ldg(Kexp + ((size_t)b * s.H_kv) * n_units + e));
-    atomicMax(&s_kn[g], __float_as_int(kn));
-  }
-  for (int e = warp; e < s.H_kv * s.L_q; e += NW) {  // warp per decode key
-    const int g = e / s.L_q, i = e % s.L_q;
-    const T* k = Kd + (((size_t)b * s.H_kv + g) * s.L_q + i) * D;
+  const int nq = min(max(q_cnt[b], 0), s.L_q);
+  float kn = 0.0f;
+  for (int u = tid; u < n_units; u += blockDim.x)
+    kn = fmaxf(kn, key_norm_of(__ldg(Kexp + (size_t)bg * n_units + u)));
+  for (int i = warp; i < s.L_q; i += NW) {  // warp per decode key
+    const T* k = Kd + ((size_t)bg * s.L_q + i) * D;
     float sq = 0.0f;
     for (int c = lane; c < D; c += 32) {
       const float v = to_float(k[c]);
@@ -158,11 +158,11 @@ sink_band_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    if (lane == 0) atomicMax(&s_kn[g], __float_as_int(norm_up(sq)));
+    kn = fmaxf(kn, norm_up(sq));
   }
-  __syncthreads();
-  for (int e = warp; e < s.H * nq; e += NW) {  // warp per predicted row
-    const int h = e / nq, r = e % nq;
+  float qn = 0.0f;
+  for (int e = warp; e < s.G * nq; e += NW) {  // warp per predicted row of the group
+    const int h = g * s.G + e / nq, r = e % nq;
     const int i = q_idx[(size_t)b * s.L_q + r];
     float sq = 0.0f;
     if (i >= 0 && i < s.L_q) {
@@ -174,57 +174,98 @@ sink_band_kernel(Shape s, const T* __restrict__ Q, const int32_t* __restrict__ q
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    if (lane == 0) {
-      const float qk = norm_up(sq) * __int_as_float(s_kn[h / s.G]);
-      atomicMax(&s_qk, __float_as_int(qk));
-    }
+    qn = fmaxf(qn, norm_up(sq));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kn = fmaxf(kn, __shfl_xor_sync(0xffffffffu, kn, o));
+    qn = fmaxf(qn, __shfl_xor_sync(0xffffffffu, qn, o));
+  }
+  if (lane == 0) {
+    atomicMax(&s_kn, __float_as_int(kn));
+    atomicMax(&s_qn, __float_as_int(qn));
   }
   __syncthreads();
-  const double B = s.scale * (double)__int_as_float(s_qk) * (1.0 + 0x1p-20);
-  const double delta = B * (D + 2) * 0x1p-23;
-  const double eps = 4.0 * delta + ((double)L / 32.0 + (double)s.H * nq + 512.0) * 0x1p-24 +
-                     0x1p-20;
+  if (tid == 0) w.qk[bg] = __fmul_ru(__int_as_float(s_qn), __int_as_float(s_kn));
+}
 
-  // ---- v_n: the smallest mass among the top n (sink_pos holds them)
-  __shared__ float s_vn;
+// eps and thr of sequence b (every caller computes the same numbers).
+__device__ __forceinline__ double sink_threshold(const Shape& s, const SinkCertWs& w, int b,
+                                                 int nq, const float* m, const int32_t* top,
+                                                 int n_sinks, int D) {
+  float qk = 0.0f;
+  for (int g = 0; g < s.H_kv; ++g) qk = fmaxf(qk, w.qk[(size_t)b * s.H_kv + g]);
+  const double B = s.scale * (double)qk * (1.0 + 0x1p-20);
+  const double delta = B * (D + 2) * 0x1p-23;
+  const double eps = 4.0 * delta + ((double)s.L_ctx / 32.0 + (double)s.H * nq + 512.0) * 0x1p-24 +
+                     0x1p-20;
+  float vn = INFINITY;  // the smallest mass among the top n
+  for (int i = 0; i < n_sinks; ++i) {
+    const int p = top[i];
+    vn = fminf(vn, (p >= 0 && p < s.L_ctx) ? fmaxf(m[p], 0.0f) : 0.0f);
+  }
+  return (double)vn * (1.0 - eps) / (1.0 + eps);
+}
+
+// (2) CTA per (slice, b): how many columns of the slice reach thr.
+__global__ void __launch_bounds__(256)
+sink_band_count_kernel(Shape s, const int32_t* __restrict__ q_cnt, const float* __restrict__ mass,
+                       int n_sinks, const int32_t* __restrict__ sink_pos, SinkCertWs w, int D) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ double s_thr;
   __shared__ int s_cnt;
+  const int b = blockIdx.y, tid = threadIdx.x;
+  const int nq = min(max(q_cnt[b], 0), s.L_q);
+  if (nq == 0) return;
+  const float* m = mass + (size_t)b * s.L_ctx;
   if (tid == 0) {
-    float vn = INFINITY;
-    for (int i = 0; i < n_sinks; ++i) {
-      const int p = out[i];
-      vn = fminf(vn, (p >= 0 && p < L) ? fmaxf(m[p], 0.0f) : 0.0f);
-    }
-    s_vn = vn;
+    s_thr = sink_threshold(s, w, b, nq, m, sink_pos + (size_t)b * n_sinks, n_sinks, D);
     s_cnt = 0;
+    if (blockIdx.x == 0) w.thr[b] = s_thr;
   }
   __syncthreads();
-  const double thr = (double)s_vn * (1.0 - eps) / (1.0 + eps);
-  // ---- how many columns reach thr: exactly n -> the top n are certified
+  const double thr = s_thr;
+  const long long per = ((long long)s.L_ctx + gridDim.x - 1) / gridDim.x;
+  const long long t0 = (long long)blockIdx.x * per;
+  const long long t1 = min(t0 + per, (long long)s.L_ctx);
   int cnt = 0;
-  for (int t = tid; t < L; t += blockDim.x) cnt += (double)fmaxf(m[t], 0.0f) >= thr ? 1 : 0;
+  for (long long t = t0 + tid; t < t1; t += blockDim.x) cnt += (double)fmaxf(m[t], 0.0f) >= thr;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-  if (lane == 0) atomicAdd(&s_cnt, cnt);
+  if ((tid & 31) == 0 && cnt) atomicAdd(&s_cnt, cnt);
   __syncthreads();
-  const int total = s_cnt;
-  if (total == n_sinks) {
+  if (tid == 0 && s_cnt) atomicAdd(w.count + b, s_cnt);
+}
+
+// (3) CTA per sequence: certified when exactly n columns reach thr (the top
+// n of sink_pos stand); otherwise the candidates in position order.
+__global__ void __launch_bounds__(sc::kBandThreads)
+sink_band_final_kernel(Shape s, const int32_t* __restrict__ q_cnt,
+                       const float* __restrict__ mass, int n_sinks, SinkCertWs w,
+                       int32_t* __restrict__ sink_pos) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int s_warp[33];
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int nq = min(max(q_cnt[b], 0), s.L_q);
+  const int total = w.count[b];
+  if (nq == 0 || total == n_sinks) {  // no rows: every mass is 0, the top n are 0 .. n-1
     if (tid == 0) w.flag[b] = 0;
     return;
   }
-  // ---- undecided: the columns reaching thr, in position order
+  const float* m = mass + (size_t)b * s.L_ctx;
+  const double thr = w.thr[b];
   int done = 0;
-  for (int t0 = 0; t0 < L && total <= sc::kCap; t0 += blockDim.x) {
+  for (int t0 = 0; t0 < s.L_ctx && total <= sc::kCap; t0 += blockDim.x) {
     const int t = t0 + tid;
-    const bool in = t < L && (double)fmaxf(m[t], 0.0f) >= thr;
+    const bool in = t < s.L_ctx && (double)fmaxf(m[t], 0.0f) >= thr;
     int chunk_total = 0;
     const int pos = done + block_exclusive_count(in, s_warp, &chunk_total);
     if (in && pos < sc::kCap) w.cand[(size_t)b * sc::kCap + pos] = t;
     done += chunk_total;
   }
-  if (tid == 0) {
-    w.count[b] = total;
-    w.flag[b] = total <= sc::kCap ? 1 : 2;
-  }
+  if (tid == 0) w.flag[b] = total <= sc::kCap ? 1 : 2;
 }
 
 // ---------------------------------------------------------------- fp64 LSE
@@ -498,10 +539,16 @@ static cudaError_t run_cert(const Shape& s, const void* Q, const int32_t* q_idx,
   const T* q = reinterpret_cast<const T*>(Q);
   const T* kp = reinterpret_cast<const T*>(Kp);
   const T* kd = reinterpret_cast<const T*>(Kd);
-  DL_LAUNCH(sink_band_kernel<T, D>, s.batch, sc::kBandThreads, 0, st, s, q, q_idx, q_cnt, kd,
-            Kexp, n_units, mass, n_sinks, w, sink_pos);
+  DL_LAUNCH(sink_bound_kernel<T, D>, s.batch * s.H_kv, 256, 0, st, s, q, q_idx, q_cnt, kd, Kexp,
+            n_units, w);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  DL_LAUNCH(sink_band_count_kernel, dim3(32, s.batch), 256, 0, st, s, q_cnt, mass, n_sinks,
+            (const int32_t*)sink_pos, w, D);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  DL_LAUNCH(sink_band_final_kernel, s.batch, sc::kBandThreads, 0, st, s, q_cnt, mass, n_sinks, w,
+            sink_pos);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int nch = cert_chunks(s);
   const int smem = (sc::kRows * D + sc::kRows * sc::kChunk) * (int)sizeof(double);
   if ((e = cudaFuncSetAttribute(sink_lse64_kernel<T, D>,

@@ -129,34 +129,50 @@ def test_token_select_near_tie_at_the_cut(exact_tie, cuda_device):
     desc = dl.make_desc(batch=batch, H=H, H_kv=H_kv, d=d, L_ctx=L_ctx, L_q=L_q, page=page,
                         n_pages=n_pages, n_slots=n_slots, dtype=dl.DL_BF16)
     scale = oracle.scale_for(d)
-    a, bpos = 100, 900  # content offsets (positions base + 1 + offset)
+    bpos = 900  # content offsets (positions base + 1 + offset)
+    pt0 = page_table[0].numpy()
+
+    def taus(g):
+        keys = S.gather_context(S.f64(kp), pt0, g, base + 1 + np.arange(content), page)
+        return S.token_select(S.f64(q[0, g]), keys, topT, scale)[1]
+
+    def row(off, g):
+        pos = base + 1 + off
+        return (int(page_table[0, pos // page]), g, pos % page)
+
+    chosen_a = []
     for g in range(H_kv):
-        rows = S.f64(q[0, g])
-        keys = S.gather_context(S.f64(kp), page_table[0].numpy(), g,
-                                base + 1 + np.arange(content), page)
-        _, tau = S.token_select(rows, keys, topT, scale)
-        target = np.sort(tau)[-topT]  # the T-th mass: raise a's key until it reaches it
         qbar = q[0, g].to(torch.float32).mean(dim=0)
-        ra = (int(page_table[0, (base + 1 + a) // page]), g, (base + 1 + a) % page)
-        rb = (int(page_table[0, (base + 1 + bpos) // page]), g, (base + 1 + bpos) % page)
-        orig = kp[ra].to(torch.float32).clone()
-        lo, hi = 0.0, 20.0
-        for _ in range(40):
-            mid = (lo + hi) / 2
-            kp[ra] = (orig + mid * qbar).to(torch.bfloat16)
-            keys = S.gather_context(S.f64(kp), page_table[0].numpy(), g,
-                                    base + 1 + np.arange(content), page)
-            _, tau = S.token_select(rows, keys, topT, scale)
-            if tau[a] > target:
-                hi = mid
-            else:
-                lo = mid
-        kp[ra] = (orig + hi * qbar).to(torch.bfloat16)
-        kp[rb] = kp[ra]
+        rb = row(bpos, g)
+        for a in range(100, 120):  # a token whose boosted copy lands exactly on the cut
+            ra = row(a, g)
+            orig_a, orig_b = kp[ra].clone(), kp[rb].clone()
+
+            def put(boost):
+                kp[ra] = (orig_a.to(torch.float32) + boost * qbar).to(torch.bfloat16)
+                kp[rb] = kp[ra]
+
+            lo, hi = 0.0, 20.0  # smallest boost with a among the top T (both keys raised)
+            for _ in range(30):
+                mid = (lo + hi) / 2
+                put(mid)
+                rank_a = int((np.argsort(-taus(g), kind="stable") == a).nonzero()[0][0])
+                if rank_a <= topT - 1:
+                    hi = mid
+                else:
+                    lo = mid
+            put(hi)
+            order = np.argsort(-taus(g), kind="stable")
+            if order[topT - 1] == a and order[topT] == bpos:
+                chosen_a.append(a)
+                break
+            kp[ra], kp[rb] = orig_a, orig_b
+        else:
+            pytest.fail("no token could be placed on the cut")
         if not exact_tie:
-            row = kp[rb].clone()
-            row[7] = (row[7].view(torch.int16) + 1).view(torch.bfloat16)
-            kp[rb] = row
+            rw = kp[rb].clone()
+            rw[7] = (rw[7].view(torch.int16) + 1).view(torch.bfloat16)
+            kp[rb] = rw
     dev = cuda_device
     ws = torch.empty(max(dl.dl_workspace_size(desc), 256), dtype=torch.uint8, device=dev)
     per = topT + 1
@@ -168,12 +184,11 @@ def test_token_select_near_tie_at_the_cut(exact_tie, cuda_device):
     assert dl.dl_get_status() == dl.DL_OK
     got = np_(tok_pos)
     for g in range(H_kv):
-        rows = S.f64(q[0, g])
-        keys = S.gather_context(S.f64(kp), page_table[0].numpy(), g,
-                                base + 1 + np.arange(content), page)
-        off, tau = S.token_select(rows, keys, topT, scale)
+        a = chosen_a[g]
+        keys = S.gather_context(S.f64(kp), pt0, g, base + 1 + np.arange(content), page)
+        off, tau = S.token_select(S.f64(q[0, g]), keys, topT, scale)
         order = np.argsort(-tau, kind="stable")
-        assert {a, bpos} & set(order[topT - 1:topT + 1].tolist()), g  # at the cut
+        assert set(order[topT - 1:topT + 1].tolist()) == {a, bpos}, g  # straddling the cut
         gap = abs(tau[a] - tau[bpos]) / tau[a]
         assert (0.0 < gap < 1e-3) if not exact_tie else gap == 0.0
         mine = got[0, g, 1:] - base - 1
