@@ -370,7 +370,7 @@ static dl_status attn_common(const dl_attn_desc* desc, const void* Q_dec, const 
   if ((st = need_ws(ws, ws_bytes, dl::attn_workspace(s))) != DL_OK) return st;
   unsigned* err = nullptr;
   if ((st = error_word(&err)) != DL_OK) return st;
-  dl::AttnArgs a;
+  dl::AttnArgs a{};
   a.s = s; a.Q = Q_dec; a.Kp = K_pool; a.Vp = V_pool; a.page_table = page_table;
   a.mode = mode; a.idx = idx; a.cnt = cnt; a.max_idx = mode == dl::kDense ? 0 : max_idx;
   a.Kd = K_dec; a.Vd = V_dec; a.O = O; a.lse = lse; a.ws = ws; a.ws_bytes = ws_bytes; a.err = err;

@@ -38,7 +38,7 @@
 // exp(l) finite and normal, and the softmax does not depend on the shift.
 //
 // Roles (512 threads, 16 warps): thread 448 (warp 14, lane 0) streams the
-// key digit planes by TMA through a ring of nine 16 KB stages (128 keys x
+// key digit planes by TMA through a ring of ten 16 KB stages (128 keys x
 // 128 bytes, one plane each); thread 480 (warp 15, lane 0) copies the
 // group's decode rows, issues the MMAs and commits them, tile by tile, into
 // two alternating sets of accumulator columns.  Warpgroup w < MT drains row
@@ -68,7 +68,7 @@ namespace bstc {
 constexpr int kThreads = bs::kThreads;                   // 512: one key per thread
 constexpr int kTileKeys = 128;                           // keys per MMA tile (M)
 constexpr int kPlaneBytes = kTileKeys * 128;             // one digit plane of a tile: 16 KB
-constexpr int kStages = 9;                               // planes in flight per CTA
+constexpr int kStages = 10;                              // planes in flight per CTA
 constexpr int kLevels = kKeyDigits + kQueryDigits - 1;   // digit-pair weight levels: 8
 constexpr int kTmemCols = 512;
 constexpr int kQOff = kStages * kPlaneBytes;             // query digit planes after the ring
@@ -279,6 +279,7 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
   __shared__ int s_qpos[256], s_qcnt;
   __shared__ double s_exp_tab[64];
   __shared__ uint8_t s_sink[bs::kMaxUnits];
+  __shared__ int s_ke[bs::kMaxUnits];  // exponent field of every key (at least 1)
   __shared__ int s_cnt[72];
   __shared__ unsigned long long s_min[bs::kWarps];
   __shared__ RadixScratch s_rad;
@@ -388,6 +389,7 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
       em = Eu;
       nk = (ke >> 8) & 255;
     }
+    s_ke[tid] = Eu;
     em = __reduce_max_sync(0xffffffffu, em);
     nk = __reduce_max_sync(0xffffffffu, nk);
     if (lane == 0) {
@@ -534,8 +536,7 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
       const int tkey = t * kTileKeys + (tid & 127);
       const bool kok = tkey < n_units;
       if (ok && drains) {
-        const int ket = kok ? __ldg(Kexp + (size_t)bg * n_units + tkey) : 0;
-        const int et = max(ket & 255, 1);
+        const int et = kok ? s_ke[tkey] : 1;
         tc_fence_after();
         const uint32_t base = tmem + lane_base + (t & 1) * L::TILE_COLS + row0;
         // V = h0 2^42 + h1 2^28 + h2 2^14 + h3, h_k = A_2k * 128 + A_2k+1 (int32),
