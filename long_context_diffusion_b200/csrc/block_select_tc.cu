@@ -37,12 +37,11 @@
 // are taken without subtracting the row maximum: |l| <= B_r <= 700 keeps
 // exp(l) finite and normal, and the softmax does not depend on the shift.
 //
-// Roles (512 threads, 16 warps): the key digit planes stream by TMA through
-// a ring of ten 16 KB stages (128 keys x 128 bytes, one plane each); thread
-// 480 (warp 15, lane 0) sets up the barriers, issues the first ten planes at
-// entry and copies the group's decode rows, then issues the MMAs and commits
-// them, tile by tile, into two alternating sets of accumulator columns;
-// thread 448 (warp 14, lane 0) refills the ring as the MMAs free it.  Warpgroup w < MT drains row
+// Roles (512 threads, 16 warps): thread 448 (warp 14, lane 0) streams the
+// key digit planes by TMA through a ring of ten 16 KB stages (128 keys x
+// 128 bytes, one plane each); thread 480 (warp 15, lane 0) copies the
+// group's decode rows, issues the MMAs and commits them, tile by tile, into
+// two alternating sets of accumulator columns.  Warpgroup w < MT drains row
 // block w (query rows 8w .. 8w+7) of every tile: thread = key, the eight
 // level columns read from tensor memory, combined into fp64 logits, the
 // columns zeroed for the tile after next, and the exponentials kept in
@@ -292,7 +291,7 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
   const int tl = nt - 1;                                 // the last tile
   const int J = nt * kKeyDigits;                         // digit planes to stream
   const bool q_whole = s.G * s.L_q <= kQRawRows;         // decode rows prefetched whole
-  auto plane_load = [&](int j) {  // control thread (the first ring), then producer thread
+  auto plane_load = [&](int j) {  // producer thread only
     const int st = j % kStages;
     mbar_arrive_expect_tx(&full[st], kPlaneBytes);
     tma_load_3d(sK + st * kPlaneBytes, &kdig_map, 0, (j / kKeyDigits) * kTileKeys,
@@ -300,9 +299,10 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
   };
 
   pdl_wait();
-  // The control thread sets up the barriers, starts the key digit stream and
-  // copies the group's decode rows; the other threads issue their small loads
-  // (into registers; the barrier does not wait for them).
+  // The small loads are issued first (into registers; a barrier does not
+  // wait for them), so that they enter the memory queues ahead of the key
+  // digit stream, which starts right after the barrier.  The control thread
+  // sets up the barriers and copies the group's decode rows.
   if (tid == kCtl) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], 1);
@@ -315,19 +315,15 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
     abort_flag = 0;
     s_Emax = 1;
     s_NK = 0;
+    s_issued_tma = 0;
     s_issued_mma = 0;
     fence_mbar_init();
     prefetch_tmap(&kdig_map);
-    if (q_whole) {  // the decode rows first: the first MMAs need their digits
+    if (q_whole) {
       const uint32_t bytes = (uint32_t)(s.G * s.L_q * 256);
       mbar_arrive_expect_tx(&qfull, bytes);
       bulk_load(sQraw, Q + ((size_t)b * s.H + (size_t)g * s.G) * s.L_q * 128, bytes, &qfull);
     }
-    // the key digit stream starts here, before the block barrier: the first
-    // kStages planes (the producer thread refills the ring after it)
-    const int n0 = J < kStages ? J : kStages;
-    for (int j = 0; j < n0; ++j) plane_load(j);
-    s_issued_tma = n0;
   }
   const int key = tid;
   const bool key_ok = key < n_units;
@@ -349,6 +345,11 @@ block_select_tc_kernel(const __grid_constant__ CUtensorMap kdig_map,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  if (tid == kProd) {  // the key digit stream: the first kStages planes
+    const int n0 = J < kStages ? J : kStages;
+    for (int j = 0; j < n0; ++j) plane_load(j);
+    s_issued_tma = n0;
+  }
   if (warp == 1 && lane == 0) s_qcnt = qcnt;
   if (tid < 64) s_exp_tab[tid] = tabv;
   if (warp == 2 && lane < n_sinks && sp0 >= 0) {  // sink units (kept whatever their score)
