@@ -14,8 +14,8 @@
 //           cp.async;
 //   dot     warp = (4 rows, 32 units), lane = unit: per 4 dimensions one
 //           float4 of the key and one load of each row (the same address for
-//           the whole warp), fp64 FMAs in dimension order (so equal keys give
-//           equal logits);
+//           the whole warp); 16 fp64 FMA chains per lane (row x dimension mod
+//           4), added in a fixed order (so equal keys give equal logits);
 //   softmax warp per row: max, e^(l - max) in fp64, sum, divide;
 //   scores  thread per unit sums its column in row order;
 //   select  the bitonic sort and ascending write of the fused kernels.
@@ -126,7 +126,13 @@ block_select_wide_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_
   for (int it = warp; it < n_rg * n_ug; it += kWarps) {
     const int r0 = (it / n_ug) * 4, u = (it % n_ug) * 32 + lane;
     const float* kr = sK + u * L::KP;
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    // 16 independent chains: row i, dimension phase c (k = c mod 4), so the
+    // FMA latency is hidden; the phases are added in a fixed order
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[i][c] = 0.0;
 #pragma unroll 4
     for (int k = 0; k < D; k += 4) {
       const float4 kv = *reinterpret_cast<const float4*>(kr + k);
@@ -134,14 +140,15 @@ block_select_wide_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_
       for (int i = 0; i < 4; ++i) {
         double q[4];
         load4<T>(sQ + (size_t)(r0 + i) * D + k, q);
-        acc[i] = fma(q[0], (double)kv.x, acc[i]);
-        acc[i] = fma(q[1], (double)kv.y, acc[i]);
-        acc[i] = fma(q[2], (double)kv.z, acc[i]);
-        acc[i] = fma(q[3], (double)kv.w, acc[i]);
+        acc[i][0] = fma(q[0], (double)kv.x, acc[i][0]);
+        acc[i][1] = fma(q[1], (double)kv.y, acc[i][1]);
+        acc[i][2] = fma(q[2], (double)kv.z, acc[i][2]);
+        acc[i][3] = fma(q[3], (double)kv.w, acc[i][3]);
       }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) sL[(size_t)(r0 + i) * Uc + u] = acc[i] * sc;
+    for (int i = 0; i < 4; ++i)
+      sL[(size_t)(r0 + i) * Uc + u] = ((acc[i][0] + acc[i][1]) + (acc[i][2] + acc[i][3])) * sc;
   }
   __syncthreads();
 
