@@ -38,8 +38,9 @@
 // Every wait is bounded and the softmax warps exchange through mbarriers (no
 // named barriers), so a role that gives up cannot leave another waiting.
 // With O == nullptr only the row LSEs are produced (the first pass of the
-// sink search): the V ring, the O^T MMAs and all O work are skipped; with
-// row_idx the rows that are not predicted are skipped too (no LSE).
+// sink search): the V ring, the O^T MMAs and all O work are skipped.  (Also
+// skipping the rows that are not predicted measured no faster: the pass is
+// not bound by its exponentials.)
 #include <mutex>
 
 #include "sm100.cuh"
@@ -178,7 +179,6 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   pdl_wait();
   const int R = s.G * s.L_q;
   const int n_dec = (s.L_q + 63) / 64;
-  __shared__ uint32_t s_rowmask[kMaxSegs];  // LSE-only: wanted rows of each (b, g) in range
   const long long U = (long long)s.batch * s.H_kv * plan.S;
   const long long u0 = (long long)blockIdx.x * U / gridDim.x;
   const long long u1 = (long long)(blockIdx.x + 1) * U / gridDim.x;
@@ -187,23 +187,7 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // the (b, g) pairs this CTA's slots touch, their tile counts in parallel
   const int bg_lo = u1 > u0 ? (int)(u0 / plan.S) : 0;
   const int nb = u1 > u0 ? (int)((u1 - 1) / plan.S) - bg_lo + 1 : 0;  // <= kMaxSegs (plan)
-  if (threadIdx.x < nb) {
-    s_nctx[threadIdx.x] = ctx_tile_count(a, bg_lo + threadIdx.x);
-    // row r = (head of the group r / L_q, position r % L_q); R <= 32
-    uint32_t mask = R >= 32 ? 0xffffffffu : ((1u << R) - 1u);
-    if (lse_only && a.row_idx != nullptr) {
-      const int b = (bg_lo + threadIdx.x) / s.H_kv;
-      const int nq = min(max(a.row_cnt[b], 0), s.L_q);
-      uint32_t pos = 0u;  // predicted positions of the decode block
-      for (int i = 0; i < nq; ++i) {
-        const int p = a.row_idx[(size_t)b * s.L_q + i];
-        if (p >= 0 && p < s.L_q) pos |= 1u << p;
-      }
-      mask = 0u;
-      for (int h = 0; h < s.G; ++h) mask |= pos << (h * s.L_q);
-    }
-    s_rowmask[threadIdx.x] = mask;
-  }
+  if (threadIdx.x < nb) s_nctx[threadIdx.x] = ctx_tile_count(a, bg_lo + threadIdx.x);
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2 * (STK + STV); ++i) mbar_init(&full_k[i], 1);
     for (int i = 0; i < 2; ++i) {
@@ -453,10 +437,9 @@ attn_tc_kt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       tmem_ld_wait();
       float x[NQ];
       bool need = false;
-      const uint32_t rmask = s_rowmask[seg[k].x - bg_lo];  // rows kept (q < R)
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
-        x[q] = (kvalid && ((rmask >> q) & 1u)) ? __uint_as_float(sv[q]) * c2 : -INFINITY;
+        x[q] = (kvalid && q < R) ? __uint_as_float(sv[q]) * c2 : -INFINITY;
         need |= x[q] > m_ref[q] + 8.0f;
       }
       // vote: does any thread of the four warps need a larger reference?

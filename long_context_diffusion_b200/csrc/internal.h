@@ -43,10 +43,6 @@ struct AttnArgs {
   void* ws;
   size_t ws_bytes;
   unsigned* err;
-  // LSE-only calls: the rows whose LSE is wanted, the positions q_idx[b][0
-  // .. q_cnt[b]) of every head (nullptr: every row); the others are skipped
-  const int32_t* row_idx;
-  const int32_t* row_cnt;
 };
 
 // ---- workspace sizing (bytes; each region rounded up to 256) ----

@@ -427,13 +427,8 @@ cudaError_t launch_sink_mass(const Shape& s, const void* Q, const int32_t* q_idx
   a.idx = nullptr; a.cnt = nullptr; a.max_idx = 0; a.Kd = Kd; a.Vd = Kd; a.O = tw.O;
   a.lse = tw.lse; a.ws = tw.attn; a.ws_bytes = attn_workspace(s); a.err = err;
   if (s.dtype == 0 && s.G * s.L_q <= 256 && attn_tc_supported(a)) {
-    // the key-major kernel can skip V and O, and the rows that are not
-    // predicted: only the predicted rows' LSEs are needed
-    if (attn_tc_kt_supported(a)) {
-      a.O = nullptr;
-      a.row_idx = q_idx;
-      a.row_cnt = q_cnt;
-    }
+    // the key-major kernel can skip V and O: only the row LSEs are needed
+    if (attn_tc_kt_supported(a)) a.O = nullptr;
     cudaError_t e = launch_attn(a, st);
     if (e != cudaSuccess) return e;
     return launch_sink_mass_tc(s, Q, q_idx, q_cnt, Kp, page_table, tw.lse,
