@@ -55,9 +55,9 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 
 # DRAM traffic of the dominant kernel from one ncu capture at the benchmark's
 # size (dram__bytes_read.sum + dram__bytes_write.sum of one sparse-layer
-# launch, batch 4: 557.85 + 5.20 MB).  Reported only while the kernel's
+# launch, batch 4: 557.87 + 4.88 MB).  Reported only while the kernel's
 # sources hash to the captured build.
-TRAFFIC_CAPTURE = {"sha": "00b5fd594cdc7551", "bytes_per_launch": 557.846528e6 + 5.20192e6,
+TRAFFIC_CAPTURE = {"sha": "a1aa471f8011b5dd", "bytes_per_launch": 557.874688e6 + 4.879104e6,
                    "sources": ["attn_tc_kt.cu", "tc_common.cuh", "sm100.cuh"]}
 
 

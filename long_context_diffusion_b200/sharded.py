@@ -7,7 +7,7 @@ across layers).  Ranks hold disjoint, contiguous ranges of KV heads, each
 with its G query heads and only those heads' KV.  A rank computes its heads'
 part of the mass (dl_sink_mass), one all-reduce (sum) of mass[b][L_ctx] over
 the ranks gives the whole mass, and every rank picks the same sinks from it
-(dl_sink_topn).  Nothing else crosses GPUs: no peer loads, no multicast.
+(dl_sink_topn).  Nothing else crosses GPUs: no peer memory is read.
 
 The reduction sums fp32 partial masses in the collective's order, so near
 ties the chosen sinks can differ from a single-GPU run by the rounding of
