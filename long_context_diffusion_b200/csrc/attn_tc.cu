@@ -32,14 +32,15 @@
 //                        to shared memory in the MMA's K-major swizzled
 //                        layout, and at the end writes its partial (O, m, l).
 // Gathered tokens (the chunked prefix: arbitrary cached positions): a tile is
-// 64 consecutive entries of the (b, g)'s position list, and the whole
-// producer warp copies its rows with 16-byte cp.async into the same swizzled
-// layout (each lane resolves two rows' positions through the page table);
-// a tile is released to the MMAs (wait for the copies, proxy fence, arrive)
-// once ST - 1 newer gathered tiles are in flight, before the producer waits
-// for its ring slot again, and before the next segment's Q is loaded.  Rows
-// past a tile's valid keys are zero-filled by the copies.  Decode tiles keep
-// their TMA path.
+// 64 consecutive entries of the (b, g)'s position list.  The pool's tensor
+// maps then have one-row boxes and the whole producer warp loads the tile's
+// rows with TMA row gathers (four rows per instruction, lane = four rows of
+// one 64-column half) into the same swizzled layout, every lane's loads
+// completing on the tile's full barrier.  Each lane resolves two rows'
+// positions through the page table; rows past the tile's valid keys, or with
+// a bad position, take the row past the pool, which TMA fills with zeros (so
+// a NaN in an unused pool row never reaches P V).  Decode tiles keep their
+// tiled TMA path.
 // The G*L_q query rows of a KV group are padded to M-tiles of 128 rows (the
 // path is HBM-bound: padding costs tensor time, not bytes).  Partials of the
 // splits of one (b, g) are merged by the combine kernel of attn_simt.cu.
@@ -58,6 +59,19 @@
 namespace dl {
 
 using namespace sm100;
+
+// Four rows y0..y3 of a 2-D tensor map whose box is one row high, columns
+// [x, x + box width), to four consecutive box rows at dst (the map's swizzle
+// applied); rows past the tensor are filled with zeros.
+__device__ __forceinline__ void tma_gather4_2d(void* dst, const CUtensorMap* map, int x, int y0,
+                                               int y1, int y2, int y3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1),
+      "r"(y2), "r"(y3)
+      : "memory");
+}
 
 // D head dim, NM M-tiles of 128 rows, REP replicas of the query rows in an
 // M-tile (4: at most 32 rows, 2: at most 64, 1 otherwise), ST K/V stages, QB
@@ -256,35 +270,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const CUtensorMap* map = is_k ? &tm_k : &tm_v;
     const CUtensorMap* map_dec = is_k ? &tm_kd : &tm_vd;
     if (a.mode == kGather && nt > 0) {
-      // ---- gathered rows: the whole warp copies, tiles released in order
-      if (lane == 0) prefetch_tmap(map_dec);
-      const __nv_bfloat16* pool =
-          reinterpret_cast<const __nv_bfloat16*>(is_k ? a.Kp : a.Vp);
-      int pend[ST] = {};  // gathered tiles whose copies may be in flight, oldest first
-      int n_pend = 0;
-      // the oldest pending tile: its copies have landed (all but the newest
-      // n_pend - 1 groups), then the fence that orders them before the MMAs
-      auto release_oldest = [&]() {
-        switch (n_pend - 1) {
-          case 0: cp_async_wait<0>(); break;
-          case 1: cp_async_wait<1>(); break;
-          case 2: cp_async_wait<2>(); break;
-          case 3: cp_async_wait<3>(); break;
-          case 4: cp_async_wait<4>(); break;
-          case 5: cp_async_wait<5>(); break;
-          default: cp_async_wait<0>(); break;
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[pend[0] % ST]);
-        for (int q = 1; q < n_pend; ++q) pend[q - 1] = pend[q];
-        --n_pend;
-      };
+      // ---- gathered rows: TMA row gathers issued by the whole warp
+      if (lane == 0) {
+        prefetch_tmap(map);
+        prefetch_tmap(map_dec);
+      }
+      const int oob_row = s.n_slots * s.H_kv * 64;  // past the pool: zero fill
       auto load_q = [&](int k) -> bool {
         const int qb = QB == 2 ? (k & 1) : 0;
         bool w = true;
         if (k >= QB) {  // the buffer's previous segment must be done with it
-          while (n_pend > 0) release_oldest();
           const int prev = k - QB;
           if (lane == 0)
             w = mbar_wait(&q_free[qb], (QB == 2 ? (prev >> 1) : prev) & 1, abort_flag);
@@ -314,9 +309,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         if (!ok) break;
         const int st = i % ST;
-        // tile i - ST (same ring slot; decode tiles hold slots too) must be
-        // released before waiting for its slot
-        while (n_pend > 0 && pend[0] <= i - ST) release_oldest();
         if (i >= ST) {
           bool w = true;
           if (lane == 0) w = mbar_wait(&empty[st], ((i / ST) - 1) & 1, abort_flag);
@@ -328,34 +320,39 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const int bg = seg[k].x;
           const int b = bg / s.H_kv, g = bg % s.H_kv;
           const int tile = seg_lo[k] + (i - seg[k].z);  // tile of the (b, g)'s list
+          // lane owns rows lane and lane + 32 (their pool rows resolved here)
+          int own[2] = {oob_row, oob_row};
 #pragma unroll
           for (int rr = 0; rr < 2; ++rr) {
             const int r = lane + 32 * rr;
-            const __nv_bfloat16* src = pool;
-            bool okr = false;
             if (rows_staged) {
               const int row = s_rows[i * 64 + r];
-              okr = row >= 0;
-              if (okr) src = pool + (size_t)row * D;
+              if (row >= 0) own[rr] = row;
             } else if (r < valid) {
               const int pos = a.idx[(size_t)bg * a.max_idx + tile * 64 + r];
               const int slot = pos >= 0 && pos < s.L_ctx
                                    ? a.page_table[(size_t)b * s.n_pages + pos / 64] : -1;
-              if (slot >= 0 && slot < s.n_slots) {
-                src = pool + (((size_t)slot * s.H_kv + g) * 64 + pos % 64) * D;
-                okr = true;
-              } else {
+              if (slot >= 0 && slot < s.n_slots)
+                own[rr] = (slot * s.H_kv + g) * 64 + pos % 64;
+              else
                 flag_error(a.err, ERR_BAD_INDEX);  // the key is left zero
-              }
             }
-#pragma unroll
-            for (int c = 0; c < C::HALVES * 8; ++c)
-              cp_async16(dst + (c >> 3) * 8192 + r * 128 + (((c & 7) ^ (r & 7)) << 4),
-                         src + c * 8, okr);
           }
-          cp_async_commit();
-          pend[n_pend++] = i;
-          if (n_pend >= ST) release_oldest();
+          if (lane == 0) mbar_arrive_expect_tx(&full[st], C::KT_BYTES);
+          __syncwarp();
+          // lane: rows 4 q4 .. 4 q4 + 3 of column half h
+          const int q4 = (lane & 15) * 4, h = lane >> 4;
+          int y[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int r = q4 + j;
+            const int lo = __shfl_sync(0xffffffffu, own[0], r & 31);
+            const int hi = __shfl_sync(0xffffffffu, own[1], r & 31);
+            y[j] = r < 32 ? lo : hi;
+          }
+          if (h < C::HALVES)
+            tma_gather4_2d(dst + h * 8192 + q4 * 128, map, h * 64, y[0], y[1], y[2], y[3],
+                           &full[st]);
         } else if (valid > 0) {
           if (lane == 0) {
             mbar_arrive_expect_tx(&full[st], C::KT_BYTES);
@@ -366,8 +363,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           mbar_arrive(&full[st]);
         }
       }
-      while (n_pend > 0) release_oldest();  // every copy has landed before leaving
-      if (*abort_flag && lane == 0) {  // nor with a decode tile's TMA in flight
+      if (*abort_flag && lane == 0) {  // do not leave with loads in flight
         for (int i = max(0, nt - ST); i < nt; ++i)
           for (uint32_t t = 0; t < (1u << 20) && !mbar_try_wait(&full[i % ST], (i / ST) & 1); ++t) {
           }
@@ -787,8 +783,10 @@ static cudaError_t run_tc(const AttnArgs& a, int max_tiles, cudaStream_t st) {
   const uint64_t pool_rows = (uint64_t)s.n_slots * s.H_kv * 64;
   const uint64_t q_rows = (uint64_t)s.batch * s.H * s.L_q;
   const uint64_t n_bg = (uint64_t)s.batch * s.H_kv;
-  if (!tc_map_2d(&mq, a.Q, D, q_rows, C::RB) || !tc_map_2d(&mk, a.Kp, D, pool_rows, 64) ||
-      !tc_map_2d(&mv, a.Vp, D, pool_rows, 64) || !tc_map_3d(&mkd, a.Kd, D, s.L_q, n_bg) ||
+  // gathered keys: one-row boxes for the row gathers; else 64-key pages
+  const uint32_t pool_box = a.mode == kGather ? 1 : 64;
+  if (!tc_map_2d(&mq, a.Q, D, q_rows, C::RB) || !tc_map_2d(&mk, a.Kp, D, pool_rows, pool_box) ||
+      !tc_map_2d(&mv, a.Vp, D, pool_rows, pool_box) || !tc_map_3d(&mkd, a.Kd, D, s.L_q, n_bg) ||
       !tc_map_3d(&mvd, a.Vd, D, s.L_q, n_bg))
     return cudaErrorInvalidValue;
   const TcLaunch L = tc_plan((int)n_bg, max_tiles, tc_sm_count());

@@ -44,7 +44,7 @@ block_select_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
 // key digits and the shape fits it; else fused on the fp64 MMA when the
 // group's query rows (G x the bound max_q on q_cnt, or x L_q) fit four MMA
 // row tiles and the keys one thread each; else, for more rows over at most
-// 128 units, the CUDA-core kernel of block_select_wide.cu; otherwise block
+// 128 units, the kernel of block_select_wide.cu; otherwise block
 // scores then selection, as separate kernels.
 cudaError_t launch_block_select(const Shape& s, const void* Q, const int32_t* q_idx,
                                 const int32_t* q_cnt, const float* Kbar, const int8_t* Kdig,

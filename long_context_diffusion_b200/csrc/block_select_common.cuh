@@ -55,7 +55,11 @@ struct BsSorted {
 
 // Marks the sink units and sorts (as select_shfl_kernel): thread i holds
 // unit i's score on entry (units past n_units are ignored).  Every thread of
-// the CTA (kThreads) calls it.
+// the CTA (kThreads) calls it.  NW: the network's width, a power of two
+// >= n_units and >= 32; each NW-aligned group of threads is sorted on its
+// own, so threads 0 .. NW-1 hold the result (a narrow network skips the
+// shared-memory stages a 512-wide one needs).
+template <int NW = bs::kThreads>
 __device__ __forceinline__ BsSorted bs_sort(double my_score, int n_units, int b, int unit_size,
                                             const int32_t* __restrict__ sink_pos, int n_sinks,
                                             BsSelScratch& sc, unsigned* err) {
@@ -78,7 +82,8 @@ __device__ __forceinline__ BsSorted bs_sort(double my_score, int n_units, int b,
   r.n_sb = __syncthreads_count(is_sink);
   uint64_t key = (i < n_units && !is_sink) ? desc_key(my_score) : ~0ull;
   int idx = i;
-  for (int k = 2; k <= kThreads; k <<= 1) {
+  static_assert(NW >= 32 && NW <= kThreads && (NW & (NW - 1)) == 0, "network width");
+  for (int k = 2; k <= NW; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
       uint64_t pk;
       int px;

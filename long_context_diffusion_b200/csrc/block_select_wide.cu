@@ -9,16 +9,19 @@
 //   to the lower index), ascending.
 //
 // With at most 128 units and R * n_units <= 8192 every logit of the (b, g)
-// fits in shared memory, so one CTA does it all in fp64 on the CUDA cores:
+// fits in shared memory, so one CTA does it all in fp64:
 //   stage   the group's query rows (gathered by q_idx) and its pooled keys by
-//           cp.async;
-//   dot     warp = (4 rows, 32 units), lane = unit: per 4 dimensions one
-//           float4 of the key and one load of each row (the same address for
-//           the whole warp); 16 fp64 FMA chains per lane (row x dimension mod
-//           4), added in a fixed order (so equal keys give equal logits);
+//           cp.async, rows padded so that the fragment loads below hit 32
+//           distinct banks;
+//   dot     fp64 mma.sync m8n8k4 (the CUDA-core fp64 rate is a fraction of
+//           the fp64 MMA rate on this part): warp item = 8 rows x 16 units,
+//           four accumulators (two 8-unit tiles x even / odd 16-dimension
+//           groups), added in a fixed order, so equal keys give equal
+//           logits;
 //   softmax warp per row: max, e^(l - max) in fp64, sum, divide;
 //   scores  thread per unit sums its column in row order;
-//   select  the bitonic sort and ascending write of the fused kernels.
+//   select  the bitonic sort and ascending write of the fused kernels, on a
+//           network as wide as the units (32, 64 or 128).
 // fp32 query values and fp32 pooled keys are exact in fp64 and their
 // products too, so the logits carry only the rounding of the sums.
 #include "block_select_common.cuh"
@@ -35,15 +38,20 @@ constexpr int kMaxCells = 8192;  // rows x units held as fp64 logits
 
 template <typename T, int D>
 struct Layout {
-  static constexpr int KP = D + 4;  // pooled-key pitch in floats: rows 16 bytes apart mod 128
-  __host__ __device__ static int rows_cap(int R) { return (R + 3) & ~3; }
+  // pitches: bf16 query rows D + 16 elements (288 B at D 128: 8 banks
+  // apart, conflict-free 8-byte loads), fp32 rows D + 4 (2-way conflicts,
+  // but 256 rows still fit), pooled keys D + 16 floats (16 banks apart)
+  static constexpr int QP = D + (sizeof(T) == 2 ? 16 : 4);
+  static constexpr int KP = D + 16;
+  __host__ __device__ static int rows_cap(int R) { return (R + 7) & ~7; }
   __host__ __device__ static int units_cap(int U) { return (U + 31) & ~31; }
-  __host__ __device__ static size_t q_bytes(int R) { return (size_t)rows_cap(R) * D * sizeof(T); }
+  __host__ __device__ static size_t q_bytes(int R) { return (size_t)rows_cap(R) * QP * sizeof(T); }
   __host__ __device__ static size_t k_bytes(int U) { return (size_t)units_cap(U) * KP * 4; }
   __host__ __device__ static size_t bytes(int R, int U) {
     return q_bytes(R) + k_bytes(U) + (size_t)rows_cap(R) * units_cap(U) * 8;
   }
 };
+constexpr size_t kSmemLimit = 232448 - sizeof(BsSelScratch);
 }  // namespace bsw
 
 template <typename T>
@@ -88,11 +96,12 @@ block_select_wide_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_
     nq = max_rows / s.G;
   }
   const int R = nq * s.G;
-  T* sQ = reinterpret_cast<T*>(smem_b);                                   // [Rc][D]
+  T* sQ = reinterpret_cast<T*>(smem_b);                                   // [Rc][QP]
   float* sK = reinterpret_cast<float*>(smem_b + L::q_bytes(max_rows));    // [Uc][KP]
   double* sL = reinterpret_cast<double*>(smem_b + L::q_bytes(max_rows) + L::k_bytes(U));  // [Rc][Uc]
 
   constexpr int QCH = D * (int)sizeof(T) / 16;  // 16-byte chunks per query row
+  constexpr int QE = 16 / (int)sizeof(T);       // elements per chunk
   for (int c = tid; c < L::rows_cap(R) * QCH; c += kThreads) {
     const int r = c / QCH, ch = c % QCH;
     const T* src = Q;
@@ -101,13 +110,13 @@ block_select_wide_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_
       const int h = g * s.G + r / nq;
       const int i = q_idx ? q_idx[(size_t)b * s.L_q + (r % nq)] : (r % nq);
       if (i >= 0 && i < s.L_q) {
-        src = Q + (((size_t)b * s.H + h) * s.L_q + i) * D + ch * (16 / sizeof(T));
+        src = Q + (((size_t)b * s.H + h) * s.L_q + i) * D + ch * QE;
         ok = true;
       } else if (ch == 0) {
         flag_error(err, ERR_BAD_INDEX);
       }
     }
-    cp_async16(sQ + (size_t)r * D + ch * (16 / sizeof(T)), src, ok);
+    cp_async16(sQ + (size_t)r * L::QP + ch * QE, src, ok);
   }
   constexpr int KCH = D / 4;  // 16-byte chunks per pooled key
   const float* kb = Kbar + (size_t)bg * U * D;
@@ -120,35 +129,45 @@ block_select_wide_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_
   cp_async_wait<0>();
   __syncthreads();
 
-  // ---- logits: work item = (4 rows, 32 units); lane = unit
+  // ---- logits on the fp64 MMA: item = (8-row tile, two 8-unit tiles).  In
+  // m8n8k4 lane (gi, t) gives A[gi][t] and B[t][gi] and holds C[gi][2t, 2t+1];
+  // k-step i of 16-dimension group kg takes dimension 16 kg + 4 t + i, so a
+  // lane reads four consecutive dimensions of its row and of its unit.
   const double sc = s.scale;
-  const int n_rg = (R + 3) >> 2, n_ug = Uc >> 5;
-  for (int it = warp; it < n_rg * n_ug; it += kWarps) {
-    const int r0 = (it / n_ug) * 4, u = (it % n_ug) * 32 + lane;
-    const float* kr = sK + u * L::KP;
-    // 16 independent chains: row i, dimension phase c (k = c mod 4), so the
-    // FMA latency is hidden; the phases are added in a fixed order
-    double acc[4][4];
+  const int gi = lane >> 2, t4 = lane & 3;
+  const int n_mt = L::rows_cap(R) >> 3, n_np = Uc >> 4;
+  for (int it = warp; it < n_mt * n_np; it += kWarps) {
+    const int r0 = (it / n_np) * 8, u0 = (it % n_np) * 16;
+    const T* qr = sQ + (size_t)(r0 + gi) * L::QP + 4 * t4;
+    const float* k0 = sK + (u0 + gi) * L::KP + 4 * t4;
+    const float* k1 = k0 + 8 * L::KP;
+    double acc[2][2][2];  // [unit tile][kg parity][C element]
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int a = 0; a < 2; ++a)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[i][c] = 0.0;
+      for (int p = 0; p < 2; ++p) acc[a][p][0] = acc[a][p][1] = 0.0;
 #pragma unroll 4
-    for (int k = 0; k < D; k += 4) {
-      const float4 kv = *reinterpret_cast<const float4*>(kr + k);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        double q[4];
-        load4<T>(sQ + (size_t)(r0 + i) * D + k, q);
-        acc[i][0] = fma(q[0], (double)kv.x, acc[i][0]);
-        acc[i][1] = fma(q[1], (double)kv.y, acc[i][1]);
-        acc[i][2] = fma(q[2], (double)kv.z, acc[i][2]);
-        acc[i][3] = fma(q[3], (double)kv.w, acc[i][3]);
-      }
+    for (int kg = 0; kg < D / 16; ++kg) {
+      double q[4];
+      load4<T>(qr + 16 * kg, q);
+      const float4 b0 = *reinterpret_cast<const float4*>(k0 + 16 * kg);
+      const float4 b1 = *reinterpret_cast<const float4*>(k1 + 16 * kg);
+      const int p = kg & 1;
+      dmma_m8n8k4(acc[0][p], q[0], (double)b0.x);
+      dmma_m8n8k4(acc[1][p], q[0], (double)b1.x);
+      dmma_m8n8k4(acc[0][p], q[1], (double)b0.y);
+      dmma_m8n8k4(acc[1][p], q[1], (double)b1.y);
+      dmma_m8n8k4(acc[0][p], q[2], (double)b0.z);
+      dmma_m8n8k4(acc[1][p], q[2], (double)b1.z);
+      dmma_m8n8k4(acc[0][p], q[3], (double)b0.w);
+      dmma_m8n8k4(acc[1][p], q[3], (double)b1.w);
     }
+    double* lr = sL + (size_t)(r0 + gi) * Uc + u0 + 2 * t4;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      sL[(size_t)(r0 + i) * Uc + u] = ((acc[i][0] + acc[i][1]) + (acc[i][2] + acc[i][3])) * sc;
+    for (int a = 0; a < 2; ++a) {
+      lr[8 * a] = (acc[a][0][0] + acc[a][1][0]) * sc;
+      lr[8 * a + 1] = (acc[a][0][1] + acc[a][1][1]) * sc;
+    }
   }
   __syncthreads();
 
@@ -178,16 +197,25 @@ block_select_wide_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_
     for (int r = 0; r < R; ++r) my += sL[(size_t)r * Uc + tid];
     score[(size_t)bg * U + tid] = my;
   }
-  const BsSorted srt = bs_sort(my, U, b, unit_size, sink_pos, n_sinks, s_sel, err);
+  const BsSorted srt =
+      U <= 32   ? bs_sort<32>(my, U, b, unit_size, sink_pos, n_sinks, s_sel, err)
+      : U <= 64 ? bs_sort<64>(my, U, b, unit_size, sink_pos, n_sinks, s_sel, err)
+                : bs_sort<128>(my, U, b, unit_size, sink_pos, n_sinks, s_sel, err);
   bs_write(srt, U, topK, bg, blk_idx, blk_cnt, max_sel, s_sel);
 }
 
 bool block_select_wide_supported(const Shape& s, int rows, int n_units) {
-  if (n_units < 1 || n_units > bsw::kMaxUnits || rows > bsw::kMaxRows) return false;
+  if (n_units < 1 || n_units > bsw::kMaxUnits || rows < 1 || rows > bsw::kMaxRows) return false;
   if ((size_t)bsw::Layout<float, 128>::rows_cap(rows) * bsw::Layout<float, 128>::units_cap(n_units) >
       (size_t)bsw::kMaxCells)
     return false;
-  return s.d == 64 || s.d == 128;
+  if (s.d != 64 && s.d != 128) return false;
+  const size_t bytes =
+      s.dtype == 0 ? (s.d == 128 ? bsw::Layout<__nv_bfloat16, 128>::bytes(rows, n_units)
+                                 : bsw::Layout<__nv_bfloat16, 64>::bytes(rows, n_units))
+                   : (s.d == 128 ? bsw::Layout<float, 128>::bytes(rows, n_units)
+                                 : bsw::Layout<float, 64>::bytes(rows, n_units));
+  return bytes <= bsw::kSmemLimit;
 }
 
 cudaError_t launch_block_select_wide(const Shape& s, const void* Q, const int32_t* q_idx,

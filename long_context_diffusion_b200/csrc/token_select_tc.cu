@@ -13,19 +13,22 @@
 // tiles of two 64-key pages; a content token at position 1024 (a chunk of
 // 1024 content tokens) is scored on the CUDA cores.  Keys are the MMA's M
 // side: S^T [128 keys x N rows] = K_tile . Q^T for each tile, all eight tiles
-// resident in TMEM at once (8 x N <= 512 columns).  Then, with thread =
-// TMEM lane = key of a tile (8 warps, four tiles each): pass 1 takes each
-// row's maximum; pass 2 the exponentials 2^(x - max) (written back over S^T)
-// and each row's sum; pass 3 each key's mass, the sum over rows of its
-// exponentials divided by the row sums.  The top-T cut is a radix select on
+// resident in TMEM at once (8 x N <= 512 columns).  With thread = TMEM lane =
+// key of a tile: pass 1 takes each row's maximum, tile by tile as the MMAs
+// finish (warps 4-7, one per lane quadrant, while the rest still streams),
+// then reduces it; then with 8 warps, four tiles each, pass 2 the
+// exponentials 2^(x - max) (written back over S^T) and each row's sum, and
+// pass 3 each key's mass, the sum over rows of its exponentials divided by
+// the row sums.  The top-T cut is a radix select on
 // the masses' bit patterns (non-negative floats order as integers) with the
 // tied entries at the cut taken in position order; the kept tokens are
 // written in ascending position order.
 //
 // Roles while streaming: warp 0 one thread: TMA of the K tiles (a ring of
-// four); warp 1 one thread: the MMAs; warps 2-3: gather the query rows into
-// shared memory; warps 4-5: the score of the token past the tiles.  Every
-// wait is bounded.
+// four); warp 1 one thread: the MMAs (each tile committed to a barrier of its
+// own); warp 2 one thread: TMA of the group's query rows (contiguous rows of
+// Q: the G heads' L_q positions); warps 2-3: the score of the token past the
+// tiles; warps 4-7: pass 1.  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -59,8 +62,8 @@ struct Layout {
   static constexpr int SCAN_OFF = HIST_OFF + 256 * 4;       // int [40]
   static constexpr int PV_OFF = SCAN_OFF + 40 * 4;          // int [2 * MAX_TILES + 1] page valid
   static constexpr int BAR_OFF = (PV_OFF + (2 * MAX_TILES + 1) * 4 + 15) / 16 * 16;
-  // full, empty [STAGES]; q_full; s_done
-  static constexpr int N_BARS = 2 * STAGES + 2;
+  // full, empty [STAGES]; q_full; s_done; tile_done [MAX_TILES]
+  static constexpr int N_BARS = 2 * STAGES + 2 + MAX_TILES;
   static constexpr int MISC_OFF = BAR_OFF + N_BARS * 8;      // tmem slot, abort flag
   static constexpr int SMEM = MISC_OFF + 16 + 1024;          // + alignment slack
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -246,7 +249,8 @@ __device__ __noinline__ void token_recheck_fp64(
 
 template <int N>
 __global__ void __launch_bounds__(ts::THREADS, 1)
-token_select_tc_kernel(const __grid_constant__ CUtensorMap tm_k, Shape s,
+token_select_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_q, Shape s,
                        const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ Kp,
                        const int32_t* __restrict__ page_table,
                        const int32_t* __restrict__ chunk_idx, int n_sel, int stride, int content,
@@ -272,6 +276,7 @@ token_select_tc_kernel(const __grid_constant__ CUtensorMap tm_k, Shape s,
   uint64_t* empty = full + STAGES;
   uint64_t* q_full = empty + STAGES;
   uint64_t* s_done = q_full + 1;
+  uint64_t* tile_done = s_done + 1;  // [MAX_TILES]: the tile's S^T is in TMEM
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
 
@@ -301,8 +306,9 @@ token_select_tc_kernel(const __grid_constant__ CUtensorMap tm_k, Shape s,
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(q_full, 64);
+    mbar_init(q_full, 1);
     mbar_init(s_done, 1);
+    for (int i = 0; i < MAX_TILES; ++i) mbar_init(&tile_done[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -311,6 +317,11 @@ token_select_tc_kernel(const __grid_constant__ CUtensorMap tm_k, Shape s,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int quad = warp & 3;
+  const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+  float m[N];  // pass 1: this thread's maxima of each row (warps 4-7)
+#pragma unroll
+  for (int r = 0; r < N; ++r) m[r] = -INFINITY;
 
   if (n_t > 0 && warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -369,44 +380,24 @@ token_select_tc_kernel(const __grid_constant__ CUtensorMap tm_k, Shape s,
           mma_f16_ss(tmem + t * N, ad, bd, idesc, k > 0 ? 1u : 0u);
         }
         mma_commit(&empty[st]);
+        mma_commit(&tile_done[t]);
       }
       if (ok) mma_commit(s_done);
       if (*abort_flag)  // give issued MMAs time to finish before TMEM is freed
         for (uint32_t k = 0; k < (1u << 16); ++k) __nanosleep(1000);
     }
-  } else if (n_t > 0 && (warp == 2 || warp == 3)) {
-    // ------------------------------------------------------------ Q gather
-    constexpr int per_row = 16;  // 16-byte chunks of a 128-element row
-    constexpr int IN_FLIGHT = 8;
-    const int gt = threadIdx.x - 64;
-    constexpr int total = N * per_row;
-    for (int e0 = 0; e0 < total; e0 += 64 * IN_FLIGHT) {
-      uint4 v[IN_FLIGHT];
-#pragma unroll
-      for (int u = 0; u < IN_FLIGHT; ++u) {
-        const int e = e0 + u * 64 + gt;
-        const int n = e / per_row, rem = e % per_row;
-        v[u] = make_uint4(0u, 0u, 0u, 0u);
-        if (e < total && n < R) {
-          const int h = g * s.G + n / s.L_q, i = n % s.L_q;
-          v[u] = __ldg(reinterpret_cast<const uint4*>(Q + (((size_t)b * s.H + h) * s.L_q + i) * D +
-                                                      rem * 8));
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < IN_FLIGHT; ++u) {
-        const int e = e0 + u * 64 + gt;
-        if (e >= total) continue;
-        const int n = e / per_row, rem = e % per_row;
-        const int h_half = rem >> 3, ch = rem & 7;
-        *reinterpret_cast<uint4*>(sQ + h_half * N * 128 + n * 128 + ((ch ^ (n & 7)) << 4)) = v[u];
-      }
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ Q, last token
+    if (n_t > 0 && threadIdx.x == 64) {
+      // the R rows of the group are rows (b H + g G) L_q .. + R - 1 of Q;
+      // rows past R (another group's or the zero fill past the end) only
+      // fill S^T columns that every pass masks
+      prefetch_tmap(&tm_q);
+      const int row0 = (b * s.H + g * s.G) * s.L_q;
+      mbar_arrive_expect_tx(q_full, 2 * N * 128);
+      for (int h = 0; h < 2; ++h) tma_load_2d(sQ + h * N * 128, &tm_q, h * 64, row0, q_full);
     }
-    fence_proxy_async_smem();
-    mbar_arrive(q_full);
-  } else if (warp == 4 || warp == 5) {
-    // ------------------------------------------------------------ last token
-    const int r = threadIdx.x - 128;
+    const int r = threadIdx.x - 64;
     float x = -INFINITY;
     if (has_left) {
       const long long pos = base + MAXC;
@@ -432,6 +423,29 @@ token_select_tc_kernel(const __grid_constant__ CUtensorMap tm_k, Shape s,
       }
     }
     if (r < N) s_xl[r] = x;
+  } else if (n_t > 0 && warp >= 4) {
+    // ------------------------------------------------------------ pass 1
+    // page validity of this lane's keys, decided as the producer decides it
+    bool pok = false;
+    if (lane < 2 * MAX_TILES && lane * 64 <= last_o) {
+      const int slot = page_table[(size_t)b * s.n_pages + page0 + lane];
+      pok = slot >= 0 && slot < s.n_slots;
+    }
+    const uint32_t pv = __ballot_sync(0xffffffffu, pok);
+    for (int t = 0; t < n_t; ++t) {
+      bool w = true;
+      if (lane == 0) w = mbar_wait(&tile_done[t], 0, abort_flag);
+      if (!__shfl_sync(0xffffffffu, w, 0)) break;
+      tc_fence_after();
+      const int o = t * 128 + quad * 32 + lane;
+      const bool kv = o >= 1 && o <= last_o && ((pv >> (o >> 6)) & 1u);
+      uint32_t v[N];
+      tmem_ld<N>(tmem + lane_base + t * N, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int r = 0; r < N; ++r)
+        m[r] = fmaxf(m[r], (kv && r < R) ? __uint_as_float(v[r]) * c2 : -INFINITY);
+    }
   }
   // ---------------------------------------------------------------- epilogue
   // every warp: TMEM lanes of its quadrant, four of the tiles
@@ -442,34 +456,19 @@ token_select_tc_kernel(const __grid_constant__ CUtensorMap tm_k, Shape s,
   __syncthreads();
   tc_fence_after();
   const bool run = n_t > 0 && !*abort_flag;
-  const int quad = warp & 3;
-  const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
   auto key_ok = [&](int o) {  // offset o from the chunk start holds a usable content token
     return o >= 1 && o <= last_o && s_pv[o >> 6] != 0;
   };
-  if (run) {
-    // pass 1: row maxima
-    float m[N];
+  if (run && warp >= 4) {  // pass 1, the reduction over the lanes of each warp
 #pragma unroll
-    for (int r = 0; r < N; ++r) m[r] = -INFINITY;
-    for (int j = warp >> 2; j < n_t; j += 2) {
-      const int o = j * 128 + quad * 32 + lane;
-      const bool kv = key_ok(o);
-      uint32_t v[N];
-      tmem_ld<N>(tmem + lane_base + j * N, v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int r = 0; r < N; ++r)
-        m[r] = fmaxf(m[r], (kv && r < R) ? __uint_as_float(v[r]) * c2 : -INFINITY);
-    }
-#pragma unroll
-    for (int r0 = 0; r0 < N; r0 += 32) s_red[warp * N + r0 + lane] = xreduce32<true>(m + r0, lane);
+    for (int r0 = 0; r0 < N; r0 += 32)
+      s_red[(warp - 4) * N + r0 + lane] = xreduce32<true>(m + r0, lane);
   }
   __syncthreads();
   if (run && threadIdx.x < N) {
     const int r = threadIdx.x;
     float mx = s_xl[r];
-    for (int w = 0; w < 8; ++w) mx = fmaxf(mx, s_red[w * N + r]);
+    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, s_red[w * N + r]);
     s_M[r] = mx;
   }
   __syncthreads();
@@ -694,6 +693,9 @@ cudaError_t launch_token_select_tc(const Shape& s, const void* Q, const void* Kp
   CUtensorMap mk;
   const int n_chunks = (s.L_ctx + chunk_stride - 1) / chunk_stride;
   if (!tc_map_2d(&mk, Kp, ts::D, (uint64_t)s.n_slots * s.H_kv * 64, 64)) return cudaErrorInvalidValue;
+  const int n_rows = s.G * s.L_q <= 32 ? 32 : 64;  // N: S^T columns, the Q box's rows
+  CUtensorMap mq;
+  if (!tc_map_2d(&mq, Q, ts::D, (uint64_t)s.batch * s.H * s.L_q, n_rows)) return cudaErrorInvalidValue;
   dim3 grid(n_sel, s.batch * s.H_kv);
   auto* q = reinterpret_cast<const __nv_bfloat16*>(Q);
   auto* k = reinterpret_cast<const __nv_bfloat16*>(Kp);
@@ -703,7 +705,7 @@ cudaError_t launch_token_select_tc(const Shape& s, const void* Q, const void* Kp
     if ((e = cudaFuncSetAttribute(token_select_tc_kernel<32>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
       return e;
-    DL_LAUNCH(token_select_tc_kernel<32>, grid, ts::THREADS, smem, st, mk, s, q, k, page_table,
+    DL_LAUNCH(token_select_tc_kernel<32>, grid, ts::THREADS, smem, st, mk, mq, s, q, k, page_table,
               chunk_idx, n_sel, chunk_stride, chunk_content, topT, Kexp, n_chunks, tok_pos,
               tok_cnt, err);
   } else {
@@ -711,7 +713,7 @@ cudaError_t launch_token_select_tc(const Shape& s, const void* Q, const void* Kp
     if ((e = cudaFuncSetAttribute(token_select_tc_kernel<64>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
       return e;
-    DL_LAUNCH(token_select_tc_kernel<64>, grid, ts::THREADS, smem, st, mk, s, q, k, page_table,
+    DL_LAUNCH(token_select_tc_kernel<64>, grid, ts::THREADS, smem, st, mk, mq, s, q, k, page_table,
               chunk_idx, n_sel, chunk_stride, chunk_content, topT, Kexp, n_chunks, tok_pos,
               tok_cnt, err);
   }
