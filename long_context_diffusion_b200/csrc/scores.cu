@@ -9,16 +9,17 @@
 // the spacing of neighbouring scores, so the kept set equals the one an
 // exact computation gives.
 //
-// Two kernels.  (1) tile: grid (128-unit tiles, b*H_kv).  Each warp owns
-// 16 pooled keys and multiplies them with every query row on the fp64
-// tensor-core MMA (m8n8k4; products of bf16 or fp32 inputs are exact in
-// fp64).  The CTA then takes, per row, the max over its 128 units, writes
-// e = exp(l - m_tile) and records (m_tile, z_tile = sum e).  (2) reduce: one
-// CTA per (b, g) merges the tile statistics of each row into the factors
-// f = exp(m_tile - M) / Z, the row's softmax being e * f, and sums the
-// columns over the rows in row order.  This is the two-pass softmax of the
-// definition with its max and sum taken tile by tile (online-softmax
-// merging), equal to it up to fp64 rounding.
+// Two kernels.  (1) tile: grid (128-unit tiles, 32-row blocks, b*H_kv).
+// Each warp owns 16 pooled keys and multiplies them with the block's query
+// rows on the fp64 tensor-core MMA (m8n8k4; products of bf16 or fp32 inputs
+// are exact in fp64).  The CTA then takes, per row, the max over its 128
+// units, writes e = exp(l - m_tile) and records (m_tile, z_tile = sum e).
+// (2) reduce: grid (128-unit tiles, b*H_kv).  Per row the tile statistics
+// give M and Z and the tile's factor f = exp(m_tile - M) / Z, the row's
+// softmax being e * f; four row groups then sum each column (rows g, g + 4,
+// ... in order) and the four partial sums are added in group order.  This is
+// the two-pass softmax of the definition with its max and sum taken tile by
+// tile (online-softmax merging), equal to it up to fp64 rounding.
 #include "common.cuh"
 #include "internal.h"
 #include "launch.cuh"
@@ -76,7 +77,7 @@ scores_tile_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
   T* sRaw = reinterpret_cast<T*>(smem_s + L::RAW_OFF);            // [kRT][D]
   __shared__ double s_red[kWarps][kRT];
   __shared__ double s_row[kRT];
-  const int bg = blockIdx.y;
+  const int bg = blockIdx.z;
   const int b = bg / s.H_kv, g = bg % s.H_kv;
   const int tile = blockIdx.x, n_tiles = gridDim.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -97,13 +98,12 @@ scores_tile_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
   const int nq = q_idx ? min(max(q_cnt[b], 0), s.L_q) : s.L_q;
   const int R = nq * s.G;
   const int R_max = s.L_q * s.G;
-  if (R == 0) {
+  const int r0 = blockIdx.y * kRT;  // this CTA's rows r0 .. r0 + kRT - 1
+  if (r0 >= R) {
     asm volatile("cp.async.wait_all;" ::: "memory");
     return;
   }
-
-  for (int r0 = 0; r0 < R; r0 += kRT) {
-    __syncthreads();  // the previous pass is done with sQ and sRaw
+  {
     // query rows r0 .. r0+31 as copied (zeros past R or for a bad index)
     for (int c = threadIdx.x; c < kRT * CPR; c += blockDim.x) {
       const int rr = c / CPR, ch = c % CPR;
@@ -235,17 +235,23 @@ scores_tile_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
   }
 }
 
-// One CTA per (b, g).  Warp per row: M = max of the tile maxima,
-// Z = sum_t z_t exp(m_t - M); the tile factors f_t = exp(m_t - M) / Z
-// replace the statistics in place.  Then thread per unit: score[u] =
-// sum over rows, in row order, of e[r][u] * f[r][tile of u].
-__global__ void __launch_bounds__(512)
+// Grid (128-unit tiles, b*H_kv).  Warp per row: M = max of the tile
+// maxima, Z = sum_t z_t exp(m_t - M), and the factor of this CTA's tile
+// f = exp(m_tile - M) / Z (dynamic shared memory, G * L_q doubles; the
+// statistics are only read).
+// Then thread = (row group rg, unit): the sum over the rows rg, rg + 4, ...
+// in order of e[r][u] * f[r], and the four groups' sums added in order.
+constexpr int kRedGroups = 4;
+
+__global__ void __launch_bounds__(kRedGroups * kUT)
 scores_reduce_kernel(const int32_t* __restrict__ q_idx, const int32_t* __restrict__ q_cnt,
                      Shape s, int n_units, const double* __restrict__ E,
-                     double2* __restrict__ stats, double* __restrict__ score) {
+                     const double2* __restrict__ stats, double* __restrict__ score) {
   pdl_trigger();
   pdl_wait();
-  const int bg = blockIdx.x;
+  extern __shared__ double s_f[];  // [G * L_q]
+  __shared__ double s_part[kRedGroups][kUT];
+  const int tile = blockIdx.x, bg = blockIdx.y;
   const int b = bg / s.H_kv;
   const int nq = q_idx ? min(max(q_cnt[b], 0), s.L_q) : s.L_q;
   const int R = nq * s.G;
@@ -253,36 +259,38 @@ scores_reduce_kernel(const int32_t* __restrict__ q_idx, const int32_t* __restric
   const int n_tiles = score_tiles(n_units);
   const size_t pitch = (size_t)n_tiles * kUT;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  double2* st = stats + (size_t)bg * R_max * n_tiles;
+  const double2* st = stats + (size_t)bg * R_max * n_tiles;
   for (int r = warp; r < R; r += nw) {
-    double2* row = st + (size_t)r * n_tiles;
+    const double2* row = st + (size_t)r * n_tiles;
     double M = -INFINITY;
     for (int t = lane; t < n_tiles; t += 32) M = fmax(M, row[t].x);
     M = warp_max_d(M);
     double Z = 0.0;
     for (int t = lane; t < n_tiles; t += 32) Z += row[t].y * exp(row[t].x - M);
     Z = warp_sum_d(Z);
-    __syncwarp();
-    for (int t = lane; t < n_tiles; t += 32) row[t].x = exp(row[t].x - M) / Z;
+    if (lane == 0) s_f[r] = exp(row[tile].x - M) / Z;
   }
   __syncthreads();
-  const double* Eb = E + (size_t)bg * R_max * pitch;
-  for (int u = threadIdx.x; u < n_units; u += blockDim.x) {
-    const int t = u / kUT;
-    double acc = 0.0;
-    int r = 0;
-    for (; r + 8 <= R; r += 8) {  // 8 rows' loads in flight, then the sums in row order
-      double e[8], f[8];
+  const int rg = threadIdx.x / kUT, ul = threadIdx.x % kUT;
+  const int u = tile * kUT + ul;
+  const double* Eb = E + (size_t)bg * R_max * pitch + u;
+  double acc = 0.0;
+  int r = rg;
+  for (; r + 8 * kRedGroups <= R; r += 8 * kRedGroups) {  // 8 loads in flight, sums in order
+    double e[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        e[q] = Eb[(size_t)(r + q) * pitch + u];
-        f[q] = st[(size_t)(r + q) * n_tiles + t].x;
-      }
+    for (int q = 0; q < 8; ++q) e[q] = Eb[(size_t)(r + q * kRedGroups) * pitch];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc += e[q] * f[q];
-    }
-    for (; r < R; ++r) acc += Eb[(size_t)r * pitch + u] * st[(size_t)r * n_tiles + t].x;
-    score[(size_t)bg * n_units + u] = acc;
+    for (int q = 0; q < 8; ++q) acc += e[q] * s_f[r + q * kRedGroups];
+  }
+  for (; r < R; r += kRedGroups) acc += Eb[(size_t)r * pitch] * s_f[r];
+  s_part[rg][ul] = acc;
+  __syncthreads();
+  if (rg == 0 && u < n_units) {
+    double sc = s_part[0][ul];
+#pragma unroll
+    for (int q = 1; q < kRedGroups; ++q) sc += s_part[q][ul];
+    score[(size_t)bg * n_units + u] = sc;
   }
 }
 
@@ -303,7 +311,7 @@ cudaError_t launch_scores(const Shape& s, const void* Q, const int32_t* q_idx,
   double* E = reinterpret_cast<double*>(ws);
   double2* stats =
       reinterpret_cast<double2*>(reinterpret_cast<char*>(ws) + scores_e_bytes(s, n_units));
-  dim3 grid(score_tiles(n_units), s.batch * s.H_kv);
+  dim3 grid(score_tiles(n_units), (s.G * s.L_q + kRT - 1) / kRT, s.batch * s.H_kv);
   const dim3 block(kWarps * 32);
   cudaError_t e;
 #define DL_TILE(T, D_)                                                                        \
@@ -323,8 +331,13 @@ cudaError_t launch_scores(const Shape& s, const void* Q, const int32_t* q_idx,
   }
 #undef DL_TILE
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  DL_LAUNCH(scores_reduce_kernel, s.batch * s.H_kv, 512, 0, st, q_idx, q_cnt, s, n_units, E, stats,
-                                                         score);
+  const size_t red_smem = (size_t)s.G * s.L_q * sizeof(double);
+  if (red_smem > 48 * 1024 &&
+      (e = cudaFuncSetAttribute(scores_reduce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)red_smem)) != cudaSuccess)
+    return e;
+  DL_LAUNCH(scores_reduce_kernel, dim3(score_tiles(n_units), s.batch * s.H_kv), kRedGroups * kUT,
+            red_smem, st, q_idx, q_cnt, s, n_units, E, stats, score);
   return cudaGetLastError();
 }
 
