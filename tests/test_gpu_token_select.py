@@ -193,3 +193,71 @@ def test_token_select_near_tie_at_the_cut(exact_tie, cuda_device):
         assert (0.0 < gap < 1e-3) if not exact_tie else gap == 0.0
         mine = got[0, g, 1:] - base - 1
         assert mine.tolist() == off.tolist(), g
+
+
+@pytest.mark.parametrize("certified", [False, True])
+def test_token_select_more_items_than_sms_with_bad_chunks(certified, cuda_device):
+    """192 (b, g, chunk) items: the persistent kernel gives some CTAs two of
+    them.  Three chunk indices are bad (-1 twice, one chunk past the context),
+    one of them a CTA's second item and one a CTA's first: those items are
+    written as -1 and reported (DL_ERR_BAD_INDEX); every other item equals
+    the oracle's selection."""
+    batch, H, H_kv, L_q, d, page = 2, 16, 16, 32, 128, 64
+    content, stride, n_chunks, topT, n_sel = 256, 320, 8, 40, 6
+    L_ctx = n_chunks * stride
+    n_pages = L_ctx // page
+    n_slots = batch * n_pages
+    sid = 12900
+    q = (synth.normals(SEED, sid, 0, batch * H * L_q * d).reshape(batch, H, L_q, d)).to(
+        torch.bfloat16)
+    kp = (synth.normals(SEED, sid + 1, 0, n_slots * H_kv * page * d).reshape(
+        n_slots, H_kv, page, d)).to(torch.bfloat16)
+    perm = torch.argsort(synth.uniforms(SEED, sid + 2, 0, n_slots)).to(torch.int32)
+    page_table = perm.reshape(batch, n_pages)
+    sel_keys = synth.uniforms(SEED, sid + 3, 0, batch * H_kv * n_chunks).reshape(
+        batch * H_kv, n_chunks)
+    chunk_idx = torch.sort(torch.argsort(sel_keys, dim=1)[:, :n_sel], dim=1).values.to(
+        torch.int32).reshape(batch, H_kv, n_sel)
+    # items are (b * H_kv + g) * n_sel + sel; with 148 CTAs, CTA c takes c and c + 148
+    bad = {(0, 3, 2): -1,          # item 20: CTA 20, first of two
+           (1, 9, 0): -1,          # item 150: CTA 2, second of two
+           (1, 7, 0): n_chunks}    # item 138: a chunk past the context
+    for (b, g, j), v in bad.items():
+        chunk_idx[b, g, j] = v
+    desc = dl.make_desc(batch=batch, H=H, H_kv=H_kv, d=d, L_ctx=L_ctx, L_q=L_q, page=page,
+                        n_pages=n_pages, n_slots=n_slots, dtype=dl.DL_BF16)
+    ws = torch.empty(max(dl.dl_workspace_size(desc), 256), dtype=torch.uint8, device=cuda_device)
+    per = topT + 1
+    tok_pos = torch.full((batch, H_kv, n_sel * per), -7, dtype=torch.int32, device=cuda_device)
+    tok_cnt = torch.full((batch, H_kv), -7, dtype=torch.int32, device=cuda_device)
+    Kexp = _chunk_exps(desc, kp, page_table, n_chunks, stride, content, cuda_device) \
+        if certified else None
+    dl.dl_token_select(desc, q.to(cuda_device), kp.to(cuda_device), page_table.to(cuda_device),
+                       chunk_idx.to(cuda_device), stride, content, topT, tok_pos, tok_cnt, ws,
+                       Kexp=Kexp)
+    torch.cuda.synchronize()
+    assert dl.dl_get_status() == dl.DL_ERR_BAD_INDEX
+    got = np_(tok_pos)
+    assert (np_(tok_cnt) == n_sel * per).all()
+    scale = oracle.scale_for(d)
+    Q, K = S.f64(q), S.f64(kp)
+    pt = np.asarray(page_table, dtype=np.int64)
+    for b in range(batch):
+        for g in range(H_kv):
+            rows = Q[b, g].reshape(-1, d)
+            for j in range(n_sel):
+                out = got[b, g, j * per:(j + 1) * per]
+                if (b, g, j) in bad:
+                    assert (out == -1).all(), (b, g, j)
+                    continue
+                c = int(chunk_idx[b, g, j])
+                base = c * stride
+                keys = S.gather_context(K, pt[b], g, base + 1 + np.arange(content), page)
+                off, tau = S.token_select(rows, keys, topT, scale)
+                assert out[0] == base, (b, g, j)
+                mine = out[1:1 + len(off)] - base - 1
+                tol = 1e-5 * tau.max()
+                if certified or cut_margin(tau, off) > tol:
+                    assert mine.tolist() == off.tolist(), (b, g, j)
+                else:
+                    assert (tau[mine] >= np.sort(tau)[-topT] - tol).all(), (b, g, j)
