@@ -10,6 +10,10 @@ about 2.1 GB of K/V pages on the device), runs the steps before the profiled
 call once, then calls it `reps` times (the first is a warm-up) and prints its
 mean time from CUDA events.  Meant to sit under `ncu -k ... -s 1 -c 1`.
 
+`workload --workload NAME` times one single-layer step of a small workload
+(tiny, llada8k or dream16k; as the bench's `workloads` sub-records: CUDA-graph
+replays with L2 flushed before each) and prints its median time.
+
 `chunk_step` instead times the chunked-prefix step (32 chunks of a BOS and
 1024 content tokens in permuted 64-token pages, 64 decode queries, top-8
 chunks, top-256 tokens per chunk): chunk scores, chunk selection, token
@@ -34,8 +38,9 @@ from long_context_diffusion_b200 import _abi as A  # noqa: E402
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["attn_sparse", "attn_dense", "block_select", "pool", "sinks", "chunk_step"],
-                    required=True)
+    ap.add_argument("--case", choices=["attn_sparse", "attn_dense", "block_select", "pool", "sinks",
+                                       "chunk_step", "workload"], required=True)
+    ap.add_argument("--workload", default="dream16k", help="for --case workload")
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--batch", type=int, default=4)
     ap.add_argument("--fp64-select", action="store_true",
@@ -44,6 +49,12 @@ def main():
     dev = torch.device("cuda", 0)
     if args.case == "chunk_step":
         return chunk_step(args.reps, dev)
+    if args.case == "workload":
+        import bench
+        rec = bench.workload_record(args.workload, dev, bench.peaks()[0], reps=args.reps)
+        print(json.dumps({k: rec[k] for k in ("workload", "us_per_step", "bytes",
+                                              "frac_of_measured")}))
+        return None
     wl = synth.workload("llada32k_step", n_layers=3, batch=args.batch)
     layer = wl.first_sparse_layer
     pt = synth.page_permutation(wl).to(dev)

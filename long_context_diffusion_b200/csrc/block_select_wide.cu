@@ -9,7 +9,8 @@
 //   to the lower index), ascending.
 //
 // With at most 128 units and R * n_units <= 8192 every logit of the (b, g)
-// fits in shared memory, so one CTA does it all in fp64:
+// fits in shared memory.  A cluster of four CTAs takes one (b, g), each CTA a
+// quarter of the rows (softmax rows are independent), in fp64:
 //   stage   the group's query rows (gathered by q_idx) and its pooled keys by
 //           cp.async, rows padded so that the fragment loads below hit 32
 //           distinct banks;
@@ -19,11 +20,15 @@
 //           groups), added in a fixed order, so equal keys give equal
 //           logits;
 //   softmax warp per row: max, e^(l - max) in fp64, sum, divide;
-//   scores  thread per unit sums its column in row order;
-//   select  the bitonic sort and ascending write of the fused kernels, on a
-//           network as wide as the units (32, 64 or 128).
+//   scores  thread per unit sums its column over the CTA's rows in row
+//           order; the first CTA of the cluster adds the four CTAs' sums in
+//           CTA order (reading the others' shared memory);
+//   select  that CTA: the bitonic sort and ascending write of the fused
+//           kernels, on a network as wide as the units (32, 64 or 128).
 // fp32 query values and fp32 pooled keys are exact in fp64 and their
 // products too, so the logits carry only the rounding of the sums.
+#include <cooperative_groups.h>
+
 #include "block_select_common.cuh"
 #include "launch.cuh"
 
@@ -35,6 +40,9 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kMaxUnits = 128;
 constexpr int kMaxRows = 256;
 constexpr int kMaxCells = 8192;  // rows x units held as fp64 logits
+constexpr int kCluster = 4;      // CTAs per (b, g), a quarter of the rows each
+// rows of one CTA of the cluster: a multiple of the MMA's 8
+__host__ __device__ inline int cta_rows(int R) { return ((R + kCluster - 1) / kCluster + 7) & ~7; }
 
 template <typename T, int D>
 struct Layout {
@@ -70,7 +78,7 @@ __device__ __forceinline__ void load4<float>(const float* p, double (&v)[4]) {
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(bsw::kThreads, 1)
+__global__ void __cluster_dims__(bsw::kCluster, 1, 1) __launch_bounds__(bsw::kThreads, 1)
 block_select_wide_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
                          const int32_t* __restrict__ q_cnt, const float* __restrict__ Kbar,
                          Shape s, int n_units, int max_rows, double* __restrict__ score,
@@ -83,8 +91,12 @@ block_select_wide_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_
   pdl_wait();
   extern __shared__ __align__(16) uint8_t smem_b[];
   __shared__ BsSelScratch s_sel;
+  __shared__ double s_part[kMaxUnits];  // this CTA's column sums
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
 
-  const int bg = blockIdx.x;
+  const int bg = blockIdx.x / kCluster;
   const int b = bg / s.H_kv, g = bg % s.H_kv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int U = n_units, Uc = L::units_cap(U);
@@ -95,10 +107,13 @@ block_select_wide_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_
     if (tid == 0) flag_error(err, ERR_BAD_INDEX);
     nq = max_rows / s.G;
   }
-  const int R = nq * s.G;
-  T* sQ = reinterpret_cast<T*>(smem_b);                                   // [Rc][QP]
-  float* sK = reinterpret_cast<float*>(smem_b + L::q_bytes(max_rows));    // [Uc][KP]
-  double* sL = reinterpret_cast<double*>(smem_b + L::q_bytes(max_rows) + L::k_bytes(U));  // [Rc][Uc]
+  const int R_all = nq * s.G;
+  const int r_lo = rank * cta_rows(R_all);                 // this CTA's rows r_lo ..
+  const int R = max(0, min(R_all - r_lo, cta_rows(R_all)));  // .. r_lo + R - 1
+  const int cap = cta_rows(max_rows);
+  T* sQ = reinterpret_cast<T*>(smem_b);                              // [Rc][QP]
+  float* sK = reinterpret_cast<float*>(smem_b + L::q_bytes(cap));    // [Uc][KP]
+  double* sL = reinterpret_cast<double*>(smem_b + L::q_bytes(cap) + L::k_bytes(U));  // [Rc][Uc]
 
   constexpr int QCH = D * (int)sizeof(T) / 16;  // 16-byte chunks per query row
   constexpr int QE = 16 / (int)sizeof(T);       // elements per chunk
@@ -107,8 +122,8 @@ block_select_wide_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_
     const T* src = Q;
     bool ok = false;
     if (r < R) {
-      const int h = g * s.G + r / nq;
-      const int i = q_idx ? q_idx[(size_t)b * s.L_q + (r % nq)] : (r % nq);
+      const int h = g * s.G + (r_lo + r) / nq;
+      const int i = q_idx ? q_idx[(size_t)b * s.L_q + ((r_lo + r) % nq)] : ((r_lo + r) % nq);
       if (i >= 0 && i < s.L_q) {
         src = Q + (((size_t)b * s.H + h) * s.L_q + i) * D + ch * QE;
         ok = true;
@@ -191,16 +206,27 @@ block_select_wide_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_
   }
   __syncthreads();
 
-  // ---- column sums in row order, then the selection of the fused kernels
-  double my = 0.0;
-  if (tid < U) {
-    for (int r = 0; r < R; ++r) my += sL[(size_t)r * Uc + tid];
-    score[(size_t)bg * U + tid] = my;
+  // ---- column sums over this CTA's rows in row order; the first CTA adds the
+  // four CTAs' sums in CTA order and selects
+  if (tid < kMaxUnits) {
+    double my = 0.0;
+    if (tid < U)
+      for (int r = 0; r < R; ++r) my += sL[(size_t)r * Uc + tid];
+    s_part[tid] = my;
   }
+  cluster.sync();  // every CTA's sums are in its shared memory
+  double col = 0.0;
+  if (rank == 0 && tid < U) {
+#pragma unroll
+    for (int q = 0; q < kCluster; ++q) col += *cluster.map_shared_rank(&s_part[tid], q);
+    score[(size_t)bg * U + tid] = col;
+  }
+  cluster.sync();  // the others' shared memory stays until it has been read
+  if (rank != 0) return;
   const BsSorted srt =
-      U <= 32   ? bs_sort<32>(my, U, b, unit_size, sink_pos, n_sinks, s_sel, err)
-      : U <= 64 ? bs_sort<64>(my, U, b, unit_size, sink_pos, n_sinks, s_sel, err)
-                : bs_sort<128>(my, U, b, unit_size, sink_pos, n_sinks, s_sel, err);
+      U <= 32   ? bs_sort<32>(col, U, b, unit_size, sink_pos, n_sinks, s_sel, err)
+      : U <= 64 ? bs_sort<64>(col, U, b, unit_size, sink_pos, n_sinks, s_sel, err)
+                : bs_sort<128>(col, U, b, unit_size, sink_pos, n_sinks, s_sel, err);
   bs_write(srt, U, topK, bg, blk_idx, blk_cnt, max_sel, s_sel);
 }
 
@@ -210,11 +236,12 @@ bool block_select_wide_supported(const Shape& s, int rows, int n_units) {
       (size_t)bsw::kMaxCells)
     return false;
   if (s.d != 64 && s.d != 128) return false;
+  const int cap = bsw::cta_rows(rows);
   const size_t bytes =
-      s.dtype == 0 ? (s.d == 128 ? bsw::Layout<__nv_bfloat16, 128>::bytes(rows, n_units)
-                                 : bsw::Layout<__nv_bfloat16, 64>::bytes(rows, n_units))
-                   : (s.d == 128 ? bsw::Layout<float, 128>::bytes(rows, n_units)
-                                 : bsw::Layout<float, 64>::bytes(rows, n_units));
+      s.dtype == 0 ? (s.d == 128 ? bsw::Layout<__nv_bfloat16, 128>::bytes(cap, n_units)
+                                 : bsw::Layout<__nv_bfloat16, 64>::bytes(cap, n_units))
+                   : (s.d == 128 ? bsw::Layout<float, 128>::bytes(cap, n_units)
+                                 : bsw::Layout<float, 64>::bytes(cap, n_units));
   return bytes <= bsw::kSmemLimit;
 }
 
@@ -228,11 +255,12 @@ cudaError_t launch_block_select_wide(const Shape& s, const void* Q, const int32_
 #define DL_BSW(T, D_)                                                                           \
   {                                                                                            \
     auto k = block_select_wide_kernel<T, D_>;                                                  \
-    const size_t smem = bsw::Layout<T, D_>::bytes(rows, n_units);                              \
+    const size_t smem = bsw::Layout<T, D_>::bytes(bsw::cta_rows(rows), n_units);               \
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != \
         cudaSuccess)                                                                           \
       return e;                                                                                \
-    DL_LAUNCH(k, s.batch * s.H_kv, bsw::kThreads, smem, st, reinterpret_cast<const T*>(Q), q_idx, \
+    DL_LAUNCH(k, s.batch * s.H_kv * bsw::kCluster, bsw::kThreads, smem, st,                      \
+              reinterpret_cast<const T*>(Q), q_idx,                                            \
               q_cnt, Kbar, s, n_units, rows, score, unit_size, topK, sink_pos, n_sinks, blk_idx, \
               blk_cnt, max_sel, err);                                                          \
   }

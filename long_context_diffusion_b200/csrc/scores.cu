@@ -235,8 +235,9 @@ scores_tile_kernel(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
   }
 }
 
-// Grid (128-unit tiles, b*H_kv).  Warp per row: M = max of the tile
-// maxima, Z = sum_t z_t exp(m_t - M), and the factor of this CTA's tile
+// Grid (128-unit tiles, b*H_kv).  Thread per row (every row's statistics
+// loaded at once): M = max of the tile maxima, Z = sum_t z_t exp(m_t - M)
+// in tile order, and the factor of this CTA's tile
 // f = exp(m_tile - M) / Z (dynamic shared memory, G * L_q doubles; the
 // statistics are only read).
 // Then thread = (row group rg, unit): the sum over the rows rg, rg + 4, ...
@@ -258,17 +259,14 @@ scores_reduce_kernel(const int32_t* __restrict__ q_idx, const int32_t* __restric
   const int R_max = s.L_q * s.G;
   const int n_tiles = score_tiles(n_units);
   const size_t pitch = (size_t)n_tiles * kUT;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const double2* st = stats + (size_t)bg * R_max * n_tiles;
-  for (int r = warp; r < R; r += nw) {
+  for (int r = threadIdx.x; r < R; r += blockDim.x) {
     const double2* row = st + (size_t)r * n_tiles;
     double M = -INFINITY;
-    for (int t = lane; t < n_tiles; t += 32) M = fmax(M, row[t].x);
-    M = warp_max_d(M);
+    for (int t = 0; t < n_tiles; ++t) M = fmax(M, row[t].x);
     double Z = 0.0;
-    for (int t = lane; t < n_tiles; t += 32) Z += row[t].y * exp(row[t].x - M);
-    Z = warp_sum_d(Z);
-    if (lane == 0) s_f[r] = exp(row[tile].x - M) / Z;
+    for (int t = 0; t < n_tiles; ++t) Z += row[t].y * exp(row[t].x - M);
+    s_f[r] = exp(row[tile].x - M) / Z;
   }
   __syncthreads();
   const int rg = threadIdx.x / kUT, ul = threadIdx.x % kUT;
