@@ -330,8 +330,15 @@ block_select_fp64(const T* __restrict__ Q, const int32_t* __restrict__ q_idx,
   // ---- selection (as select_shfl_kernel, on the scores in shared memory)
   const int i = tid;  // key position in the network, kMaxUnits = kThreads
   if (i < n_units) score[(size_t)bg * n_units + i] = s_score[i];
-  BsSorted r = bs_sort(i < n_units ? s_score[i] : 0.0, n_units, b, unit_size, sink_pos, n_sinks,
-                       s_sel, err);
+  // a network as wide as the units (the 512-wide one for at most 32 units
+  // spends most of its stages on padding)
+  const double my = i < n_units ? s_score[i] : 0.0;
+  BsSorted r =
+      n_units <= 32    ? bs_sort<32>(my, n_units, b, unit_size, sink_pos, n_sinks, s_sel, err)
+      : n_units <= 64  ? bs_sort<64>(my, n_units, b, unit_size, sink_pos, n_sinks, s_sel, err)
+      : n_units <= 128 ? bs_sort<128>(my, n_units, b, unit_size, sink_pos, n_sinks, s_sel, err)
+      : n_units <= 256 ? bs_sort<256>(my, n_units, b, unit_size, sink_pos, n_sinks, s_sel, err)
+                       : bs_sort<512>(my, n_units, b, unit_size, sink_pos, n_sinks, s_sel, err);
   bs_write(r, n_units, topK, bg, blk_idx, blk_cnt, max_sel, s_sel);
 }
 
