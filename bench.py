@@ -411,15 +411,17 @@ def run_ours(args):
     torch.manual_seed(0)
     desc = dl.make_desc(wl_full.batch, wl_full.H, wl_full.H_kv, wl_full.d, wl_full.L_ctx,
                         wl_full.L_q, wl_full.B, wl_full.n_pages, wl_full.n_slots, dl.DL_BF16)
-    heads = args.shard == "heads"
+    heads = args.shard == "heads" or args.shard_sim > 1
     kv_heads, sink_group, wl = None, None, wl_full
     if heads:
         # this rank holds only its KV heads; the sink mass is all-reduced
         from long_context_diffusion_b200 import sharded
-        hs = sharded.HeadShard.of(desc, rank, world)
+        # --shard-sim W: rank 0's share of a head split over W GPUs, run alone
+        hs = (sharded.HeadShard.of(desc, 0, args.shard_sim) if args.shard_sim > 1
+              else sharded.HeadShard.of(desc, rank, world))
         desc, kv_heads = hs.desc, (hs.g0, hs.g1)
         wl = wl_full.replace(H=hs.desc.H, H_kv=hs.desc.H_kv)
-        if world > 1:
+        if world > 1 and args.shard_sim <= 1:
             import torch.distributed as dist
             sink_group = dist.group.WORLD
     t_gen = time.time()
@@ -660,7 +662,9 @@ def run_ours(args):
         "warmup": W, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "strong" if heads else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_of(wl_full, f"heads{world}" if heads else "replicas"),
+        "config": config_of(wl_full, (f"heads{args.shard_sim}, rank 0 alone: no all-reduce"
+                                      if args.shard_sim > 1 else f"heads{world}")
+                            if heads else "replicas"),
         "kv_tokens_per_s": kv_tokens * (1 if heads else world) / t_step,
         "kv_tokens_per_step": kv_tokens,
         "roofline": roof,
@@ -775,6 +779,10 @@ def main():
                     help="replicas: each GPU steps its own batch (weak scaling); heads: the "
                          "GPUs split the KV heads of one batch and all-reduce the sink mass "
                          "(strong scaling)")
+    ap.add_argument("--shard-sim", type=int, default=0,
+                    help="one GPU runs rank 0's share of a head split over this many GPUs, "
+                         "without the sink-mass all-reduce (the per-rank compute of a "
+                         "head-sharded step)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours" and args.layers == 32:
         args.warmup = 3
